@@ -1,0 +1,281 @@
+"""Multi-LoRA delta (SGMV / BGMV) for B200 -- Python binding of liblora_sgmv.so.
+
+The binding only marshals arguments (tensor pointers, sizes, the current CUDA
+stream) into the C ABI declared in include/lora_sgmv.h; every step of the
+computation runs in the library's kernels.  There is no fallback: if the
+shared library is missing or cannot be loaded, every call raises LoraError.
+
+Tensors: bf16 activations and pools on one CUDA device, int32 metadata, int64
+pool offsets, fp32 intermediate and per-adapter weights.  The workspace is a
+uint8 CUDA tensor; if none is given, one is taken from a per-device cache.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+__all__ = [
+    "LoraError", "load", "library_path", "lora_version", "lora_workspace_size", "lora_workspace_init",
+    "lora_get_error", "lora_route", "lora_bgmv", "lora_sgmv_shrink", "lora_sgmv_expand",
+    "lora_apply_multi", "make_pool_struct", "Workspace", "OP_BGMV", "OP_SGMV_SHRINK", "OP_SGMV_EXPAND",
+    "OP_APPLY_MULTI", "OP_ROUTE", "STATUS",
+]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIBNAME = "liblora_sgmv.so"
+
+OP_BGMV, OP_SGMV_SHRINK, OP_SGMV_EXPAND, OP_APPLY_MULTI, OP_ROUTE = range(5)
+STATUS = {0: "LORA_OK", 1: "LORA_ERR_INVALID_ARG", 2: "LORA_ERR_UNSUPPORTED", 4: "LORA_ERR_BAD_ADAPTER",
+          8: "LORA_ERR_BAD_SEGMENT", 16: "LORA_ERR_CUDA", 32: "LORA_ERR_WORKSPACE"}
+MAX_ADS_PER_REQ = 8
+
+
+class LoraError(RuntimeError):
+    def __init__(self, what: str, code: int = -1):
+        self.code = code
+        names = [v for k, v in STATUS.items() if k and (code > 0 and code & k)]
+        super().__init__(f"{what}: {'|'.join(names) or code}")
+
+
+class LoraPoolStruct(ctypes.Structure):
+    _fields_ = [("A", ctypes.c_void_p), ("B", ctypes.c_void_p), ("A_off", ctypes.c_void_p),
+                ("B_off", ctypes.c_void_p), ("rank", ctypes.c_void_p), ("A_elems", ctypes.c_int64),
+                ("B_elems", ctypes.c_int64), ("n_adapters", ctypes.c_int32), ("d_in", ctypes.c_int32),
+                ("d_out", ctypes.c_int32), ("max_rank", ctypes.c_int32)]
+
+
+_lib = None
+_lock = threading.Lock()
+
+
+def library_path() -> str:
+    return os.environ.get("LORA_SGMV_LIB", os.path.join(_PKG, _LIBNAME))
+
+
+def load():
+    """Load liblora_sgmv.so (built in-tree by adapter_gemv_sgmv_b200.build)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        path = library_path()
+        if not os.path.exists(path):
+            raise LoraError(f"{path} not found; build it with `python -m adapter_gemv_sgmv_b200.build`")
+        lib = ctypes.CDLL(path)
+        P, i32, i64, f32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+        PP = ctypes.POINTER(LoraPoolStruct)
+        lib.lora_version.restype = ctypes.c_char_p
+        lib.lora_version.argtypes = []
+        lib.lora_workspace_size.restype = sz
+        lib.lora_workspace_size.argtypes = [ctypes.c_int, i32, i32, i32, i32, i32, i32, i32]
+        lib.lora_workspace_init.restype = ctypes.c_int
+        lib.lora_workspace_init.argtypes = [P, P]
+        lib.lora_get_error.restype = ctypes.c_int
+        lib.lora_get_error.argtypes = [P, P]
+        lib.lora_route.restype = ctypes.c_int
+        lib.lora_route.argtypes = [P, i32, i32, P, P, P, P, P, sz, P]
+        lib.lora_bgmv.restype = ctypes.c_int
+        lib.lora_bgmv.argtypes = [P, i64, P, i64, PP, P, i32, f32, P, sz, P]
+        lib.lora_sgmv_shrink.restype = ctypes.c_int
+        lib.lora_sgmv_shrink.argtypes = [P, i64, P, i64, PP, P, P, i32, i32, P, sz, P]
+        lib.lora_sgmv_expand.restype = ctypes.c_int
+        lib.lora_sgmv_expand.argtypes = [P, i64, P, i64, PP, P, P, i32, i32, f32, P, sz, P]
+        lib.lora_apply_multi.restype = ctypes.c_int
+        lib.lora_apply_multi.argtypes = [P, i64, P, i64, PP, P, P, P, P, i32, i32, i32, P, sz, P]
+        _lib = lib
+    return _lib
+
+
+def lora_version() -> str:
+    return load().lora_version().decode()
+
+
+def lora_workspace_size(op: int, N: int, n_adapters: int, d_in: int, d_out: int, max_rank: int,
+                        n_items: int = 0, max_ads_per_req: int = 1) -> int:
+    return int(load().lora_workspace_size(op, N, n_adapters, d_in, d_out, max_rank, n_items,
+                                          max_ads_per_req))
+
+
+# ----------------------------------------------------------------------------
+# marshalling helpers
+# ----------------------------------------------------------------------------
+def _torch():
+    import torch
+    return torch
+
+
+def _stream_ptr(stream=None) -> int:
+    torch = _torch()
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream)
+
+
+def _ptr(t) -> int:
+    return 0 if t is None else int(t.data_ptr())
+
+
+def _check_dev(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise LoraError("tensors must live on a CUDA device", 1)
+
+
+def make_pool_struct(pool, max_rank: int | None = None) -> LoraPoolStruct:
+    """lora_pool from an object with A, B (bf16), A_off, B_off (int64), rank (int32), d_in, d_out."""
+    torch = _torch()
+    for name, dt in (("A", torch.bfloat16), ("B", torch.bfloat16), ("A_off", torch.int64),
+                     ("B_off", torch.int64), ("rank", torch.int32)):
+        t = getattr(pool, name)
+        if t.dtype != dt or not t.is_contiguous():
+            raise LoraError(f"pool.{name} must be a contiguous {dt} tensor", 1)
+    _check_dev(pool.A, pool.B, pool.A_off, pool.B_off, pool.rank)
+    if max_rank is None:
+        max_rank = int(getattr(pool, "max_rank"))
+    return LoraPoolStruct(_ptr(pool.A), _ptr(pool.B), _ptr(pool.A_off), _ptr(pool.B_off), _ptr(pool.rank),
+                          int(pool.A.numel()), int(pool.B.numel()), int(pool.rank.numel()),
+                          int(pool.d_in), int(pool.d_out), int(max_rank))
+
+
+class Workspace:
+    """A caller-owned workspace tensor, zeroed once (its error word starts clear)."""
+
+    def __init__(self, nbytes: int, device=None):
+        torch = _torch()
+        self.tensor = torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device or "cuda")
+
+    @property
+    def nbytes(self) -> int:
+        return int(self.tensor.numel())
+
+    def ptr(self) -> int:
+        return int(self.tensor.data_ptr())
+
+
+_ws_cache: dict = {}
+
+
+def _workspace(nbytes: int, device) -> Workspace:
+    torch = _torch()
+    dev = torch.device(device)
+    key = (dev.type, dev.index if dev.index is not None else torch.cuda.current_device())
+    ws = _ws_cache.get(key)
+    if ws is None or ws.nbytes < nbytes:
+        ws = Workspace(max(nbytes, 2 * (ws.nbytes if ws else 0)), device=dev)
+        _ws_cache[key] = ws
+    return ws
+
+
+def _rc(rc: int, what: str):
+    if rc != 0:
+        raise LoraError(what, rc)
+
+
+def _mat(t, d: int, name: str):
+    torch = _torch()
+    if t.dtype != torch.bfloat16 or t.dim() != 2 or t.stride(1) != 1 or t.shape[1] != d:
+        raise LoraError(f"{name} must be a 2-D bf16 tensor with {d} unit-stride columns", 1)
+    return t.stride(0)
+
+
+def lora_workspace_init(ws: Workspace, stream=None):
+    _rc(load().lora_workspace_init(ws.ptr(), _stream_ptr(stream)), "lora_workspace_init")
+
+
+def lora_get_error(ws: Workspace, stream=None) -> int:
+    """Device error bits of the workspace (cleared by the read); 0 if none."""
+    return int(load().lora_get_error(ws.ptr(), _stream_ptr(stream)))
+
+
+# ----------------------------------------------------------------------------
+# the entry points
+# ----------------------------------------------------------------------------
+def lora_route(ids, n_adapters: int, perm, seg_off, seg_ad, n_seg, ws: Workspace | None = None,
+               stream=None):
+    """Stable grouping of ids by adapter into caller tensors (see lora_route in the header)."""
+    lib = load()
+    _check_dev(ids, perm, seg_off, seg_ad, n_seg)
+    N = int(ids.numel())
+    need = lora_workspace_size(OP_ROUTE, N, n_adapters, 8, 8, 8)
+    ws = ws or _workspace(need, ids.device)
+    _rc(lib.lora_route(_ptr(ids), N, int(n_adapters), _ptr(perm), _ptr(seg_off), _ptr(seg_ad), _ptr(n_seg),
+                       ws.ptr(), ws.nbytes, _stream_ptr(stream)), "lora_route")
+    return ws
+
+
+def lora_bgmv(X, Y, pool, ids, scale: float, ws: Workspace | None = None, stream=None,
+              max_rank: int | None = None):
+    """Y[n] += scale * B[ids[n]] A[ids[n]] X[n] in place (ids[n] == -1: untouched)."""
+    lib = load()
+    _check_dev(X, Y, ids)
+    ps = make_pool_struct(pool, max_rank)
+    ldx = _mat(X, ps.d_in, "X")
+    ldy = _mat(Y, ps.d_out, "Y")
+    N = int(ids.numel())
+    need = lora_workspace_size(OP_BGMV, N, ps.n_adapters, ps.d_in, ps.d_out, ps.max_rank)
+    ws = ws or _workspace(need, X.device)
+    _rc(lib.lora_bgmv(_ptr(X), ldx, _ptr(Y), ldy, ctypes.byref(ps), _ptr(ids), N, float(scale),
+                      ws.ptr(), ws.nbytes, _stream_ptr(stream)), "lora_bgmv")
+    return ws
+
+
+def lora_sgmv_shrink(X, V, pool, seg_off, seg_ad, ws: Workspace | None = None, stream=None,
+                     max_rank: int | None = None):
+    """V[n, :rank[a]] = A[a] X[n] for rows of segment k (a = seg_ad[k]); V is fp32 [N, >= max_rank]."""
+    lib = load()
+    torch = _torch()
+    _check_dev(X, V, seg_off, seg_ad)
+    ps = make_pool_struct(pool, max_rank)
+    ldx = _mat(X, ps.d_in, "X")
+    if V.dtype != torch.float32 or V.dim() != 2 or V.stride(1) != 1:
+        raise LoraError("V must be a 2-D fp32 tensor with unit-stride columns", 1)
+    N = int(X.shape[0])
+    n_seg = int(seg_ad.numel())
+    need = lora_workspace_size(OP_SGMV_SHRINK, N, ps.n_adapters, ps.d_in, ps.d_out, ps.max_rank, n_seg)
+    ws = ws or _workspace(need, X.device)
+    _rc(lib.lora_sgmv_shrink(_ptr(X), ldx, _ptr(V), V.stride(0), ctypes.byref(ps), _ptr(seg_off),
+                             _ptr(seg_ad), n_seg, N, ws.ptr(), ws.nbytes, _stream_ptr(stream)),
+        "lora_sgmv_shrink")
+    return ws
+
+
+def lora_sgmv_expand(V, Y, pool, seg_off, seg_ad, scale: float, ws: Workspace | None = None,
+                     stream=None, max_rank: int | None = None):
+    """Y[n] += scale * B[a] V[n, :rank[a]] for rows of segment k (a = seg_ad[k])."""
+    lib = load()
+    torch = _torch()
+    _check_dev(V, Y, seg_off, seg_ad)
+    ps = make_pool_struct(pool, max_rank)
+    ldy = _mat(Y, ps.d_out, "Y")
+    if V.dtype != torch.float32 or V.dim() != 2 or V.stride(1) != 1:
+        raise LoraError("V must be a 2-D fp32 tensor with unit-stride columns", 1)
+    N = int(Y.shape[0])
+    n_seg = int(seg_ad.numel())
+    need = lora_workspace_size(OP_SGMV_EXPAND, N, ps.n_adapters, ps.d_in, ps.d_out, ps.max_rank, n_seg)
+    ws = ws or _workspace(need, Y.device)
+    _rc(lib.lora_sgmv_expand(_ptr(V), V.stride(0), _ptr(Y), ldy, ctypes.byref(ps), _ptr(seg_off),
+                             _ptr(seg_ad), n_seg, N, float(scale), ws.ptr(), ws.nbytes, _stream_ptr(stream)),
+        "lora_sgmv_expand")
+    return ws
+
+
+def lora_apply_multi(X, Y, pool, req_off, ad_off, ad_id, ad_scale, max_ads_per_req: int = 3,
+                     ws: Workspace | None = None, stream=None, max_rank: int | None = None):
+    """Y[n] += sum_p ad_scale[p] B[ad_id[p]] A[ad_id[p]] X[n] over request q's adapters."""
+    lib = load()
+    _check_dev(X, Y, req_off, ad_off, ad_id, ad_scale)
+    ps = make_pool_struct(pool, max_rank)
+    ldx = _mat(X, ps.d_in, "X")
+    ldy = _mat(Y, ps.d_out, "Y")
+    N = int(X.shape[0])
+    n_req = int(req_off.numel()) - 1
+    need = lora_workspace_size(OP_APPLY_MULTI, N, ps.n_adapters, ps.d_in, ps.d_out, ps.max_rank, n_req,
+                               max_ads_per_req)
+    ws = ws or _workspace(need, X.device)
+    _rc(lib.lora_apply_multi(_ptr(X), ldx, _ptr(Y), ldy, ctypes.byref(ps), _ptr(req_off), _ptr(ad_off),
+                             _ptr(ad_id), _ptr(ad_scale), n_req, N, int(max_ads_per_req), ws.ptr(),
+                             ws.nbytes, _stream_ptr(stream)), "lora_apply_multi")
+    return ws

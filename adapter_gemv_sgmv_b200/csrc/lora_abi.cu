@@ -1,0 +1,458 @@
+// The C ABI (include/lora_sgmv.h): host-side validation, workspace layout and
+// kernel launches.  No entry point allocates memory; every validation below
+// runs before the first CUDA call, so a rejected call touches no device.
+
+#include <string.h>
+
+#include "lora_internal.cuh"
+
+using namespace lora;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
+
+bool misaligned(const void *p, size_t a) { return ((uintptr_t)p) & (a - 1); }
+
+int32_t n_chunks_for(int op, int32_t d_in)
+{
+    return op == LORA_OP_BGMV ? (d_in + kBgmvChunk - 1) / kBgmvChunk : 1;
+}
+
+struct Layout {
+    size_t hdr, perm, seg_off, seg_ad, groups, V, total;
+    int32_t max_groups, n_chunks;
+};
+
+bool layout(int op, int32_t N, int32_t n_adapters, int32_t d_in, int32_t max_rank, int32_t n_items,
+            int32_t max_ads, Layout *L)
+{
+    if (N < 0 || n_adapters < 1 || n_adapters > LORA_MAX_ADAPTERS || d_in <= 0 || max_rank < 8 ||
+        max_rank > LORA_MAX_RANK)
+        return false;
+    const bool routed = op == LORA_OP_BGMV || op == LORA_OP_ROUTE;
+    if (!routed && n_items < 0)
+        return false;
+    if (op == LORA_OP_APPLY_MULTI && (max_ads < 1 || max_ads > LORA_MAX_ADS_PER_REQ))
+        return false;
+    const int64_t items = routed ? (int64_t)(N < n_adapters ? N : n_adapters) : n_items;
+    memset(L, 0, sizeof *L);
+    L->max_groups = (int32_t)((int64_t)N / kGroup + items + 1);
+    L->n_chunks = n_chunks_for(op, d_in);
+    size_t off = 0;
+    L->hdr = off;
+    off = align_up(off + sizeof(WsHeader));
+    L->perm = off;
+    off = align_up(off + (routed ? (size_t)N * 4 : 0));
+    L->seg_off = off;
+    off = align_up(off + (op == LORA_OP_BGMV ? (size_t)(items + 1) * 4 : 0));
+    L->seg_ad = off;
+    off = align_up(off + (op == LORA_OP_BGMV ? (size_t)items * 4 : 0));
+    L->groups = off;
+    off = align_up(off + (size_t)L->max_groups * sizeof(Group));
+    L->V = off;
+    size_t v = 0;
+    if (op == LORA_OP_BGMV)
+        v = (size_t)L->n_chunks * N * max_rank * 4;
+    else if (op == LORA_OP_APPLY_MULTI)
+        v = (size_t)N * max_ads * max_rank * 4;
+    off = align_up(off + v);
+    L->total = off;
+    return true;
+}
+
+lora_status check_pool(const lora_pool *p)
+{
+    if (!p || !p->A || !p->B || !p->A_off || !p->B_off || !p->rank)
+        return LORA_ERR_INVALID_ARG;
+    if (p->A_elems < 0 || p->B_elems < 0)
+        return LORA_ERR_INVALID_ARG;
+    if (p->n_adapters < 1 || p->n_adapters > LORA_MAX_ADAPTERS)
+        return LORA_ERR_UNSUPPORTED;
+    if (p->d_in <= 0 || p->d_out <= 0 || (p->d_in & 7) || (p->d_out & 7))
+        return LORA_ERR_UNSUPPORTED;
+    if (p->max_rank < 8 || p->max_rank > LORA_MAX_RANK || (p->max_rank & 7))
+        return LORA_ERR_UNSUPPORTED;
+    if (misaligned(p->A, 16) || misaligned(p->B, 16))
+        return LORA_ERR_UNSUPPORTED;
+    return LORA_OK;
+}
+
+lora_status check_mat(const void *M, int64_t ld, int32_t d, int32_t N)
+{
+    if (N > 0 && !M)
+        return LORA_ERR_INVALID_ARG;
+    if (ld < d)
+        return LORA_ERR_INVALID_ARG;
+    if ((ld & 7) || misaligned(M, 16))
+        return LORA_ERR_UNSUPPORTED;
+    return LORA_OK;
+}
+
+lora_status check_ws(void *ws, size_t ws_bytes, const Layout &L)
+{
+    if (!ws || misaligned(ws, kAlign) || ws_bytes < L.total)
+        return LORA_ERR_WORKSPACE;
+    return LORA_OK;
+}
+
+PoolDev pool_dev(const lora_pool *p)
+{
+    PoolDev d;
+    d.A = static_cast<const __nv_bfloat16 *>(p->A);
+    d.B = static_cast<const __nv_bfloat16 *>(p->B);
+    d.A_off = p->A_off;
+    d.B_off = p->B_off;
+    d.rank = p->rank;
+    d.A_elems = p->A_elems;
+    d.B_elems = p->B_elems;
+    d.n_adapters = p->n_adapters;
+    d.max_rank = p->max_rank;
+    d.d_in = p->d_in;
+    d.d_out = p->d_out;
+    return d;
+}
+
+template <class T>
+T *at(void *ws, size_t off) { return reinterpret_cast<T *>(static_cast<char *>(ws) + off); }
+
+#define LORA_TRY(x)                         \
+    do {                                    \
+        lora_status _s = (x);               \
+        if (_s != LORA_OK)                  \
+            return _s;                      \
+    } while (0)
+
+#define LORA_CUDA(x)                        \
+    do {                                    \
+        if ((x) != cudaSuccess)             \
+            return LORA_ERR_CUDA;           \
+    } while (0)
+
+}  // namespace
+
+extern "C" {
+
+const char *lora_version(void) { return "lora_sgmv_b200 0.1 (sm_100a)"; }
+
+size_t lora_workspace_size(int op, int32_t N, int32_t n_adapters, int32_t d_in, int32_t d_out,
+                           int32_t max_rank, int32_t n_items, int32_t max_ads_per_req)
+{
+    (void)d_out;
+    if (op < LORA_OP_BGMV || op > LORA_OP_ROUTE)
+        return 0;
+    Layout L;
+    if (!layout(op, N, n_adapters, d_in, max_rank, n_items, max_ads_per_req, &L))
+        return 0;
+    return L.total;
+}
+
+lora_status lora_workspace_init(void *ws, void *stream)
+{
+    if (!ws || misaligned(ws, kAlign))
+        return LORA_ERR_WORKSPACE;
+    LORA_CUDA(cudaMemsetAsync(ws, 0, sizeof(WsHeader), (cudaStream_t)stream));
+    return LORA_OK;
+}
+
+int lora_get_error(void *ws, void *stream)
+{
+    if (!ws || misaligned(ws, kAlign))
+        return LORA_ERR_WORKSPACE;
+    cudaStream_t s = (cudaStream_t)stream;
+    uint32_t err = 0;
+    if (cudaMemcpyAsync(&err, ws, sizeof err, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return LORA_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess)
+        return LORA_ERR_CUDA;
+    if (err) {
+        if (cudaMemsetAsync(ws, 0, sizeof err, s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess)
+            return LORA_ERR_CUDA;
+    }
+    return (int)err;
+}
+
+lora_status lora_route(const int32_t *ids, int32_t N, int32_t n_adapters, int32_t *perm,
+                       int32_t *seg_off, int32_t *seg_ad, int32_t *n_seg_out,
+                       void *ws, size_t ws_bytes, void *stream)
+{
+    if (N < 0 || (N > 0 && (!ids || !perm || !seg_ad)) || !seg_off || !n_seg_out)
+        return LORA_ERR_INVALID_ARG;
+    if (n_adapters < 1 || n_adapters > LORA_MAX_ADAPTERS)
+        return LORA_ERR_UNSUPPORTED;
+    Layout L;
+    if (!layout(LORA_OP_ROUTE, N, n_adapters, 8, 8, 0, 1, &L))
+        return LORA_ERR_INVALID_ARG;
+    LORA_TRY(check_ws(ws, ws_bytes, L));
+    PlanArgs pa = {};
+    pa.mode = kModeRoute;
+    pa.N = N;
+    pa.ids = ids;
+    pa.n_adapters = n_adapters;
+    pa.perm = perm;
+    pa.seg_off = seg_off;
+    pa.seg_ad = seg_ad;
+    pa.n_seg_out = n_seg_out;
+    pa.groups = at<Group>(ws, L.groups);
+    pa.max_groups = L.max_groups;
+    pa.hdr = at<WsHeader>(ws, L.hdr);
+    LORA_CUDA(launch_plan(pa, (cudaStream_t)stream));
+    return LORA_OK;
+}
+
+lora_status lora_bgmv(const void *X, int64_t ldx, void *Y, int64_t ldy, const lora_pool *pool,
+                      const int32_t *ids, int32_t N, float scale,
+                      void *ws, size_t ws_bytes, void *stream)
+{
+    LORA_TRY(check_pool(pool));
+    if (N < 0 || (N > 0 && !ids))
+        return LORA_ERR_INVALID_ARG;
+    LORA_TRY(check_mat(X, ldx, pool->d_in, N));
+    LORA_TRY(check_mat(Y, ldy, pool->d_out, N));
+    Layout L;
+    if (!layout(LORA_OP_BGMV, N, pool->n_adapters, pool->d_in, pool->max_rank, 0, 1, &L))
+        return LORA_ERR_INVALID_ARG;
+    LORA_TRY(check_ws(ws, ws_bytes, L));
+    if (N == 0)
+        return LORA_OK;
+    cudaStream_t s = (cudaStream_t)stream;
+    WsHeader *hdr = at<WsHeader>(ws, L.hdr);
+    int32_t *perm = at<int32_t>(ws, L.perm);
+    int32_t *seg_off = at<int32_t>(ws, L.seg_off);
+    int32_t *seg_ad = at<int32_t>(ws, L.seg_ad);
+    Group *groups = at<Group>(ws, L.groups);
+    float *V = at<float>(ws, L.V);
+
+    PlanArgs pa = {};
+    pa.mode = kModeRoute;
+    pa.N = N;
+    pa.ids = ids;
+    pa.n_adapters = pool->n_adapters;
+    pa.perm = perm;
+    pa.seg_off = seg_off;
+    pa.seg_ad = seg_ad;
+    pa.groups = groups;
+    pa.max_groups = L.max_groups;
+    pa.hdr = hdr;
+    LORA_CUDA(launch_plan(pa, s));
+
+    ShrinkArgs sa = {};
+    sa.X = static_cast<const __nv_bfloat16 *>(X);
+    sa.ldx = ldx;
+    sa.perm = perm;
+    sa.groups = groups;
+    sa.hdr = hdr;
+    sa.mode = kModeRoute;
+    sa.seg_ad = seg_ad;
+    sa.pool = pool_dev(pool);
+    sa.kc = kBgmvChunk;
+    sa.V = V;
+    sa.ldv = pool->max_rank;
+    sa.chunk_stride = (int64_t)N * pool->max_rank;
+    sa.slot_stride = 0;
+    sa.err = &hdr->err;
+    LORA_CUDA(launch_shrink(sa, L.max_groups, L.n_chunks, 1, s));
+
+    ExpandArgs ea = {};
+    ea.Y = static_cast<__nv_bfloat16 *>(Y);
+    ea.ldy = ldy;
+    ea.perm = perm;
+    ea.groups = groups;
+    ea.hdr = hdr;
+    ea.mode = kModeRoute;
+    ea.seg_ad = seg_ad;
+    ea.scale = scale;
+    ea.pool = pool_dev(pool);
+    ea.V = V;
+    ea.ldv = pool->max_rank;
+    ea.chunk_stride = (int64_t)N * pool->max_rank;
+    ea.n_chunks = L.n_chunks;
+    ea.slot_stride = 0;
+    ea.max_ads = 1;
+    ea.err = &hdr->err;
+    LORA_CUDA(launch_expand(ea, L.max_groups, s));
+    return LORA_OK;
+}
+
+lora_status lora_sgmv_shrink(const void *X, int64_t ldx, float *V, int64_t ldv,
+                             const lora_pool *pool, const int32_t *seg_off, const int32_t *seg_ad,
+                             int32_t n_seg, int32_t N, void *ws, size_t ws_bytes, void *stream)
+{
+    LORA_TRY(check_pool(pool));
+    if (N < 0 || n_seg < 0 || !seg_off || (n_seg > 0 && !seg_ad))
+        return LORA_ERR_INVALID_ARG;
+    LORA_TRY(check_mat(X, ldx, pool->d_in, N));
+    if ((N > 0 && !V) || ldv < pool->max_rank)
+        return LORA_ERR_INVALID_ARG;
+    Layout L;
+    if (!layout(LORA_OP_SGMV_SHRINK, N, pool->n_adapters, pool->d_in, pool->max_rank, n_seg, 1, &L))
+        return LORA_ERR_INVALID_ARG;
+    LORA_TRY(check_ws(ws, ws_bytes, L));
+    if (N == 0 || n_seg == 0)
+        return LORA_OK;
+    cudaStream_t s = (cudaStream_t)stream;
+    WsHeader *hdr = at<WsHeader>(ws, L.hdr);
+    Group *groups = at<Group>(ws, L.groups);
+
+    PlanArgs pa = {};
+    pa.mode = kModeSgmv;
+    pa.N = N;
+    pa.item_off = seg_off;
+    pa.n_items = n_seg;
+    pa.groups = groups;
+    pa.max_groups = L.max_groups;
+    pa.hdr = hdr;
+    LORA_CUDA(launch_plan(pa, s));
+
+    ShrinkArgs sa = {};
+    sa.X = static_cast<const __nv_bfloat16 *>(X);
+    sa.ldx = ldx;
+    sa.perm = nullptr;
+    sa.groups = groups;
+    sa.hdr = hdr;
+    sa.mode = kModeSgmv;
+    sa.seg_ad = seg_ad;
+    sa.pool = pool_dev(pool);
+    sa.kc = pool->d_in;
+    sa.V = V;
+    sa.ldv = ldv;
+    sa.chunk_stride = 0;
+    sa.slot_stride = 0;
+    sa.err = &hdr->err;
+    LORA_CUDA(launch_shrink(sa, L.max_groups, 1, 1, s));
+    return LORA_OK;
+}
+
+lora_status lora_sgmv_expand(const float *V, int64_t ldv, void *Y, int64_t ldy,
+                             const lora_pool *pool, const int32_t *seg_off, const int32_t *seg_ad,
+                             int32_t n_seg, int32_t N, float scale,
+                             void *ws, size_t ws_bytes, void *stream)
+{
+    LORA_TRY(check_pool(pool));
+    if (N < 0 || n_seg < 0 || !seg_off || (n_seg > 0 && !seg_ad))
+        return LORA_ERR_INVALID_ARG;
+    LORA_TRY(check_mat(Y, ldy, pool->d_out, N));
+    if ((N > 0 && !V) || ldv < pool->max_rank)
+        return LORA_ERR_INVALID_ARG;
+    Layout L;
+    if (!layout(LORA_OP_SGMV_EXPAND, N, pool->n_adapters, pool->d_in, pool->max_rank, n_seg, 1, &L))
+        return LORA_ERR_INVALID_ARG;
+    LORA_TRY(check_ws(ws, ws_bytes, L));
+    if (N == 0 || n_seg == 0)
+        return LORA_OK;
+    cudaStream_t s = (cudaStream_t)stream;
+    WsHeader *hdr = at<WsHeader>(ws, L.hdr);
+    Group *groups = at<Group>(ws, L.groups);
+
+    PlanArgs pa = {};
+    pa.mode = kModeSgmv;
+    pa.N = N;
+    pa.item_off = seg_off;
+    pa.n_items = n_seg;
+    pa.groups = groups;
+    pa.max_groups = L.max_groups;
+    pa.hdr = hdr;
+    LORA_CUDA(launch_plan(pa, s));
+
+    ExpandArgs ea = {};
+    ea.Y = static_cast<__nv_bfloat16 *>(Y);
+    ea.ldy = ldy;
+    ea.perm = nullptr;
+    ea.groups = groups;
+    ea.hdr = hdr;
+    ea.mode = kModeSgmv;
+    ea.seg_ad = seg_ad;
+    ea.scale = scale;
+    ea.pool = pool_dev(pool);
+    ea.V = V;
+    ea.ldv = ldv;
+    ea.chunk_stride = 0;
+    ea.n_chunks = 1;
+    ea.slot_stride = 0;
+    ea.max_ads = 1;
+    ea.err = &hdr->err;
+    LORA_CUDA(launch_expand(ea, L.max_groups, s));
+    return LORA_OK;
+}
+
+lora_status lora_apply_multi(const void *X, int64_t ldx, void *Y, int64_t ldy,
+                             const lora_pool *pool, const int32_t *req_off, const int32_t *ad_off,
+                             const int32_t *ad_id, const float *ad_scale, int32_t n_req, int32_t N,
+                             int32_t max_ads_per_req, void *ws, size_t ws_bytes, void *stream)
+{
+    LORA_TRY(check_pool(pool));
+    if (N < 0 || n_req < 0 || !req_off || !ad_off || (n_req > 0 && (!ad_id || !ad_scale)))
+        return LORA_ERR_INVALID_ARG;
+    if (max_ads_per_req < 1 || max_ads_per_req > LORA_MAX_ADS_PER_REQ)
+        return LORA_ERR_UNSUPPORTED;
+    LORA_TRY(check_mat(X, ldx, pool->d_in, N));
+    LORA_TRY(check_mat(Y, ldy, pool->d_out, N));
+    Layout L;
+    if (!layout(LORA_OP_APPLY_MULTI, N, pool->n_adapters, pool->d_in, pool->max_rank, n_req,
+                max_ads_per_req, &L))
+        return LORA_ERR_INVALID_ARG;
+    LORA_TRY(check_ws(ws, ws_bytes, L));
+    if (N == 0 || n_req == 0)
+        return LORA_OK;
+    cudaStream_t s = (cudaStream_t)stream;
+    WsHeader *hdr = at<WsHeader>(ws, L.hdr);
+    Group *groups = at<Group>(ws, L.groups);
+    float *V = at<float>(ws, L.V);
+    const int32_t ldv = max_ads_per_req * pool->max_rank;
+
+    PlanArgs pa = {};
+    pa.mode = kModeMulti;
+    pa.N = N;
+    pa.item_off = req_off;
+    pa.n_items = n_req;
+    pa.ad_off = ad_off;
+    pa.max_ads = max_ads_per_req;
+    pa.groups = groups;
+    pa.max_groups = L.max_groups;
+    pa.hdr = hdr;
+    LORA_CUDA(launch_plan(pa, s));
+
+    ShrinkArgs sa = {};
+    sa.X = static_cast<const __nv_bfloat16 *>(X);
+    sa.ldx = ldx;
+    sa.perm = nullptr;
+    sa.groups = groups;
+    sa.hdr = hdr;
+    sa.mode = kModeMulti;
+    sa.ad_off = ad_off;
+    sa.ad_id = ad_id;
+    sa.pool = pool_dev(pool);
+    sa.kc = pool->d_in;
+    sa.V = V;
+    sa.ldv = ldv;
+    sa.chunk_stride = 0;
+    sa.slot_stride = pool->max_rank;
+    sa.err = &hdr->err;
+    LORA_CUDA(launch_shrink(sa, L.max_groups, 1, max_ads_per_req, s));
+
+    ExpandArgs ea = {};
+    ea.Y = static_cast<__nv_bfloat16 *>(Y);
+    ea.ldy = ldy;
+    ea.perm = nullptr;
+    ea.groups = groups;
+    ea.hdr = hdr;
+    ea.mode = kModeMulti;
+    ea.ad_off = ad_off;
+    ea.ad_id = ad_id;
+    ea.ad_scale = ad_scale;
+    ea.scale = 1.0f;
+    ea.pool = pool_dev(pool);
+    ea.V = V;
+    ea.ldv = ldv;
+    ea.chunk_stride = 0;
+    ea.n_chunks = 1;
+    ea.slot_stride = pool->max_rank;
+    ea.max_ads = max_ads_per_req;
+    ea.err = &hdr->err;
+    LORA_CUDA(launch_expand(ea, L.max_groups, s));
+    return LORA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,120 @@
+// Internal declarations shared by the kernel files and the C-ABI layer.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "lora_sgmv.h"
+
+namespace lora {
+
+constexpr int kMaxRank = LORA_MAX_RANK;
+constexpr int kGroup = 8;            // tokens per work group in the CUDA-core kernels
+constexpr int kThreads = 128;        // threads per CTA of the CUDA-core kernels
+constexpr int kStageK = 1024;        // d_in elements of X staged in shared memory at a time
+constexpr int kExpandPerThread = 8;  // consecutive outputs per thread in the expand
+constexpr int kExpandTile = kThreads * kExpandPerThread;
+constexpr int kBgmvChunk = 512;      // split of d_in across CTAs in the decode shrink
+
+// Head of every workspace (256 bytes).
+struct WsHeader {
+    uint32_t err;       // device error bits (lora_status values), sticky until lora_get_error
+    int32_t n_seg;      // distinct adapters found by the grouping
+    int32_t n_groups;   // work groups written by the plan kernel
+    int32_t pad[61];
+};
+static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
+
+// A run of at most kGroup tokens that share one item (segment or request).
+// Tokens are positions p0 .. p0+cnt-1: row indices, or indices into perm.
+struct Group {
+    int32_t p0, cnt, item, pad;
+};
+
+enum Mode : int32_t { kModeRoute = 0, kModeSgmv = 1, kModeMulti = 2 };
+
+// ---------------------------------------------------------------- plan kernel
+struct PlanArgs {
+    int32_t mode;
+    int32_t N;
+    // route (decode): unsorted ids
+    const int32_t *ids;
+    int32_t n_adapters;
+    int32_t *perm;       // out [N]
+    int32_t *seg_off;    // out [min(N, n_adapters) + 1]
+    int32_t *seg_ad;     // out [min(N, n_adapters)]
+    int32_t *n_seg_out;  // optional out
+    // sgmv: caller's segments; multi: caller's requests
+    const int32_t *item_off;  // [n_items + 1]
+    int32_t n_items;
+    const int32_t *ad_off;    // multi only: adapter list bounds
+    int32_t max_ads;
+    // groups
+    Group *groups;
+    int32_t max_groups;
+    WsHeader *hdr;
+};
+
+// ----------------------------------------------------------- CUDA-core kernels
+// Device view of one projection's adapter pool.
+struct PoolDev {
+    const __nv_bfloat16 *A;
+    const __nv_bfloat16 *B;
+    const int64_t *A_off;
+    const int64_t *B_off;
+    const int32_t *rank;
+    int64_t A_elems, B_elems;
+    int32_t n_adapters, max_rank, d_in, d_out;
+};
+
+struct ShrinkArgs {
+    const __nv_bfloat16 *X;
+    int64_t ldx;
+    const int32_t *perm;   // nullable
+    const Group *groups;
+    const WsHeader *hdr;
+    int32_t mode;
+    const int32_t *seg_ad;   // route / sgmv: adapter of an item
+    const int32_t *ad_off;   // multi
+    const int32_t *ad_id;    // multi
+    PoolDev pool;
+    int32_t kc;
+    float *V;
+    int64_t ldv;           // elements between positions
+    int64_t chunk_stride;  // elements between split-K partial planes
+    int32_t slot_stride;   // elements between stacked adapters of one row
+    uint32_t *err;
+};
+
+struct ExpandArgs {
+    __nv_bfloat16 *Y;
+    int64_t ldy;
+    const int32_t *perm;
+    const Group *groups;
+    const WsHeader *hdr;
+    int32_t mode;
+    const int32_t *seg_ad;
+    const int32_t *ad_off;
+    const int32_t *ad_id;
+    const float *ad_scale;
+    float scale;
+    PoolDev pool;
+    const float *V;
+    int64_t ldv;
+    int64_t chunk_stride;
+    int32_t n_chunks;
+    int32_t slot_stride;
+    int32_t max_ads;
+    uint32_t *err;
+};
+
+// Launchers (return the CUDA error of the launch).
+cudaError_t launch_plan(const PlanArgs &a, cudaStream_t s);
+cudaError_t launch_shrink(const ShrinkArgs &a, int grid_groups, int n_chunks, int max_ads, cudaStream_t s);
+cudaError_t launch_expand(const ExpandArgs &a, int grid_groups, cudaStream_t s);
+
+// Shared memory the plan kernel needs for a route over n_adapters.
+size_t plan_smem_bytes(int32_t mode, int32_t n_adapters);
+
+}  // namespace lora

@@ -1,0 +1,206 @@
+/*
+ * lora_sgmv.h -- C ABI of the B200 (sm_100a) multi-LoRA delta library.
+ *
+ * What it computes.  "Serving several LoRAs, ControlNet and IP-Adapter"
+ * (AI-infra handbook), section "LoRA: merged or alongside": a LoRA adds a
+ * low-rank increment W' = W + B A to a weight (A is r x d, B is d x r, r from
+ * 8 to 128); served unmerged, each adapted layer adds x A^T B^T to x W^T.
+ * For a token row x[n] and an adapter a of rank r_a this library adds
+ *
+ *     y[n] += s * B[a] (A[a] x[n])          (shrink d_in -> r_a, expand r_a -> d_out)
+ *
+ * in place to y.  A mixed batch is grouped by adapter index, each group runs
+ * its own low-rank product inside one kernel, and the results land back in the
+ * original token order (same page, exercise 2's answer; the segmented
+ * gather-matrix-vector kernels of Punica, "Punica: multi-tenant LoRA serving",
+ * contribution 1).  Several LoRAs stacked on one request add their deltas
+ * (same page, table row "Stacking several LoRAs"); the weight s of each is a
+ * runtime scalar (same page: the LoRA weight may change every denoising step).
+ *
+ * Conventions common to every entry point
+ * ---------------------------------------
+ * - Types: activations and adapter weights are bf16 (passed as void*), the
+ *   rank-r intermediate V is fp32, all sums are accumulated in fp32 and each
+ *   output element of y is rounded to bf16 exactly once (round to nearest even).
+ * - Memory: every pointer except `pool` itself and the ones documented as host
+ *   pointers is DEVICE memory owned by the caller.  The library allocates
+ *   nothing and keeps no state between calls; all scratch lives in the
+ *   caller's workspace `ws` (see lora_workspace_size).
+ * - Layout: X is [N, d_in] row-major with leading dimension ldx (elements),
+ *   Y is [N, d_out] with ldy.  Adapter pool (lora_pool): adapter a's A is
+ *   [rank[a], d_in] row-major starting at element A_off[a] of pool->A, its B is
+ *   [d_out, rank[a]] row-major starting at element B_off[a] of pool->B; adapters
+ *   may have different ranks and are never padded to the maximum rank.
+ * - Requirements (checked on the host before anything is launched):
+ *   d_in and d_out multiples of 8; 8 <= max_rank <= 128, max_rank % 8 == 0;
+ *   1 <= n_adapters <= LORA_MAX_ADAPTERS; ldx >= d_in and ldy >= d_out, both
+ *   multiples of 8; X, Y, pool->A, pool->B 16-byte aligned; ws 256-byte aligned
+ *   and at least lora_workspace_size(...) bytes.  Violations return
+ *   LORA_ERR_INVALID_ARG or LORA_ERR_UNSUPPORTED and launch nothing.
+ * - Requirements checked on the device (the metadata lives in device memory):
+ *   adapter ids in [0, n_adapters) (or -1 = no adapter where stated),
+ *   rank[a] a multiple of 8 in [8, max_rank], A_off[a] and B_off[a]
+ *   non-negative multiples of 8 whose matrices end inside A_elems / B_elems,
+ *   segment/request offsets non-decreasing and
+ *   within [0, N].  A violation sets a bit in the workspace's error word and
+ *   skips the affected work (those rows keep their old y); it never traps.
+ *   Read and clear the word with lora_get_error.
+ * - Asynchrony: every compute entry point only enqueues kernels on `stream`
+ *   (a cudaStream_t; NULL = the legacy default stream) and returns.  Calls
+ *   that share one workspace must be ordered (same stream or events).
+ * - Thread safety: the library is stateless; concurrent calls with distinct
+ *   workspaces are safe.
+ */
+#ifndef LORA_SGMV_H
+#define LORA_SGMV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define LORA_API __attribute__((visibility("default")))
+#else
+#define LORA_API
+#endif
+
+#define LORA_MAX_RANK 128
+#define LORA_MAX_ADAPTERS 32768
+#define LORA_MAX_ADS_PER_REQ 8
+
+/* Status codes.  Host-side codes are returned directly; device-side codes are
+ * bits of the workspace error word returned by lora_get_error (OR-ed). */
+typedef enum {
+    LORA_OK = 0,
+    LORA_ERR_INVALID_ARG = 1,   /* host: null pointer, negative size, bad leading dimension */
+    LORA_ERR_UNSUPPORTED = 2,   /* host: shape, rank bound, alignment or limit not supported */
+    LORA_ERR_BAD_ADAPTER = 4,   /* device: adapter id, rank or pool offset out of range */
+    LORA_ERR_BAD_SEGMENT = 8,   /* device: segment/request offsets decreasing or outside [0, N] */
+    LORA_ERR_CUDA = 16,         /* host: a CUDA runtime call (launch, copy) failed */
+    LORA_ERR_WORKSPACE = 32     /* host: workspace null, misaligned or too small */
+} lora_status;
+
+/* One projection's resident adapter pool ("all LoRAs stay resident", same
+ * page, section "Placement").  The struct itself is a HOST object read during
+ * the call; every pointer in it is device memory. */
+typedef struct lora_pool {
+    const void *A;          /* bf16, packed A matrices                                  */
+    const void *B;          /* bf16, packed B matrices                                  */
+    const int64_t *A_off;   /* [n_adapters] element offset of adapter a's A in A        */
+    const int64_t *B_off;   /* [n_adapters] element offset of adapter a's B in B        */
+    const int32_t *rank;    /* [n_adapters] rank of adapter a                           */
+    int64_t A_elems;        /* elements in A: adapter a must satisfy A_off[a] + rank[a]*d_in <= A_elems */
+    int64_t B_elems;        /* elements in B: B_off[a] + d_out*rank[a] <= B_elems       */
+    int32_t n_adapters;
+    int32_t d_in;
+    int32_t d_out;
+    int32_t max_rank;       /* an upper bound of rank[a] over the pool (host-checked)   */
+} lora_pool;
+
+/* Operation codes for lora_workspace_size. */
+typedef enum {
+    LORA_OP_BGMV = 0,
+    LORA_OP_SGMV_SHRINK = 1,
+    LORA_OP_SGMV_EXPAND = 2,
+    LORA_OP_APPLY_MULTI = 3,
+    LORA_OP_ROUTE = 4
+} lora_op;
+
+/* Bytes of workspace `op` needs for N token rows.  n_items = n_seg for the
+ * SGMV ops, n_req for lora_apply_multi, ignored otherwise; max_ads_per_req is
+ * used by lora_apply_multi only.  Pure host function, no CUDA call.  Returns
+ * 0 for arguments the corresponding entry point would reject. */
+LORA_API size_t lora_workspace_size(int op, int32_t N, int32_t n_adapters, int32_t d_in, int32_t d_out,
+                           int32_t max_rank, int32_t n_items, int32_t max_ads_per_req);
+
+/* Clear the workspace's error word (cudaMemsetAsync of its 256-byte header on
+ * `stream`).  Call once on a fresh workspace. */
+LORA_API lora_status lora_workspace_init(void *ws, void *stream);
+
+/* Synchronise `stream`, read the workspace's error word, clear it, and return
+ * the device-side status bits (LORA_ERR_BAD_ADAPTER | LORA_ERR_BAD_SEGMENT) or
+ * LORA_OK; LORA_ERR_CUDA if the copy itself fails. */
+LORA_API int lora_get_error(void *ws, void *stream);
+
+/*
+ * lora_route -- group an unsorted batch by adapter index (exercise 2's answer
+ * on the handbook page: group the activations by LoRA index, then put the
+ * results back in the original order).  A stable counting sort:
+ *   perm[0..n_valid)   token indices grouped by adapter (ascending id), in
+ *                      original order within a group; tokens with id -1 are
+ *                      left out;
+ *   seg_ad[0..n_seg)   the distinct adapters present, ascending;
+ *   seg_off[0..n_seg]  group bounds in perm (seg_off[0] = 0);
+ *   *n_seg_out         n_seg (device int32).
+ * Capacities: perm >= N, seg_off >= min(N, n_adapters) + 1, seg_ad >=
+ * min(N, n_adapters).  ids: device int32 [N], -1 = no adapter; any other id
+ * outside [0, n_adapters) sets LORA_ERR_BAD_ADAPTER and is left out.
+ */
+LORA_API lora_status lora_route(const int32_t *ids, int32_t N, int32_t n_adapters, int32_t *perm,
+                       int32_t *seg_off, int32_t *seg_ad, int32_t *n_seg_out,
+                       void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * lora_bgmv -- decode: one token per request, each with its own adapter.
+ *   Y[n] += scale * B[ids[n]] A[ids[n]] X[n]   for ids[n] != -1
+ * ids: device int32 [N], unsorted, -1 = no adapter (row untouched).  The
+ * grouping (lora_route) runs inside the call, so every distinct adapter's A
+ * and B are streamed from HBM once however many tokens share it.
+ */
+LORA_API lora_status lora_bgmv(const void *X, int64_t ldx, void *Y, int64_t ldy, const lora_pool *pool,
+                      const int32_t *ids, int32_t N, float scale,
+                      void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * lora_sgmv_shrink -- prefill, tokens already grouped into segments:
+ *   V[n][j] = sum_i A[a][j][i] X[n][i],  j < rank[a],  a = seg_ad[k],
+ *   for seg_off[k] <= n < seg_off[k+1].
+ * V: device fp32 [N, ldv], ldv >= max_rank.  Entries j >= rank[a] and rows
+ * outside every segment are not written.  seg_off: device int32 [n_seg+1],
+ * non-decreasing, within [0, N]; empty segments are allowed.  seg_ad: device
+ * int32 [n_seg].
+ */
+LORA_API lora_status lora_sgmv_shrink(const void *X, int64_t ldx, float *V, int64_t ldv,
+                             const lora_pool *pool, const int32_t *seg_off, const int32_t *seg_ad,
+                             int32_t n_seg, int32_t N, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * lora_sgmv_expand -- the second half of the segmented product:
+ *   Y[n][o] += scale * sum_{j < rank[a]} B[a][o][j] V[n][j]
+ * for every row n inside segment k (a = seg_ad[k]); other rows untouched.
+ * Same segment arguments as lora_sgmv_shrink.
+ */
+LORA_API lora_status lora_sgmv_expand(const float *V, int64_t ldv, void *Y, int64_t ldy,
+                             const lora_pool *pool, const int32_t *seg_off, const int32_t *seg_ad,
+                             int32_t n_seg, int32_t N, float scale,
+                             void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * lora_apply_multi -- requests that stack several co-occurring adapters
+ * ("Co-occurrence Patterns of LoRA Adapters in Production Diffusion Model
+ * Inference Services", abstract: multi-adapter requests; handbook table row
+ * "Stacking several LoRAs"):
+ *   Y[n] += sum_{p in ad_off[q]..ad_off[q+1]} ad_scale[p] * B[ad_id[p]] A[ad_id[p]] X[n]
+ * for req_off[q] <= n < req_off[q+1].  All of a row's deltas are summed in
+ * fp32 before the single bf16 rounding of y.  req_off, ad_off: device int32
+ * [n_req+1], non-decreasing; ad_id: device int32; ad_scale: device fp32.
+ * A request may list at most max_ads_per_req (<= LORA_MAX_ADS_PER_REQ)
+ * adapters (device-checked: LORA_ERR_BAD_SEGMENT); an adapter listed twice
+ * counts twice.
+ */
+LORA_API lora_status lora_apply_multi(const void *X, int64_t ldx, void *Y, int64_t ldy,
+                             const lora_pool *pool, const int32_t *req_off, const int32_t *ad_off,
+                             const int32_t *ad_id, const float *ad_scale, int32_t n_req, int32_t N,
+                             int32_t max_ads_per_req, void *ws, size_t ws_bytes, void *stream);
+
+/* Library version string (host). */
+LORA_API const char *lora_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LORA_SGMV_H */

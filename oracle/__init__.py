@@ -257,3 +257,55 @@ def route(*a, **k):
 def widen_bf16(bits: np.ndarray) -> np.ndarray:
     """bf16 bit patterns -> float64, exactly (the same widening the C oracle applies)."""
     return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def round_bf16(x: np.ndarray) -> np.ndarray:
+    """Round float64 values to the nearest bf16 (ties to even), once, directly from
+    float64 (no intermediate float32 rounding); returned as float64.  This models the
+    single rounding of the bf16 output y that the library's interface fixes."""
+    x = np.asarray(x, dtype=np.float64)
+    mag = np.abs(x)
+    f = mag.astype(np.float32)                       # near |x|, at most half an fp32 ulp away
+    base = (f.view(np.uint32) & np.uint32(0xFFFF0000)).astype(np.int64)
+    best = None
+    best_err = None
+    for step in (-1, 0, 1):
+        c_bits = np.clip(base + step * 0x10000, 0, 0x7F7F0000).astype(np.uint32)
+        c = c_bits.view(np.float32).astype(np.float64)
+        err = np.abs(mag - c)
+        if best is None:
+            best, best_err, best_bits = c, err, c_bits
+            continue
+        even = ((c_bits >> np.uint32(16)) & np.uint32(1)) == 0
+        take = (err < best_err) | ((err == best_err) & even)
+        best = np.where(take, c, best)
+        best_err = np.where(take, err, best_err)
+        best_bits = np.where(take, c_bits, best_bits)
+    return np.copysign(best, x)
+
+
+def host_pool_subset(pool, used):
+    """Copy adapters `used` of a device-resident pool to a HostPool.
+
+    `pool` is any object with A, B (bf16 tensors), A_off_h, B_off_h, ranks_h (numpy),
+    d_in, d_out (the seeded workload pools).  Returns (HostPool, remap) with
+    remap[a] = index of adapter a in the subset (-1 if absent).  Marshalling only."""
+    import torch
+    used = np.asarray(sorted(set(int(a) for a in np.asarray(used).ravel())), dtype=np.int64)
+    remap = -np.ones(len(pool.ranks_h), dtype=np.int32)
+    remap[used] = np.arange(len(used), dtype=np.int32)
+    ranks = pool.ranks_h[used].astype(np.int32)
+    A_parts, B_parts = [], []
+    for a in used:
+        r = int(pool.ranks_h[a])
+        ao, bo = int(pool.A_off_h[a]), int(pool.B_off_h[a])
+        A_parts.append(pool.A[ao:ao + r * pool.d_in].detach().cpu().view(torch.int16).numpy().view(np.uint16))
+        B_parts.append(pool.B[bo:bo + r * pool.d_out].detach().cpu().view(torch.int16).numpy().view(np.uint16))
+    A_off = np.zeros(len(used), np.int64)
+    B_off = np.zeros(len(used), np.int64)
+    if len(used):
+        A_off[1:] = np.cumsum(ranks.astype(np.int64) * pool.d_in)[:-1]
+        B_off[1:] = np.cumsum(ranks.astype(np.int64) * pool.d_out)[:-1]
+    A = np.concatenate(A_parts) if A_parts else np.zeros(8, np.uint16)
+    B = np.concatenate(B_parts) if B_parts else np.zeros(8, np.uint16)
+    return HostPool(A=A, B=B, A_off=A_off, B_off=B_off, rank=ranks, d_in=pool.d_in, d_out=pool.d_out), remap

@@ -70,31 +70,56 @@ def bound(y_ref: np.ndarray) -> float:
     return 1e-2 * rms + 1e-3
 
 
-def compact_pool(hp_full_getter, ranks_h, A_off_h, B_off_h, d_in, d_out, used: np.ndarray):
-    """Build a HostPool holding only the adapters in `used` (ascending), fetching each
-    adapter's A and B via hp_full_getter(a) -> (A_bits, B_bits).  Returns (pool, remap)
-    where remap[a_full] = a_compact (-1 if absent)."""
-    used = np.asarray(sorted(set(int(a) for a in used)), dtype=np.int64)
-    remap = -np.ones(len(ranks_h), dtype=np.int32)
-    remap[used] = np.arange(len(used), dtype=np.int32)
-    ranks = ranks_h[used].astype(np.int32)
-    As, Bs = [], []
-    for a in used:
-        Aa, Ba = hp_full_getter(int(a))
-        As.append(Aa)
-        Bs.append(Ba)
-    A_off = np.zeros(len(used), np.int64)
-    B_off = np.zeros(len(used), np.int64)
-    if len(used):
-        A_off[1:] = np.cumsum(ranks.astype(np.int64) * d_in)[:-1]
-        B_off[1:] = np.cumsum(ranks.astype(np.int64) * d_out)[:-1]
-    A = np.concatenate(As) if As else np.zeros(8, np.uint16)
-    B = np.concatenate(Bs) if Bs else np.zeros(8, np.uint16)
-    return HostPool(A=A, B=B, A_off=A_off, B_off=B_off, rank=ranks, d_in=d_in, d_out=d_out), remap
-
-
 def compact_from_device_pool(pool, used):
     """Compact a workloads.Pool (possibly on the GPU, possibly GBs) to the adapters used."""
-    def get(a):
-        return to_host(pool.adapter_A(a)).reshape(-1), to_host(pool.adapter_B(a)).reshape(-1)
-    return compact_pool(get, pool.ranks_h, pool.A_off_h, pool.B_off_h, pool.d_in, pool.d_out, used)
+    from oracle import host_pool_subset
+    return host_pool_subset(pool, used)
+
+
+def check_parity(y_gpu_f64: np.ndarray, y_exact: np.ndarray, what: str):
+    """The parity bar: |y_gpu - round_bf16(y_exact)| <= 1e-2 * rms(y_ref) + 1e-3 elementwise,
+    rms taken over the whole compared output.  Returns (max_err, bound)."""
+    from oracle import round_bf16
+    ref = round_bf16(y_exact)
+    b = bound(ref)
+    err = np.abs(np.asarray(y_gpu_f64, np.float64) - ref)
+    m = float(err.max()) if err.size else 0.0
+    if not (m <= b):
+        i = np.unravel_index(int(np.argmax(err)), err.shape)
+        raise AssertionError(f"{what}: max |err| {m:.4g} > bound {b:.4g} at {i}: gpu "
+                             f"{y_gpu_f64[i]!r} ref {ref[i]!r} exact {y_exact[i]!r}")
+    return m, b
+
+
+def check_close_f32(v_gpu: np.ndarray, v_exact: np.ndarray, what: str):
+    """fp32 outputs (the shrink's V): |v - v_exact| <= 1e-2 * rms(v_exact) + 1e-3."""
+    b = bound(v_exact)
+    err = np.abs(np.asarray(v_gpu, np.float64) - v_exact)
+    m = float(err.max()) if err.size else 0.0
+    assert m <= b, f"{what}: max |err| {m:.4g} > bound {b:.4g}"
+    return m, b
+
+
+class DevPool:
+    """A HostPool copied to a device, shaped like workloads.Pool for the binding."""
+
+    def __init__(self, hp: HostPool, device="cuda", max_rank=None):
+        import torch
+        def bf(a):
+            a = np.ascontiguousarray(a, np.uint16)
+            if a.size == 0:
+                a = np.zeros(8, np.uint16)
+            return torch.from_numpy(a.view(np.int16).copy()).to(device).view(torch.bfloat16)
+        self.A = bf(hp.A)
+        self.B = bf(hp.B)
+        self.A_off = torch.tensor(hp.A_off, dtype=torch.int64, device=device)
+        self.B_off = torch.tensor(hp.B_off, dtype=torch.int64, device=device)
+        self.rank = torch.tensor(hp.rank, dtype=torch.int32, device=device)
+        self.d_in = hp.d_in
+        self.d_out = hp.d_out
+        self.max_rank = int(max_rank or max(8, int(hp.rank.max()) if hp.rank.size else 8))
+
+
+def dev_bf16(bits: np.ndarray, device="cuda"):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(bits, np.uint16).view(np.int16).copy()).to(device).view(torch.bfloat16)

@@ -1,0 +1,129 @@
+"""The C ABI without a GPU: the library loads, exports every entry point the
+header declares, sizes workspaces, and rejects bad arguments on the host.
+
+Every rejected call below carries at least one defect the host checks catch
+before the first CUDA call, and each case also passes a null workspace, so no
+case can reach a kernel launch even if the check under test were missing
+(the call would then fail on the workspace check instead, and the test would
+report the wrong status code).
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import adapter_gemv_sgmv_b200 as L
+from adapter_gemv_sgmv_b200 import build as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "lora_sgmv.h")
+
+OK, INVALID, UNSUPPORTED, WORKSPACE = 0, 1, 2, 32
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return L.load()
+
+
+def declared():
+    src = open(HEADER).read()
+    return re.findall(r"LORA_API\s+[\w\s\*]+?\b(lora_\w+)\s*\(", src)
+
+
+def test_header_declares_the_entry_points():
+    names = set(declared())
+    assert {"lora_bgmv", "lora_sgmv_shrink", "lora_sgmv_expand", "lora_apply_multi", "lora_route",
+            "lora_workspace_size", "lora_workspace_init", "lora_get_error", "lora_version"} <= names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    raw = ctypes.CDLL(L.library_path())
+    for name in declared():
+        assert hasattr(raw, name), name
+    assert "sm_100a" in L.lora_version()
+
+
+def test_workspace_size(lib):
+    s1 = L.lora_workspace_size(L.OP_BGMV, 256, 128, 4096, 4096, 16)
+    s2 = L.lora_workspace_size(L.OP_BGMV, 512, 128, 4096, 4096, 16)
+    assert 0 < s1 < s2 and s1 % 256 == 0
+    assert L.lora_workspace_size(L.OP_SGMV_SHRINK, 1000, 64, 4096, 14336, 64, n_items=16) > 0
+    assert L.lora_workspace_size(L.OP_APPLY_MULTI, 100, 8, 64, 64, 32, 4, 3) >= 100 * 3 * 32 * 4
+    # rejected shapes size to 0
+    assert L.lora_workspace_size(L.OP_BGMV, -1, 128, 4096, 4096, 16) == 0
+    assert L.lora_workspace_size(L.OP_BGMV, 4, 128, 4096, 4096, 256) == 0
+    assert L.lora_workspace_size(L.OP_APPLY_MULTI, 4, 8, 64, 64, 16, 1, 9) == 0
+    assert L.lora_workspace_size(99, 4, 8, 64, 64, 16) == 0
+
+
+FAKE = 0x10000          # a 256-byte-aligned address that is never dereferenced
+
+
+def _pool(**kw):
+    d = dict(A=FAKE, B=FAKE, A_off=FAKE, B_off=FAKE, rank=FAKE, A_elems=1 << 20, B_elems=1 << 20,
+             n_adapters=4, d_in=64, d_out=32, max_rank=16)
+    d.update(kw)
+    return L.LoraPoolStruct(**d)
+
+
+def _bgmv(lib, pool, X=FAKE, ldx=64, Y=FAKE, ldy=32, ids=FAKE, N=4, ws=None, ws_bytes=0):
+    return lib.lora_bgmv(X, ldx, Y, ldy, ctypes.byref(pool) if pool is not None else None, ids, N, 1.0,
+                         ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("case,want", [
+    (dict(pool=None), INVALID),
+    (dict(pool=_pool(A=0)), INVALID),
+    (dict(pool=_pool(rank=0)), INVALID),
+    (dict(pool=_pool(A_elems=-1)), INVALID),
+    (dict(pool=_pool(n_adapters=0)), UNSUPPORTED),
+    (dict(pool=_pool(n_adapters=40000)), UNSUPPORTED),
+    (dict(pool=_pool(d_in=60)), UNSUPPORTED),
+    (dict(pool=_pool(d_out=0)), UNSUPPORTED),
+    (dict(pool=_pool(max_rank=4)), UNSUPPORTED),
+    (dict(pool=_pool(max_rank=136)), UNSUPPORTED),
+    (dict(pool=_pool(max_rank=20)), UNSUPPORTED),
+    (dict(pool=_pool(A=FAKE + 8)), UNSUPPORTED),
+    (dict(ids=0), INVALID),
+    (dict(N=-1), INVALID),
+    (dict(X=0), INVALID),
+    (dict(ldx=32), INVALID),
+    (dict(ldx=68), UNSUPPORTED),
+    (dict(X=FAKE + 2), UNSUPPORTED),
+    (dict(Y=FAKE + 4), UNSUPPORTED),
+    (dict(ldy=16), INVALID),
+    (dict(ws=None), WORKSPACE),
+    (dict(ws=FAKE + 16, ws_bytes=1 << 30), WORKSPACE),
+    (dict(ws=FAKE, ws_bytes=256), WORKSPACE),
+])
+def test_bgmv_host_validation(lib, case, want):
+    kw = dict(pool=_pool())
+    kw.update(case)
+    assert _bgmv(lib, **kw) == want
+
+
+def test_other_entry_points_validate(lib):
+    p = ctypes.byref(_pool())
+    # sgmv shrink: ldv below max_rank / null segments / negative n_seg
+    assert lib.lora_sgmv_shrink(FAKE, 64, FAKE, 8, p, FAKE, FAKE, 2, 4, None, 0, None) == INVALID
+    assert lib.lora_sgmv_shrink(FAKE, 64, FAKE, 16, p, None, FAKE, 2, 4, None, 0, None) == INVALID
+    assert lib.lora_sgmv_shrink(FAKE, 64, FAKE, 16, p, FAKE, FAKE, -1, 4, None, 0, None) == INVALID
+    assert lib.lora_sgmv_shrink(FAKE, 64, FAKE, 16, p, FAKE, FAKE, 2, 4, None, 0, None) == WORKSPACE
+    # sgmv expand
+    assert lib.lora_sgmv_expand(FAKE, 8, FAKE, 32, p, FAKE, FAKE, 2, 4, 1.0, None, 0, None) == INVALID
+    assert lib.lora_sgmv_expand(FAKE, 16, FAKE + 2, 32, p, FAKE, FAKE, 2, 4, 1.0, None, 0, None) == UNSUPPORTED
+    assert lib.lora_sgmv_expand(FAKE, 16, FAKE, 32, p, FAKE, FAKE, 2, 4, 1.0, None, 0, None) == WORKSPACE
+    # multi: max_ads_per_req out of range, null adapter list
+    assert lib.lora_apply_multi(FAKE, 64, FAKE, 32, p, FAKE, FAKE, FAKE, FAKE, 2, 4, 9, None, 0, None) == UNSUPPORTED
+    assert lib.lora_apply_multi(FAKE, 64, FAKE, 32, p, FAKE, FAKE, None, FAKE, 2, 4, 3, None, 0, None) == INVALID
+    assert lib.lora_apply_multi(FAKE, 64, FAKE, 32, p, FAKE, FAKE, FAKE, FAKE, 2, 4, 3, None, 0, None) == WORKSPACE
+    # route
+    assert lib.lora_route(FAKE, 4, 0, FAKE, FAKE, FAKE, FAKE, None, 0, None) == UNSUPPORTED
+    assert lib.lora_route(None, 4, 8, FAKE, FAKE, FAKE, FAKE, None, 0, None) == INVALID
+    assert lib.lora_route(FAKE, 4, 8, FAKE, FAKE, FAKE, FAKE, None, 0, None) == WORKSPACE
+    # workspace helpers reject a null / misaligned workspace before touching CUDA
+    assert lib.lora_workspace_init(None, None) == WORKSPACE
+    assert lib.lora_get_error(FAKE + 8, None) == WORKSPACE
