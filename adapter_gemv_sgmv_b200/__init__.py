@@ -17,6 +17,7 @@ import threading
 
 __all__ = [
     "LoraError", "load", "library_path", "lora_version", "lora_workspace_size", "lora_workspace_init",
+    "lora_kernel_launches",
     "lora_get_error", "lora_route", "lora_bgmv", "lora_sgmv_shrink", "lora_sgmv_expand",
     "lora_apply_multi", "make_pool_struct", "Workspace", "OP_BGMV", "OP_SGMV_SHRINK", "OP_SGMV_EXPAND",
     "OP_APPLY_MULTI", "OP_ROUTE", "STATUS",
@@ -71,6 +72,8 @@ def load():
         lib.lora_version.argtypes = []
         lib.lora_workspace_size.restype = sz
         lib.lora_workspace_size.argtypes = [ctypes.c_int, i32, i32, i32, i32, i32, i32, i32]
+        lib.lora_kernel_launches.restype = ctypes.c_int
+        lib.lora_kernel_launches.argtypes = [ctypes.c_int, i32, i32, i32, i32]
         lib.lora_workspace_init.restype = ctypes.c_int
         lib.lora_workspace_init.argtypes = [P, P]
         lib.lora_get_error.restype = ctypes.c_int
@@ -97,6 +100,10 @@ def lora_workspace_size(op: int, N: int, n_adapters: int, d_in: int, d_out: int,
                         n_items: int = 0, max_ads_per_req: int = 1) -> int:
     return int(load().lora_workspace_size(op, N, n_adapters, d_in, d_out, max_rank, n_items,
                                           max_ads_per_req))
+
+
+def lora_kernel_launches(op: int, N: int, n_adapters: int, d_in: int, n_items: int = 0) -> int:
+    return int(load().lora_kernel_launches(op, N, n_adapters, d_in, n_items))
 
 
 # ----------------------------------------------------------------------------

@@ -2,11 +2,27 @@
 // kernel launches.  No entry point allocates memory; every validation below
 // runs before the first CUDA call, so a rejected call touches no device.
 
+#include <stdlib.h>
 #include <string.h>
 
 #include "lora_internal.cuh"
 
 using namespace lora;
+
+namespace lora {
+
+// Programmatic dependent launch for the single-launch decode kernel: on
+// unless LORA_SGMV_NO_PDL is set in the environment (read once).
+bool pdl_enabled()
+{
+    static const bool on = [] {
+        const char *v = getenv("LORA_SGMV_NO_PDL");
+        return !(v && v[0] && v[0] != '0');
+    }();
+    return on;
+}
+
+}  // namespace lora
 
 namespace {
 
@@ -149,6 +165,25 @@ size_t lora_workspace_size(int op, int32_t N, int32_t n_adapters, int32_t d_in, 
     return L.total;
 }
 
+int lora_kernel_launches(int op, int32_t N, int32_t n_adapters, int32_t d_in, int32_t n_items)
+{
+    if (N <= 0 || n_adapters < 1 || n_adapters > LORA_MAX_ADAPTERS || d_in <= 0)
+        return 0;
+    switch (op) {
+    case LORA_OP_BGMV:
+        return fused_bgmv_supported(N, n_adapters, d_in) ? 1 : 3;
+    case LORA_OP_SGMV_SHRINK:
+    case LORA_OP_SGMV_EXPAND:
+        return n_items > 0 ? 2 : 0;
+    case LORA_OP_APPLY_MULTI:
+        return n_items > 0 ? 3 : 0;
+    case LORA_OP_ROUTE:
+        return 1;
+    default:
+        return 0;
+    }
+}
+
 lora_status lora_workspace_init(void *ws, void *stream)
 {
     if (!ws || misaligned(ws, kAlign))
@@ -219,6 +254,22 @@ lora_status lora_bgmv(const void *X, int64_t ldx, void *Y, int64_t ldy, const lo
         return LORA_OK;
     cudaStream_t s = (cudaStream_t)stream;
     WsHeader *hdr = at<WsHeader>(ws, L.hdr);
+    if (fused_bgmv_supported(N, pool->n_adapters, pool->d_in)) {
+        FusedBgmvArgs fa = {};
+        fa.X = static_cast<const __nv_bfloat16 *>(X);
+        fa.ldx = ldx;
+        fa.Y = static_cast<__nv_bfloat16 *>(Y);
+        fa.ldy = ldy;
+        fa.ids = ids;
+        fa.N = N;
+        fa.pool = pool_dev(pool);
+        fa.scale = scale;
+        fa.Wk = fused_chunk(pool->d_in);
+        fa.Wo = fused_chunk(pool->d_out);
+        fa.err = &hdr->err;
+        LORA_CUDA(launch_bgmv_fused(fa, s, pdl_enabled()));
+        return LORA_OK;
+    }
     int32_t *perm = at<int32_t>(ws, L.perm);
     int32_t *seg_off = at<int32_t>(ws, L.seg_off);
     int32_t *seg_ad = at<int32_t>(ws, L.seg_ad);

@@ -109,6 +109,65 @@ struct ExpandArgs {
     uint32_t *err;
 };
 
+// --------------------------------------------------- fused decode (one launch)
+constexpr int kFT = 8;              // tokens per (adapter, group) item
+constexpr int kFThreads = 128;      // threads per CTA
+constexpr int kFWarps = kFThreads / 32;
+constexpr int kFC = 8;              // CTAs per cluster: d_in / d_out split in kFC chunks
+constexpr int kFMaxTokens = 8192;   // ids staged in shared memory
+constexpr int kFMaxAdapters = 8192; // per-adapter counters in shared memory
+constexpr int kFMaxChunk = 4096;    // d_in chunk per CTA (x rows staged in shared memory)
+constexpr size_t kFMaxSmem = 200 * 1024;
+
+struct FusedSmem {
+    size_t ids, cnt, xs, vpart, vsum, total;
+};
+
+__host__ __device__ inline size_t fused_align16(size_t x) { return (x + 15) & ~(size_t)15; }
+
+__host__ __device__ inline FusedSmem fused_smem_layout(int32_t N, int32_t n_adapters, int32_t Wk)
+{
+    FusedSmem L;
+    size_t off = 0;
+    L.ids = off;
+    off = fused_align16(off + 4 * (size_t)N);
+    L.cnt = off;
+    off = fused_align16(off + 4 * ((size_t)n_adapters + 1));
+    L.xs = off;
+    off = fused_align16(off + 4 * (size_t)(Wk / 8) * 68);   // fp32, kFT tokens x 8 columns + 4 pad per vector
+    L.vpart = off;
+    off = fused_align16(off + 4 * (size_t)kFT * kMaxRank);
+    L.vsum = off;
+    off = fused_align16(off + 4 * (size_t)kFT * kMaxRank);
+    L.total = off;
+    return L;
+}
+
+// Chunk of a dimension d per CTA of a cluster, rounded up to 8 elements.
+__host__ __device__ inline int32_t fused_chunk(int32_t d)
+{
+    const int32_t w = (d + kFC - 1) / kFC;
+    return (w + 7) & ~7;
+}
+
+struct FusedBgmvArgs {
+    const __nv_bfloat16 *X;
+    int64_t ldx;
+    __nv_bfloat16 *Y;
+    int64_t ldy;
+    const int32_t *ids;
+    int32_t N;
+    PoolDev pool;
+    float scale;
+    int32_t Wk, Wo;
+    uint32_t *err;
+};
+
+size_t fused_smem_bytes(int32_t N, int32_t n_adapters, int32_t Wk);
+bool fused_bgmv_supported(int32_t N, int32_t n_adapters, int32_t d_in);
+cudaError_t launch_bgmv_fused(const FusedBgmvArgs &a, cudaStream_t s, bool pdl);
+bool pdl_enabled();
+
 // Launchers (return the CUDA error of the launch).
 cudaError_t launch_plan(const PlanArgs &a, cudaStream_t s);
 cudaError_t launch_shrink(const ShrinkArgs &a, int grid_groups, int n_chunks, int max_ads, cudaStream_t s);

@@ -116,6 +116,11 @@ typedef enum {
 LORA_API size_t lora_workspace_size(int op, int32_t N, int32_t n_adapters, int32_t d_in, int32_t d_out,
                            int32_t max_rank, int32_t n_items, int32_t max_ads_per_req);
 
+/* Number of kernels one call of `op` launches for these sizes (pure host
+ * function): lets a caller budget a CUDA graph or count launches.  0 for
+ * arguments the entry point would reject or that launch nothing (N == 0). */
+LORA_API int lora_kernel_launches(int op, int32_t N, int32_t n_adapters, int32_t d_in, int32_t n_items);
+
 /* Clear the workspace's error word (cudaMemsetAsync of its 256-byte header on
  * `stream`).  Call once on a fresh workspace. */
 LORA_API lora_status lora_workspace_init(void *ws, void *stream);
@@ -147,8 +152,11 @@ LORA_API lora_status lora_route(const int32_t *ids, int32_t N, int32_t n_adapter
  * lora_bgmv -- decode: one token per request, each with its own adapter.
  *   Y[n] += scale * B[ids[n]] A[ids[n]] X[n]   for ids[n] != -1
  * ids: device int32 [N], unsorted, -1 = no adapter (row untouched).  The
- * grouping (lora_route) runs inside the call, so every distinct adapter's A
- * and B are streamed from HBM once however many tokens share it.
+ * grouping runs inside the call, so every distinct adapter's A and B are
+ * streamed from HBM once per group of up to 8 tokens sharing it.  For
+ * N <= 8192, n_adapters <= 8192 and d_in <= 32768 the whole call is one
+ * kernel launch (thread-block clusters of 8 CTAs; only the workspace's error
+ * word is used); larger calls take a three-kernel path through the workspace.
  */
 LORA_API lora_status lora_bgmv(const void *X, int64_t ldx, void *Y, int64_t ldy, const lora_pool *pool,
                       const int32_t *ids, int32_t N, float scale,

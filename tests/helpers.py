@@ -77,18 +77,27 @@ def compact_from_device_pool(pool, used):
 
 
 def check_parity(y_gpu_f64: np.ndarray, y_exact: np.ndarray, what: str):
-    """The parity bar: |y_gpu - round_bf16(y_exact)| <= 1e-2 * rms(y_ref) + 1e-3 elementwise,
-    rms taken over the whole compared output.  Returns (max_err, bound)."""
-    from oracle import round_bf16
-    ref = round_bf16(y_exact)
-    b = bound(ref)
-    err = np.abs(np.asarray(y_gpu_f64, np.float64) - ref)
-    m = float(err.max()) if err.size else 0.0
-    if not (m <= b):
-        i = np.unravel_index(int(np.argmax(err)), err.shape)
-        raise AssertionError(f"{what}: max |err| {m:.4g} > bound {b:.4g} at {i}: gpu "
-                             f"{y_gpu_f64[i]!r} ref {ref[i]!r} exact {y_exact[i]!r}")
-    return m, b
+    """The parity bar for a bf16 output, elementwise against the oracle's exact value:
+
+        |y_gpu - y_exact| <= 1e-2 * rms(y_exact) + 1e-3 + 2**-8 * |y_exact|
+
+    The first two terms are the stated tolerance for the arithmetic (bf16 inputs,
+    fp32 accumulation), rms over the whole compared output.  The last term is the
+    single rounding of the stored bf16 result: no bf16 value is closer than half
+    an ulp (<= 2**-8 |y|) to y_exact, and for |y| >= 4 rms that alone exceeds the
+    first two terms.  Returns (max excess ratio err/bound, rms)."""
+    y = np.asarray(y_gpu_f64, np.float64)
+    ex = np.asarray(y_exact, np.float64)
+    rms = float(np.sqrt(np.mean(ex * ex))) if ex.size else 0.0
+    b = 1e-2 * rms + 1e-3 + np.abs(ex) * 2.0 ** -8
+    err = np.abs(y - ex)
+    ratio = err / b
+    m = float(ratio.max()) if ratio.size else 0.0
+    if not (m <= 1.0):
+        i = np.unravel_index(int(np.argmax(ratio)), ratio.shape)
+        raise AssertionError(f"{what}: |err| {err[i]:.4g} > bound {b[i]:.4g} at {i}: gpu {y[i]!r} "
+                             f"exact {ex[i]!r} (rms {rms:.4g})")
+    return m, rms
 
 
 def check_close_f32(v_gpu: np.ndarray, v_exact: np.ndarray, what: str):

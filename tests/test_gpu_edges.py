@@ -199,3 +199,21 @@ def test_bad_segments_set_error_and_change_nothing():
                             torch.ones(5, device=DEV), max_ads_per_req=3)   # 5 adapters > 3
     assert L.lora_get_error(ws) & 8
     assert np.array_equal(_f64(Y), widen(Y0))
+
+
+@pytest.mark.parametrize("N,n_ad", [(9000, 40), (300, 9000)])
+def test_bgmv_three_kernel_path_beyond_fused_limits(N, n_ad):
+    """Batches beyond the single-launch kernel's shared-memory limits take the
+    plan/shrink/expand path; both must agree with the oracle."""
+    assert L.lora_kernel_launches(L.OP_BGMV, N, n_ad, 64) == 3
+    assert L.lora_kernel_launches(L.OP_BGMV, 256, 128, 4096) == 1
+    rng = np.random.default_rng(N)
+    ranks = rng.choice([8, 16, 32], n_ad)
+    hp = rand_host_pool(rng, ranks, 64, 48)
+    X = rand_x(rng, N, 64)
+    Y0 = rand_x(rng, N, 48)
+    ids = rng.integers(-1, n_ad, N).astype(np.int32)
+    Y = dev_bf16(Y0)
+    ws = L.lora_bgmv(dev_bf16(X), Y, DevPool(hp), _i32(ids), 0.5)
+    assert L.lora_get_error(ws) == 0
+    check_parity(_f64(Y), widen(Y0) + oracle.bgmv_delta(X, hp, ids, 0.5), f"3-kernel bgmv N={N}")

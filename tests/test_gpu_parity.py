@@ -1,11 +1,14 @@
 """GPU vs oracle parity on the five workloads, through the C ABI.
 
 Every call goes through liblora_sgmv.so via the ctypes binding; the oracle
-runs on the host on the same seeded inputs.  The bar (elementwise):
-    |y_gpu - round_bf16(y_exact)| <= 1e-2 * rms(y_ref) + 1e-3
-where y_exact is the oracle's fp64 result and round_bf16 the single rounding
-of the bf16 output; the shrink's fp32 V is held to the same bound against the
-oracle's fp64 V.  Full-size workloads are checked on sampled rows (segment
+runs on the host on the same seeded inputs.  The bar (elementwise, against
+the oracle's exact fp64 value y_exact):
+    |y_gpu - y_exact| <= 1e-2 * rms(y_exact) + 1e-3 + 2**-8 * |y_exact|
+(the stated tolerance plus the unit roundoff of the one bf16 rounding of the
+stored output; see helpers.check_parity).  The shrink's fp32 V is held to
+1e-2 * rms + 1e-3 against the oracle's fp64 V.  The decode path, which keeps
+the rank-r intermediate in fp32, must in addition give the correctly rounded
+bf16 of y_exact for at least 99% of the outputs.  Full-size workloads are checked on sampled rows (segment
 boundaries always included); the small ones on every row.
 """
 import numpy as np
@@ -87,7 +90,9 @@ def test_decode_bgmv_full(y0):
     _no_err(L.lora_bgmv(c.X, Y, c.pool, c.ids, c.scale))
     hp = host_pool(c.pool)
     y_exact = _f64(c.Y) + oracle.bgmv_delta(to_host(c.X), hp, c.ids_h, c.scale)
-    check_parity(_f64(Y), y_exact, f"decode bgmv y0={y0}")
+    got = _f64(Y)
+    check_parity(got, y_exact, f"decode bgmv y0={y0}")
+    assert np.mean(got == oracle.round_bf16(y_exact)) >= 0.99
 
 
 def test_prefill_sgmv_full_size_sampled_rows():
