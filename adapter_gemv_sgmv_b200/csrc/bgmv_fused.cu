@@ -4,30 +4,35 @@
 // The operation ("Serving several LoRAs, ControlNet and IP-Adapter", section
 // "LoRA: merged or alongside" and exercise 2's answer): y[n] += s B[a] A[a] x[n]
 // for a batch whose tokens carry their own adapter ids, grouped by adapter so
-// that each distinct adapter's A and B are streamed from HBM once (the
-// segmented gather matrix-vector product of "Punica: multi-tenant LoRA
+// that each distinct adapter's A and B are streamed from HBM once per group
+// (the segmented gather matrix-vector product of "Punica: multi-tenant LoRA
 // serving", contribution 1).
 //
 // Work layout on B200:
 // * every CTA rebuilds the grouping in shared memory (ids -> per-adapter
 //   counts -> exclusive scan of groups per adapter); item k is the k-th
-//   (adapter, group) pair in adapter order.  Clusters are persistent: the
-//   grid holds as many clusters as fit on the GPU at once, and cluster c
-//   takes items c, c + n_clusters, ...;
-// * the kFC CTAs of a cluster split d_in for the shrink: CTA c reduces its
-//   d_in chunk for all tokens of the item with 16-byte streaming loads of A,
-//   packed fp32x2 FMAs over token pairs and a warp reduce-scatter, leaving a
-//   partial rank-r vector per token in its shared memory;
-// * after a cluster barrier every CTA sums the kFC partials through
-//   distributed shared memory (fixed order, so the result is deterministic)
-//   and expands its own d_out chunk: B rows streamed with 16-byte loads, y
-//   read and written once, two outputs per thread per step;
-// * the item's B chunk and y rows are bulk-prefetched into L2 before the
-//   shrink, so their HBM latency hides behind the shrink and the exchange;
-// * programmatic dependent launch: the grouping and the L2 prefetch of the
-//   first item's adapter weights (immutable inputs) run before
-//   griddepcontrol.wait, i.e. while the previous kernel on the stream is
-//   still finishing; x, y and the workspace are touched only after it.
+//   (adapter, group of up to 16 tokens) pair in adapter order.  Clusters are
+//   persistent: the grid holds as many clusters as fit on the GPU at once and
+//   cluster c takes items c, c + n_clusters, ...
+// * an item is a 16-row tile of tokens, so both halves are tiny dense
+//   contractions done with warp-level tensor-core MMAs (m16n8k16, bf16 in,
+//   fp32 accumulate): with CUDA-core FMAs the instruction issue, not HBM,
+//   bounds decode.  Inside each 32-wide block of the reduction dimension the
+//   k order is permuted identically for both operands, so every thread's
+//   operand fragments are plain 16-byte global loads (no shared-memory
+//   staging, no bf16 unpacking): quad position q owns columns 8q..8q+7.
+// * shrink: the kFC CTAs of a cluster split d_in; CTA c computes its partial
+//   V_c = X_tile A[:, chunk]^T (16 tokens x r), its warps splitting the rank
+//   tiles and/or the chunk, reduced into shared memory;
+// * the cluster sums the kFC partials through distributed shared memory
+//   (fixed order: deterministic) and splits V into bf16 hi + lo parts, so the
+//   expand MMAs see V to ~16 significant bits instead of bf16's 8;
+// * expand: CTA c owns a d_out chunk; its warps walk 8-output tiles,
+//   Y_tile += s * (V_hi + V_lo) B[tile]^T, and update y in place;
+// * the item's y rows are bulk-prefetched into L2 early; the grouping and
+//   the first A fragments are loaded before griddepcontrol.wait
+//   (programmatic dependent launch), i.e. while the previous kernel on the
+//   stream is still finishing -- they only read immutable inputs.
 
 #include <cooperative_groups.h>
 
@@ -38,31 +43,25 @@
 namespace lora {
 namespace {
 
-constexpr int kXPad = 68;   // floats per 8-column vector of staged x (64 + 4: no bank conflicts)
-
+// Read-only 16-byte load that does not allocate in L1 (weights are used once
+// per CTA).  Not volatile: the compiler may batch independent loads.
 __device__ __forceinline__ uint4 ld_stream(const void *p)
 {
     uint4 r;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-                 : "l"(p));
+    asm("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+        : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+        : "l"(p));
     return r;
 }
 
-// element e (0..7) of 8 packed bf16 values, widened exactly to fp32
-__device__ __forceinline__ float bf_at(const uint4 &u, int e)
+// D += A * B for one m16n8k16 tile, bf16 inputs, fp32 accumulators.
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1)
 {
-    const uint32_t w = e < 2 ? u.x : e < 4 ? u.y : e < 6 ? u.z : u.w;
-    return (e & 1) ? __uint_as_float(w & 0xffff0000u) : __uint_as_float(w << 16);
-}
-
-// (d0, d1) += (a0, a1) * (b0, b1), one rounding per lane (Blackwell packed FMA)
-__device__ __forceinline__ void ffma2(float &d0, float &d1, float a0, float a1, float b0, float b1)
-{
-    asm("{\n\t.reg .b64 ra, rb, rc;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-        "mov.b64 rc, {%0, %1};\n\tfma.rn.f32x2 rc, ra, rb, rc;\n\tmov.b64 {%0, %1}, rc;\n\t}"
-        : "+f"(d0), "+f"(d1)
-        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+                 "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                 : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
 __device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes)
@@ -114,32 +113,15 @@ __device__ unsigned long long g_phase[65536 * 12];
     } while (0)
 #endif
 
-// Sum 32 per-lane values v[0..31] over the 32 lanes of a warp so that lane l
-// ends with the total of value l (31 shuffles instead of 32 x 5).
-__device__ __forceinline__ float reduce_scatter32(float (&v)[32], int lane)
-{
-#pragma unroll
-    for (int s = 16; s >= 1; s >>= 1) {
-        const bool upper = (lane & s) != 0;
-#pragma unroll
-        for (int i = 0; i < s; ++i) {
-            const float send = upper ? v[i] : v[i + s];
-            const float keep = upper ? v[i + s] : v[i];
-            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, s);
-        }
-    }
-    return v[0];
-}
-
 __device__ __forceinline__ bool adapter_ok(const PoolDev &P, int32_t a, int32_t *r_out, int64_t *aoff,
                                            int64_t *boff)
 {
     if (a < 0 || a >= P.n_adapters)
         return false;
     const int32_t r = P.rank[a];
+    const int64_t ao = P.A_off[a], bo = P.B_off[a];
     if (r < 8 || r > P.max_rank || (r & 7))
         return false;
-    const int64_t ao = P.A_off[a], bo = P.B_off[a];
     if (ao < 0 || (ao & 7) || ao + (int64_t)r * P.d_in > P.A_elems)
         return false;
     if (bo < 0 || (bo & 7) || bo + (int64_t)r * P.d_out > P.B_elems)
@@ -150,25 +132,155 @@ __device__ __forceinline__ bool adapter_ok(const PoolDev &P, int32_t a, int32_t 
     return true;
 }
 
-__global__ void __launch_bounds__(kFThreads, 6) k_bgmv_fused(FusedBgmvArgs p)
+// Shrink of one warp: NT rank tiles (8 ranks each, from rank tile nt0) over
+// the 32-column blocks [b0, b1) starting at column kb0; all A and x
+// fragments of a batch of BPB blocks are requested before any MMA runs.
+template <int NT>
+__device__ __forceinline__ void shrink_tiles(const __nv_bfloat16 *Aa, int d_in, int nt0, int kb0, int k1,
+                                             int b0, int b1, const __nv_bfloat16 *x0, const __nv_bfloat16 *x1,
+                                             bool row0, bool row1, int g, int qd, float (&acc)[4][4])
+{
+    constexpr int BPB = NT == 1 ? 4 : 2;   // blocks per batch (register budget)
+    for (int bb = b0; bb < b1; bb += BPB) {
+        uint4 aw[BPB][NT], xa[BPB], xb[BPB];
+#pragma unroll
+        for (int k = 0; k < BPB; ++k) {
+            const int col = kb0 + (bb + k) * 32 + qd * 8;
+            const bool ok = bb + k < b1 && col < k1;
+#pragma unroll
+            for (int i = 0; i < NT; ++i)
+                aw[k][i] = ok ? ld_stream(Aa + (int64_t)((nt0 + i) * 8 + g) * d_in + col) : make_uint4(0, 0, 0, 0);
+            xa[k] = (ok && row0) ? __ldg(reinterpret_cast<const uint4 *>(x0 + col)) : make_uint4(0, 0, 0, 0);
+            xb[k] = (ok && row1) ? __ldg(reinterpret_cast<const uint4 *>(x1 + col)) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int k = 0; k < BPB; ++k) {
+#pragma unroll
+            for (int i = 0; i < NT; ++i) {
+                // two k16 steps: low and high 8 bytes of each 16-byte fragment
+                mma16816(acc[i], xa[k].x, xb[k].x, xa[k].y, xb[k].y, aw[k][i].x, aw[k][i].y);
+                mma16816(acc[i], xa[k].z, xb[k].z, xa[k].w, xb[k].w, aw[k][i].z, aw[k][i].w);
+            }
+        }
+    }
+}
+
+// Expand of one warp over its output tiles ot = warp, warp + nw, ... < n_ot
+// (8 outputs each, from output o0): Y += s (V_hi + V_lo) B^T with NKB
+// 32-rank blocks; a batch's B fragments and y values are all requested
+// before its MMAs, and the V fragments are read from shared memory once.
+template <int NKB>
+__device__ __forceinline__ void expand_tiles(const __nv_bfloat16 *Ba, int r, int o0, int n_ot, int warp, int nw,
+                                             const __nv_bfloat16 *vhi, const __nv_bfloat16 *vlo, int g, int qd,
+                                             __nv_bfloat16 *y0row, __nv_bfloat16 *y1row, bool row0, bool row1,
+                                             float sc)
+{
+    constexpr int TPB = NKB == 1 ? 8 : NKB == 2 ? 4 : 2;   // tiles per batch
+    constexpr bool HOIST = NKB <= 2;                       // keep V fragments in registers
+    uint4 h0[HOIST ? NKB : 1], h1[HOIST ? NKB : 1], l0[HOIST ? NKB : 1], l1[HOIST ? NKB : 1];
+    if (HOIST) {
+#pragma unroll
+        for (int kb = 0; kb < (HOIST ? NKB : 1); ++kb) {
+            const int kc = kb * 32 + qd * 8;
+            h0[kb] = *reinterpret_cast<const uint4 *>(vhi + g * kVS + kc);
+            h1[kb] = *reinterpret_cast<const uint4 *>(vhi + (g + 8) * kVS + kc);
+            l0[kb] = *reinterpret_cast<const uint4 *>(vlo + g * kVS + kc);
+            l1[kb] = *reinterpret_cast<const uint4 *>(vlo + (g + 8) * kVS + kc);
+        }
+    }
+    for (int ot0 = warp; ot0 < n_ot; ot0 += TPB * nw) {
+        uint4 bw[TPB][NKB];
+        __nv_bfloat162 ya[TPB], yb[TPB];
+#pragma unroll
+        for (int t = 0; t < TPB; ++t) {
+            const int ot = ot0 + t * nw;
+            const bool ok = ot < n_ot;
+            const int ob = o0 + ot * 8;
+            const __nv_bfloat16 *brow = Ba + (int64_t)(ob + g) * r;
+#pragma unroll
+            for (int kb = 0; kb < NKB; ++kb) {
+                const int kc = kb * 32 + qd * 8;   // r and kc are multiples of 8
+                bw[t][kb] = (ok && kc < r) ? ld_stream(brow + kc) : make_uint4(0, 0, 0, 0);
+            }
+            const __nv_bfloat162 z = __floats2bfloat162_rn(0.f, 0.f);
+            ya[t] = (ok && row0) ? *reinterpret_cast<const __nv_bfloat162 *>(y0row + ob + 2 * qd) : z;
+            yb[t] = (ok && row1) ? *reinterpret_cast<const __nv_bfloat162 *>(y1row + ob + 2 * qd) : z;
+        }
+#pragma unroll
+        for (int t = 0; t < TPB; ++t) {
+            const int ot = ot0 + t * nw;
+            if (ot < n_ot) {
+                float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int kb = 0; kb < NKB; ++kb) {
+                    uint4 a0, a1, c0, c1;
+                    if (HOIST) {
+                        a0 = h0[HOIST ? kb : 0];
+                        a1 = h1[HOIST ? kb : 0];
+                        c0 = l0[HOIST ? kb : 0];
+                        c1 = l1[HOIST ? kb : 0];
+                    } else {
+                        const int kc = kb * 32 + qd * 8;
+                        a0 = *reinterpret_cast<const uint4 *>(vhi + g * kVS + kc);
+                        a1 = *reinterpret_cast<const uint4 *>(vhi + (g + 8) * kVS + kc);
+                        c0 = *reinterpret_cast<const uint4 *>(vlo + g * kVS + kc);
+                        c1 = *reinterpret_cast<const uint4 *>(vlo + (g + 8) * kVS + kc);
+                    }
+                    mma16816(d, a0.x, a1.x, a0.y, a1.y, bw[t][kb].x, bw[t][kb].y);
+                    mma16816(d, c0.x, c1.x, c0.y, c1.y, bw[t][kb].x, bw[t][kb].y);
+                    mma16816(d, a0.z, a1.z, a0.w, a1.w, bw[t][kb].z, bw[t][kb].w);
+                    mma16816(d, c0.z, c1.z, c0.w, c1.w, bw[t][kb].z, bw[t][kb].w);
+                }
+                // D fragment: tokens g, g+8; outputs ob + 2qd, ob + 2qd + 1
+                const int o = o0 + ot * 8 + 2 * qd;
+                if (row0) {
+                    const float2 y = __bfloat1622float2(ya[t]);
+                    *reinterpret_cast<__nv_bfloat162 *>(y0row + o) =
+                        __floats2bfloat162_rn(fmaf(sc, d[0], y.x), fmaf(sc, d[1], y.y));
+                }
+                if (row1) {
+                    const float2 y = __bfloat1622float2(yb[t]);
+                    *reinterpret_cast<__nv_bfloat162 *>(y1row + o) =
+                        __floats2bfloat162_rn(fmaf(sc, d[2], y.x), fmaf(sc, d[3], y.y));
+                }
+            }
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kFThreads, 5) k_bgmv_fused(FusedBgmvArgs p)
 {
     extern __shared__ __align__(16) unsigned char sm_raw[];
     const FusedSmem L = fused_smem_layout(p.N, p.pool.n_adapters, p.Wk);
     int32_t *ids_s = reinterpret_cast<int32_t *>(sm_raw + L.ids);
     int32_t *ipre = reinterpret_cast<int32_t *>(sm_raw + L.cnt);    // [n_ad + 1]
-    float *xs = reinterpret_cast<float *>(sm_raw + L.xs);           // [Wk/8][kXPad]
     float *vpart = reinterpret_cast<float *>(sm_raw + L.vpart);     // [kMaxRank][kFT], read by the cluster
-    float *vsum = reinterpret_cast<float *>(sm_raw + L.vsum);       // [kMaxRank][kFT]
+    // V split into bf16 hi and lo parts, token-major: [kFT][kVS] each
+    __nv_bfloat16 *vhi = reinterpret_cast<__nv_bfloat16 *>(sm_raw + L.vsum);
+    __nv_bfloat16 *vlo = vhi + kFT * kVS;
     __shared__ int32_t tok[kFT];
-    __shared__ int32_t s_ad, s_g, s_cnt, s_bad;
+    __shared__ int32_t s_ad, s_g, s_cnt, s_bad, s_r;
+    __shared__ int64_t s_aoff, s_boff;
     __shared__ int32_t sm_scan[kFWarps + 1];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int g = lane >> 2, qd = lane & 3;    // MMA fragment row group and quad position
     const uint32_t crank = cluster_ctarank();
     const int N = p.N, n_ad = p.pool.n_adapters;
     const int d_in = p.pool.d_in, d_out = p.pool.d_out;
     [[maybe_unused]] bool first = true;
     PHASE(0);
+
+    // pool metadata towards L2 while the ids arrive (whole 16-byte lines only)
+    if (tid == 0) {
+        const uint32_t rb = (uint32_t)(n_ad * 4) & ~15u, ob = (uint32_t)(n_ad * 8) & ~15u;
+        if (rb)
+            prefetch_l2(p.pool.rank, rb);
+        if (ob) {
+            prefetch_l2(p.pool.A_off, ob);
+            prefetch_l2(p.pool.B_off, ob);
+        }
+    }
 
     // ---- grouping, rebuilt by every CTA in shared memory (immutable inputs only)
     for (int a = tid; a < n_ad; a += kFThreads)
@@ -215,9 +327,9 @@ __global__ void __launch_bounds__(kFThreads, 6) k_bgmv_fused(FusedBgmvArgs p)
         __syncthreads();
         int run = sm_scan[warp] + incl - local;
         for (int a = b; a < e; ++a) {
-            const int g = (ipre[a] + kFT - 1) / kFT;
+            const int gr = (ipre[a] + kFT - 1) / kFT;
             ipre[a] = run;
-            run += g;
+            run += gr;
         }
         if (tid == 0)
             ipre[n_ad] = sm_scan[kFWarps];
@@ -226,41 +338,14 @@ __global__ void __launch_bounds__(kFThreads, 6) k_bgmv_fused(FusedBgmvArgs p)
     PHASE(2);
     const int n_items = ipre[n_ad];
     const int n_cl = (int)n_clusters_x();
-    int item = (int)cluster_id_x();
-
-    // prefetch the first item's adapter weights into L2 before waiting on the
-    // previous kernel: they are immutable inputs
     const int k0 = min(d_in, (int)crank * p.Wk), k1 = min(d_in, k0 + p.Wk);
     const int o0 = min(d_out, (int)crank * p.Wo), o1 = min(d_out, o0 + p.Wo);
-    if (item < n_items && warp == 1) {
-        int lo = 0, hi = n_ad;   // last adapter with ipre[a] <= item
-        while (hi - lo > 1) {
-            const int mid = (lo + hi) >> 1;
-            if (ipre[mid] <= item)
-                lo = mid;
-            else
-                hi = mid;
-        }
-        int32_t r;
-        int64_t aoff, boff;
-        if (adapter_ok(p.pool, lo, &r, &aoff, &boff)) {
-            if (k1 > k0)
-                for (int j = lane; j < r; j += 32)
-                    prefetch_l2(p.pool.A + aoff + (int64_t)j * d_in + k0, (uint32_t)((k1 - k0) * 2));
-            if (lane == 0 && o1 > o0)
-                prefetch_l2(p.pool.B + boff + (int64_t)o0 * r, (uint32_t)((o1 - o0) * r * 2));
-        }
-    }
-    pdl_trigger();
-    pdl_wait();   // from here on x, y and the workspace may be touched
-    PHASE(3);
-    if (s_bad && blockIdx.x == 0 && tid == 0)
-        atomicOr(p.err, (uint32_t)LORA_ERR_BAD_ADAPTER);
+    bool waited = false;
 
-    for (; item < n_items; item += n_cl) {
-        // ---- the item's adapter and tokens
+    for (int item = (int)cluster_id_x(); item < n_items; item += n_cl) {
+        // ---- the item's adapter, metadata and tokens (immutable inputs only)
         if (tid == 0) {
-            int lo = 0, hi = n_ad;
+            int lo = 0, hi = n_ad;   // last adapter with ipre[a] <= item
             while (hi - lo > 1) {
                 const int mid = (lo + hi) >> 1;
                 if (ipre[mid] <= item)
@@ -270,17 +355,31 @@ __global__ void __launch_bounds__(kFThreads, 6) k_bgmv_fused(FusedBgmvArgs p)
             }
             s_ad = lo;
             s_g = item - ipre[lo];
+            int32_t r = 0;
+            int64_t ao = 0, bo = 0;
+            s_r = adapter_ok(p.pool, lo, &r, &ao, &bo) ? r : 0;
+            s_aoff = ao;
+            s_boff = bo;
         }
         __syncthreads();
         const int a = s_ad;
-        int32_t r;
-        int64_t aoff, boff;
-        if (!adapter_ok(p.pool, a, &r, &aoff, &boff)) {
+        const int r = s_r;
+        if (r == 0) {
+            // the same decision in every CTA of the cluster
+            if (!waited) {
+                pdl_trigger();
+                pdl_wait();
+                waited = true;
+            }
             if (crank == 0 && tid == 0)
                 atomicOr(p.err, (uint32_t)LORA_ERR_BAD_ADAPTER);
             __syncthreads();
-            continue;   // the same decision in every CTA of the cluster
+            continue;
         }
+        const __nv_bfloat16 *Aa = p.pool.A + s_aoff;
+        const __nv_bfloat16 *Ba = p.pool.B + s_boff;
+        if (tid == 32 && o1 > o0)   // this CTA's B chunk towards L2 (immutable input)
+            prefetch_l2(Ba + (int64_t)o0 * r, (uint32_t)((o1 - o0) * r * 2));
         if (warp == 0) {
             const int lo = s_g * kFT;
             int seen = 0;
@@ -298,150 +397,144 @@ __global__ void __launch_bounds__(kFThreads, 6) k_bgmv_fused(FusedBgmvArgs p)
             if (lane == 0)
                 s_cnt = min(kFT, seen - lo);
         }
-        for (int e = tid; e < kFT * kMaxRank; e += kFThreads)
+        for (int e = tid; e < kMaxRank * kFT; e += kFThreads)
             vpart[e] = 0.f;
         __syncthreads();
-        PHASE(4);
         const int cnt = s_cnt;
-        const int npair = (cnt + 1) >> 1;
-        const __nv_bfloat16 *Bc = p.pool.B + boff + (int64_t)o0 * r;
+        // the tokens' y rows towards L2: a prefetch only fills L2, which is the
+        // point of coherence, so it cannot expose data older than a write that
+        // the previous kernel completes later
+        if (tid >= 32 && tid < 32 + cnt && o1 > o0)
+            prefetch_l2(p.Y + (int64_t)tok[tid - 32] * p.ldy + o0, (uint32_t)((o1 - o0) * 2));
+        PHASE(3);
 
-        // ---- expand operands towards L2: B chunk and the tokens' y rows
-        if (o1 > o0) {
-            if (tid == 0)
-                prefetch_l2(Bc, (uint32_t)((o1 - o0) * r * 2));
-            if (tid >= 32 && tid < 32 + cnt)
-                prefetch_l2(p.Y + (int64_t)tok[tid - 32] * p.ldy + o0, (uint32_t)((o1 - o0) * 2));
+        // ---- shrink work split: rank tiles of 8 in groups of up to 4 per warp;
+        // warps left over split this CTA's d_in chunk (32-column blocks)
+        const int n_nt = r >> 3;                        // rank tiles
+        const int ngrp = (n_nt + 3) >> 2;               // warp groups of <= 4 rank tiles
+        const int kparts = max(1, kFWarps / ngrp);
+        const int nblk = (k1 - k0 + 31) >> 5;           // 32-column blocks of the chunk
+        const int my_grp = warp / kparts, my_kp = warp - (warp / kparts) * kparts;
+        const int b0 = my_kp * nblk / kparts, b1 = (my_kp + 1) * nblk / kparts;
+
+        // ---- shrink: V_c[16 x r] = X_tile[16 x chunk] A[:, chunk]^T; this
+        // CTA's A rows are requested into L2 first (immutable input)
+        if (k1 > k0)
+            for (int j = tid; j < r; j += kFThreads)
+                prefetch_l2(Aa + (int64_t)j * d_in + k0, (uint32_t)((k1 - k0) * 2));
+        if (!waited) {
+            pdl_trigger();
+            pdl_wait();   // from here on x, y and the workspace may be touched
+            waited = true;
         }
-
-        // ---- stage x for this CTA's d_in chunk, token-contiguous, zero-padded to kFT tokens
-        const int nv = (k1 - k0) >> 3;
-        for (int idx = tid; idx < kFT * nv; idx += kFThreads) {
-            const int t = idx & (kFT - 1), v = idx >> 3;
-            uint4 u = make_uint4(0, 0, 0, 0);
-            if (t < cnt)
-                u = __ldg(reinterpret_cast<const uint4 *>(p.X + (int64_t)tok[t] * p.ldx + k0 + v * 8));
-            float *dst = xs + v * kXPad + t;
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-                dst[e * kFT] = bf_at(u, e);
-        }
-        __syncthreads();
-        PHASE(5);
-
-        // ---- shrink: a warp owns 4 rank rows and a share of the chunk's vectors
         {
-            const int n_rb = r >> 2;
-            const int kparts = max(1, kFWarps / n_rb);
-            const int units = n_rb * kparts;
-            const __nv_bfloat16 *Aa = p.pool.A + aoff + k0;
-            for (int u = warp; u < units; u += kFWarps) {
-                const int rb = u / kparts, kp = u - rb * kparts;
-                const int v0 = kp * nv / kparts, v1 = (kp + 1) * nv / kparts;
-                float acc[32];
+            const bool row0 = g < cnt, row1 = g + 8 < cnt;
+            const __nv_bfloat16 *x0 = p.X + (int64_t)(row0 ? tok[g] : 0) * p.ldx;
+            const __nv_bfloat16 *x1 = p.X + (int64_t)(row1 ? tok[g + 8] : 0) * p.ldx;
+            for (int grp = my_grp; grp < ngrp; grp += kFWarps / kparts) {
+                const int gt0 = grp * 4, nt = min(n_nt, gt0 + 4) - gt0;
+                float acc[4][4];
 #pragma unroll
-                for (int q = 0; q < 32; ++q)
-                    acc[q] = 0.f;
-                const __nv_bfloat16 *A0 = Aa + (int64_t)(rb * 4) * d_in;
-#pragma unroll 2
-                for (int v = v0 + lane; v < v1; v += 32) {
-                    uint4 ar[4];
+                for (int i = 0; i < 4; ++i)
 #pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        ar[i] = ld_stream(A0 + (int64_t)i * d_in + v * 8);
-                    const float4 *x4 = reinterpret_cast<const float4 *>(xs + v * kXPad);
+                    for (int j = 0; j < 4; ++j)
+                        acc[i][j] = 0.f;
+                switch (nt) {
+                case 1: shrink_tiles<1>(Aa, d_in, gt0, k0, k1, b0, b1, x0, x1, row0, row1, g, qd, acc); break;
+                case 2: shrink_tiles<2>(Aa, d_in, gt0, k0, k1, b0, b1, x0, x1, row0, row1, g, qd, acc); break;
+                case 3: shrink_tiles<3>(Aa, d_in, gt0, k0, k1, b0, b1, x0, x1, row0, row1, g, qd, acc); break;
+                default: shrink_tiles<4>(Aa, d_in, gt0, k0, k1, b0, b1, x0, x1, row0, row1, g, qd, acc); break;
+                }
+                // D fragment: rows (tokens) g, g+8; cols (ranks) 2qd, 2qd+1 of each rank tile
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const float4 xa = x4[e * 2], xb = x4[e * 2 + 1];
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const float av = bf_at(ar[i], e);
-                            ffma2(acc[i * 8 + 0], acc[i * 8 + 1], av, av, xa.x, xa.y);
-                            if (npair > 1)
-                                ffma2(acc[i * 8 + 2], acc[i * 8 + 3], av, av, xa.z, xa.w);
-                            if (npair > 2) {
-                                ffma2(acc[i * 8 + 4], acc[i * 8 + 5], av, av, xb.x, xb.y);
-                                ffma2(acc[i * 8 + 6], acc[i * 8 + 7], av, av, xb.z, xb.w);
-                            }
+                for (int i = 0; i < 4; ++i) {
+                    if (i < nt) {
+                        const int j = (gt0 + i) * 8 + 2 * qd;
+                        if (row0) {
+                            atomicAdd(&vpart[j * kFT + g], acc[i][0]);
+                            atomicAdd(&vpart[(j + 1) * kFT + g], acc[i][1]);
+                        }
+                        if (row1) {
+                            atomicAdd(&vpart[j * kFT + g + 8], acc[i][2]);
+                            atomicAdd(&vpart[(j + 1) * kFT + g + 8], acc[i][3]);
                         }
                     }
                 }
-                const float val = reduce_scatter32(acc, lane);
-                const int i = lane >> 3, t = lane & 7;
-                if (t < cnt)
-                    atomicAdd(&vpart[(rb * 4 + i) * kFT + t], val);
             }
         }
+        if (!waited) {
+            pdl_trigger();
+            pdl_wait();
+            waited = true;
+        }
+        if (s_bad && blockIdx.x == 0 && tid == 0 && item == (int)cluster_id_x())
+            atomicOr(p.err, (uint32_t)LORA_ERR_BAD_ADAPTER);
+        PHASE(4);
         __syncthreads();
-        PHASE(6);
+        PHASE(5);
 
-        // ---- exchange partials across the cluster (fixed summation order)
+        // ---- exchange partials across the cluster (fixed summation order),
+        // then split V into bf16 hi + lo, token-major, zero beyond cnt and r
         cluster_arrive();
         cluster_wait();
         {
             namespace cg = cooperative_groups;
             cg::cluster_group cl = cg::this_cluster();
-            for (int idx = tid; idx < kFT * r; idx += kFThreads) {
-                const int t = idx & (kFT - 1), j = idx >> 3;
-                float s = 0.f;
-                if (t < cnt) {
+            const int rp = (r + 31) & ~31;
+            // kFT * rp <= 16 * 128 elements: at most 16 per thread, 4 at a time
+            for (int base = 0; base < kFT * rp; base += 4 * kFThreads) {
+                float s[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                    for (int c = 0; c < kFC; ++c)
-                        s += cl.map_shared_rank(vpart, c)[j * kFT + t];
+                for (int c = 0; c < kFC; ++c) {
+                    const float *rv = cl.map_shared_rank(vpart, c);
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int idx = base + u * kFThreads + tid;
+                        const int t = idx & (kFT - 1), j = idx >> 4;
+                        if (idx < kFT * rp && t < cnt && j < r)
+                            s[u] += rv[j * kFT + t];
+                    }
                 }
-                vsum[j * kFT + t] = s;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int idx = base + u * kFThreads + tid;
+                    if (idx < kFT * rp) {
+                        const int t = idx & (kFT - 1), j = idx >> 4;
+                        const __nv_bfloat16 h = __float2bfloat16_rn(s[u]);
+                        vhi[t * kVS + j] = h;
+                        vlo[t * kVS + j] = __float2bfloat16_rn(s[u] - __bfloat162float(h));
+                    }
+                }
             }
         }
         cluster_arrive();   // our reads of the other CTAs' partials are done
         __syncthreads();
-        PHASE(7);
+        PHASE(6);
 
-        // ---- expand this CTA's d_out chunk, two outputs per thread per step
-        const float sc = p.scale;
-        for (int o = o0 + 2 * tid; o < o1; o += 2 * kFThreads) {
-            float c0[kFT], c1[kFT];
-#pragma unroll
-            for (int t = 0; t < kFT; ++t) {
-                c0[t] = 0.f;
-                c1[t] = 0.f;
-            }
-            const __nv_bfloat16 *b0 = Bc + (int64_t)(o - o0) * r;
-#pragma unroll 2
-            for (int jc = 0; jc < r; jc += 8) {
-                const uint4 u0 = ld_stream(b0 + jc), u1 = ld_stream(b0 + r + jc);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float f0 = bf_at(u0, e), f1 = bf_at(u1, e);
-                    const float4 *v4 = reinterpret_cast<const float4 *>(vsum + (jc + e) * kFT);
-                    const float4 va = v4[0], vb = v4[1];
-                    ffma2(c0[0], c0[1], f0, f0, va.x, va.y);
-                    ffma2(c1[0], c1[1], f1, f1, va.x, va.y);
-                    if (npair > 1) {
-                        ffma2(c0[2], c0[3], f0, f0, va.z, va.w);
-                        ffma2(c1[2], c1[3], f1, f1, va.z, va.w);
-                    }
-                    if (npair > 2) {
-                        ffma2(c0[4], c0[5], f0, f0, vb.x, vb.y);
-                        ffma2(c1[4], c1[5], f1, f1, vb.x, vb.y);
-                        ffma2(c0[6], c0[7], f0, f0, vb.z, vb.w);
-                        ffma2(c1[6], c1[7], f1, f1, vb.z, vb.w);
-                    }
-                }
-            }
-#pragma unroll
-            for (int t = 0; t < kFT; ++t) {
-                if (t < cnt) {
-                    __nv_bfloat162 *yp = reinterpret_cast<__nv_bfloat162 *>(p.Y + (int64_t)tok[t] * p.ldy + o);
-                    const float2 y = __bfloat1622float2(*yp);
-                    *yp = __floats2bfloat162_rn(y.x + sc * c0[t], y.y + sc * c1[t]);
-                }
+        // ---- expand: Y[16 x o-tile] += s (V_hi + V_lo) B[o-tile]^T, 8 outputs per tile
+        {
+            const int n_ot = (o1 - o0) >> 3;
+            const bool row0 = g < cnt, row1 = g + 8 < cnt;
+            __nv_bfloat16 *y0row = p.Y + (int64_t)(row0 ? tok[g] : 0) * p.ldy;
+            __nv_bfloat16 *y1row = p.Y + (int64_t)(row1 ? tok[g + 8] : 0) * p.ldy;
+            switch ((r + 31) >> 5) {
+            case 1: expand_tiles<1>(Ba, r, o0, n_ot, warp, kFWarps, vhi, vlo, g, qd, y0row, y1row, row0, row1, p.scale); break;
+            case 2: expand_tiles<2>(Ba, r, o0, n_ot, warp, kFWarps, vhi, vlo, g, qd, y0row, y1row, row0, row1, p.scale); break;
+            case 3: expand_tiles<3>(Ba, r, o0, n_ot, warp, kFWarps, vhi, vlo, g, qd, y0row, y1row, row0, row1, p.scale); break;
+            default: expand_tiles<4>(Ba, r, o0, n_ot, warp, kFWarps, vhi, vlo, g, qd, y0row, y1row, row0, row1, p.scale); break;
             }
         }
         __syncthreads();
-        PHASE(8);
+        PHASE(7);
         cluster_wait();     // no CTA reuses its partials while another may still read them
-        PHASE(9);
+        PHASE(8);
         first = false;
+    }
+    if (!waited) {
+        pdl_trigger();
+        pdl_wait();
+        if (s_bad && blockIdx.x == 0 && tid == 0)
+            atomicOr(p.err, (uint32_t)LORA_ERR_BAD_ADAPTER);
     }
 }
 

@@ -110,35 +110,35 @@ struct ExpandArgs {
 };
 
 // --------------------------------------------------- fused decode (one launch)
-constexpr int kFT = 8;              // tokens per (adapter, group) item
+constexpr int kFT = 16;             // tokens per (adapter, group) item = MMA tile rows
 constexpr int kFThreads = 128;      // threads per CTA
 constexpr int kFWarps = kFThreads / 32;
 constexpr int kFC = 8;              // CTAs per cluster: d_in / d_out split in kFC chunks
+constexpr int kVS = 160;            // bf16 row stride of the staged rank-r vectors (bank-conflict-free)
 constexpr int kFMaxTokens = 8192;   // ids staged in shared memory
-constexpr int kFMaxAdapters = 8192; // per-adapter counters in shared memory
-constexpr int kFMaxChunk = 4096;    // d_in chunk per CTA (x rows staged in shared memory)
+constexpr int kFMaxAdapters = 8192; // per-adapter group offsets in shared memory
+constexpr int kFMaxChunk = 1 << 20; // d_in chunk per CTA (nothing of it is staged)
 constexpr size_t kFMaxSmem = 200 * 1024;
 
 struct FusedSmem {
-    size_t ids, cnt, xs, vpart, vsum, total;
+    size_t ids, cnt, vpart, vsum, total;
 };
 
 __host__ __device__ inline size_t fused_align16(size_t x) { return (x + 15) & ~(size_t)15; }
 
 __host__ __device__ inline FusedSmem fused_smem_layout(int32_t N, int32_t n_adapters, int32_t Wk)
 {
+    (void)Wk;
     FusedSmem L;
     size_t off = 0;
     L.ids = off;
     off = fused_align16(off + 4 * (size_t)N);
     L.cnt = off;
     off = fused_align16(off + 4 * ((size_t)n_adapters + 1));
-    L.xs = off;
-    off = fused_align16(off + 4 * (size_t)(Wk / 8) * 68);   // fp32, kFT tokens x 8 columns + 4 pad per vector
     L.vpart = off;
-    off = fused_align16(off + 4 * (size_t)kFT * kMaxRank);
+    off = fused_align16(off + 4 * (size_t)kMaxRank * kFT);
     L.vsum = off;
-    off = fused_align16(off + 4 * (size_t)kFT * kMaxRank);
+    off = fused_align16(off + 2 * 2 * (size_t)kFT * kVS);   // bf16 hi and lo
     L.total = off;
     return L;
 }
