@@ -19,7 +19,7 @@ __all__ = [
     "LoraError", "load", "library_path", "lora_version", "lora_workspace_size", "lora_workspace_init",
     "lora_kernel_launches",
     "lora_get_error", "lora_route", "lora_bgmv", "lora_sgmv_shrink", "lora_sgmv_expand",
-    "lora_apply_multi", "make_pool_struct", "Workspace", "OP_BGMV", "OP_SGMV_SHRINK", "OP_SGMV_EXPAND",
+    "lora_apply_multi", "lora_apply_multi_static", "make_pool_struct", "Workspace", "OP_BGMV", "OP_SGMV_SHRINK", "OP_SGMV_EXPAND",
     "OP_APPLY_MULTI", "OP_ROUTE", "STATUS",
 ]
 
@@ -88,6 +88,8 @@ def load():
         lib.lora_sgmv_expand.argtypes = [P, i64, P, i64, PP, P, P, i32, i32, f32, P, sz, P]
         lib.lora_apply_multi.restype = ctypes.c_int
         lib.lora_apply_multi.argtypes = [P, i64, P, i64, PP, P, P, P, P, i32, i32, i32, P, sz, P]
+        lib.lora_apply_multi_static.restype = ctypes.c_int
+        lib.lora_apply_multi_static.argtypes = [P, i64, P, i64, PP, P, P, P, P, i32, i32, i32, P, P]
         _lib = lib
     return _lib
 
@@ -286,3 +288,23 @@ def lora_apply_multi(X, Y, pool, req_off, ad_off, ad_id, ad_scale, max_ads_per_r
                              _ptr(ad_id), _ptr(ad_scale), n_req, N, int(max_ads_per_req), ws.ptr(),
                              ws.nbytes, _stream_ptr(stream)), "lora_apply_multi")
     return ws
+
+
+def lora_apply_multi_static(X, Y, pool, req_off, ad_off, ad_id, ad_scale, max_ads_per_req: int = 3,
+                            err_out=None, stream=None, max_rank: int | None = None):
+    """lora_apply_multi without a workspace, for callers that cannot allocate device memory.
+
+    The scratch is a fixed array inside the library (see lora_apply_multi_static in the
+    header): calls must not overlap on the GPU, the first call on a device should come
+    before any stream capture, and too-large calls raise LoraError (LORA_ERR_WORKSPACE).
+    err_out: optional 1-element int32/uint32 CUDA tensor that receives the device status bits."""
+    lib = load()
+    _check_dev(X, Y, req_off, ad_off, ad_id, ad_scale, err_out)
+    ps = make_pool_struct(pool, max_rank)
+    ldx = _mat(X, ps.d_in, "X")
+    ldy = _mat(Y, ps.d_out, "Y")
+    N = int(X.shape[0])
+    n_req = int(req_off.numel()) - 1
+    _rc(lib.lora_apply_multi_static(_ptr(X), ldx, _ptr(Y), ldy, ctypes.byref(ps), _ptr(req_off), _ptr(ad_off),
+                                    _ptr(ad_id), _ptr(ad_scale), n_req, N, int(max_ads_per_req), _ptr(err_out),
+                                    _stream_ptr(stream)), "lora_apply_multi_static")

@@ -204,6 +204,40 @@ LORA_API lora_status lora_apply_multi(const void *X, int64_t ldx, void *Y, int64
                              const int32_t *ad_id, const float *ad_scale, int32_t n_req, int32_t N,
                              int32_t max_ads_per_req, void *ws, size_t ws_bytes, void *stream);
 
+/*
+ * lora_apply_multi_static -- lora_apply_multi without a caller workspace.
+ * The pages have no counterpart to this entry point; it exists for callers
+ * that cannot allocate device memory: code inside a region captured into a
+ * CUDA graph where allocation is not allowed, a process whose device memory
+ * belongs to another allocator, or a plugin that is handed only its input and
+ * output buffers.  It computes exactly what lora_apply_multi computes (same
+ * arguments minus the workspace, same kernels) and allocates nothing: no
+ * cudaMalloc, cudaFree or allocating library call.
+ *
+ * Its scratch (the work-group list, the error word and the fp32 rank-r
+ * intermediate, N * max_ads_per_req * max_rank floats plus a few KB) lives in
+ * one array of LORA_STATIC_SCRATCH_BYTES compiled into the library; every GPU
+ * that loads the library holds those bytes until the process exits.  Calls
+ * whose scratch would not fit return LORA_ERR_WORKSPACE and launch nothing
+ * (use lora_apply_multi with a workspace instead).
+ *
+ * All calls share the one array and it keeps the last call's contents: each
+ * call first clears the error word on `stream`, so calls that overlap on the
+ * GPU (different streams without ordering, or several host threads) race on
+ * the scratch and must not be issued.  The first call on a device looks up
+ * the array's device address (cudaGetSymbolAddress, once per device, with the
+ * device current); make that first call before any stream capture.
+ *
+ * err_out: optional device uint32; when non-null the call's device-side status
+ * bits (as lora_get_error would return them) are copied there on `stream`.
+ */
+#define LORA_STATIC_SCRATCH_BYTES (32u << 20)
+LORA_API lora_status lora_apply_multi_static(const void *X, int64_t ldx, void *Y, int64_t ldy,
+                                             const lora_pool *pool, const int32_t *req_off,
+                                             const int32_t *ad_off, const int32_t *ad_id,
+                                             const float *ad_scale, int32_t n_req, int32_t N,
+                                             int32_t max_ads_per_req, uint32_t *err_out, void *stream);
+
 /* Library version string (host). */
 LORA_API const char *lora_version(void);
 
