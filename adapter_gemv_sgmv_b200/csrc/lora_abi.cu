@@ -22,11 +22,30 @@ bool pdl_enabled()
     return on;
 }
 
+// Tensor-core (tcgen05) path for long segments / requests: on unless
+// LORA_SGMV_NO_TC is set in the environment (read once).
+bool tc_enabled()
+{
+    static const bool on = [] {
+        const char *v = getenv("LORA_SGMV_NO_TC");
+        return !(v && v[0] && v[0] != '0');
+    }();
+    return on;
+}
+
 }  // namespace lora
 
 namespace {
 
 constexpr size_t kAlign = 256;
+
+// Items long enough on average for 128-row tensor-core tiles to pay off.
+bool long_items(int32_t N, int32_t n_items)
+{
+    return tc_enabled() && N >= kTcGroup && (int64_t)N >= 64LL * (n_items > 0 ? n_items : 1);
+}
+
+bool aligned_v(const void *V, int64_t ldv) { return ((uintptr_t)V & 15) == 0 && (ldv & 3) == 0; }
 
 size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
 
@@ -232,6 +251,7 @@ lora_status lora_route(const int32_t *ids, int32_t N, int32_t n_adapters, int32_
     pa.n_seg_out = n_seg_out;
     pa.groups = at<Group>(ws, L.groups);
     pa.max_groups = L.max_groups;
+    pa.group = kGroup;
     pa.hdr = at<WsHeader>(ws, L.hdr);
     LORA_CUDA(launch_plan(pa, (cudaStream_t)stream));
     return LORA_OK;
@@ -286,6 +306,7 @@ lora_status lora_bgmv(const void *X, int64_t ldx, void *Y, int64_t ldy, const lo
     pa.seg_ad = seg_ad;
     pa.groups = groups;
     pa.max_groups = L.max_groups;
+    pa.group = kGroup;
     pa.hdr = hdr;
     LORA_CUDA(launch_plan(pa, s));
 
@@ -347,6 +368,35 @@ lora_status lora_sgmv_shrink(const void *X, int64_t ldx, float *V, int64_t ldv,
     WsHeader *hdr = at<WsHeader>(ws, L.hdr);
     Group *groups = at<Group>(ws, L.groups);
 
+    if (long_items(N, n_seg) && aligned_v(V, ldv)) {
+        TcArgs ta = {};
+        if (tc_encode_x(ta, X, N, pool->d_in, ldx)) {
+            PlanArgs pa = {};
+            pa.mode = kModeSgmv;
+            pa.N = N;
+            pa.item_off = seg_off;
+            pa.n_items = n_seg;
+            pa.groups = groups;
+            pa.max_groups = L.max_groups;
+            pa.group = kTcGroup;
+            pa.hdr = hdr;
+            LORA_CUDA(launch_plan(pa, s));
+            ta.mode = kModeSgmv;
+            ta.groups = groups;
+            ta.hdr = hdr;
+            ta.seg_ad = seg_ad;
+            ta.max_ads = 1;
+            ta.scale = 1.0f;
+            ta.pool = pool_dev(pool);
+            ta.V = V;
+            ta.ldv = ldv;
+            ta.slot_stride = 0;
+            ta.err = &hdr->err;
+            LORA_CUDA(launch_tc_shrink(ta, N / kTcGroup + n_seg + 1, s));
+            return LORA_OK;
+        }
+    }
+
     PlanArgs pa = {};
     pa.mode = kModeSgmv;
     pa.N = N;
@@ -354,6 +404,7 @@ lora_status lora_sgmv_shrink(const void *X, int64_t ldx, float *V, int64_t ldv,
     pa.n_items = n_seg;
     pa.groups = groups;
     pa.max_groups = L.max_groups;
+    pa.group = kGroup;
     pa.hdr = hdr;
     LORA_CUDA(launch_plan(pa, s));
 
@@ -397,6 +448,37 @@ lora_status lora_sgmv_expand(const float *V, int64_t ldv, void *Y, int64_t ldy,
     WsHeader *hdr = at<WsHeader>(ws, L.hdr);
     Group *groups = at<Group>(ws, L.groups);
 
+    if (long_items(N, n_seg) && aligned_v(V, ldv)) {
+        TcArgs ta = {};
+        if (tc_encode_y(ta, Y, N, pool->d_out, ldy)) {
+            PlanArgs pa = {};
+            pa.mode = kModeSgmv;
+            pa.N = N;
+            pa.item_off = seg_off;
+            pa.n_items = n_seg;
+            pa.groups = groups;
+            pa.max_groups = L.max_groups;
+            pa.group = kTcGroup;
+            pa.hdr = hdr;
+            LORA_CUDA(launch_plan(pa, s));
+            ta.mode = kModeSgmv;
+            ta.groups = groups;
+            ta.hdr = hdr;
+            ta.seg_ad = seg_ad;
+            ta.max_ads = 1;
+            ta.scale = scale;
+            ta.pool = pool_dev(pool);
+            ta.V = const_cast<float *>(V);
+            ta.ldv = ldv;
+            ta.slot_stride = 0;
+            ta.Y = static_cast<__nv_bfloat16 *>(Y);
+            ta.ldy = ldy;
+            ta.err = &hdr->err;
+            LORA_CUDA(launch_tc_expand(ta, s));
+            return LORA_OK;
+        }
+    }
+
     PlanArgs pa = {};
     pa.mode = kModeSgmv;
     pa.N = N;
@@ -404,6 +486,7 @@ lora_status lora_sgmv_expand(const float *V, int64_t ldv, void *Y, int64_t ldy,
     pa.n_items = n_seg;
     pa.groups = groups;
     pa.max_groups = L.max_groups;
+    pa.group = kGroup;
     pa.hdr = hdr;
     LORA_CUDA(launch_plan(pa, s));
 
@@ -453,6 +536,42 @@ lora_status lora_apply_multi(const void *X, int64_t ldx, void *Y, int64_t ldy,
     float *V = at<float>(ws, L.V);
     const int32_t ldv = max_ads_per_req * pool->max_rank;
 
+    if (long_items(N, n_req) && max_ads_per_req * pool->max_rank <= kKMax) {
+        TcArgs ta = {};
+        if (tc_encode_x(ta, X, N, pool->d_in, ldx) && tc_encode_y(ta, Y, N, pool->d_out, ldy)) {
+            PlanArgs pa = {};
+            pa.mode = kModeMulti;
+            pa.N = N;
+            pa.item_off = req_off;
+            pa.n_items = n_req;
+            pa.ad_off = ad_off;
+            pa.max_ads = max_ads_per_req;
+            pa.groups = groups;
+            pa.max_groups = L.max_groups;
+            pa.group = kTcGroup;
+            pa.hdr = hdr;
+            LORA_CUDA(launch_plan(pa, s));
+            ta.mode = kModeMulti;
+            ta.groups = groups;
+            ta.hdr = hdr;
+            ta.ad_off = ad_off;
+            ta.ad_id = ad_id;
+            ta.ad_scale = ad_scale;
+            ta.max_ads = max_ads_per_req;
+            ta.scale = 1.0f;
+            ta.pool = pool_dev(pool);
+            ta.V = V;
+            ta.ldv = ldv;
+            ta.slot_stride = pool->max_rank;
+            ta.Y = static_cast<__nv_bfloat16 *>(Y);
+            ta.ldy = ldy;
+            ta.err = &hdr->err;
+            LORA_CUDA(launch_tc_shrink(ta, N / kTcGroup + n_req + 1, s));
+            LORA_CUDA(launch_tc_expand(ta, s));
+            return LORA_OK;
+        }
+    }
+
     PlanArgs pa = {};
     pa.mode = kModeMulti;
     pa.N = N;
@@ -462,6 +581,7 @@ lora_status lora_apply_multi(const void *X, int64_t ldx, void *Y, int64_t ldy,
     pa.max_ads = max_ads_per_req;
     pa.groups = groups;
     pa.max_groups = L.max_groups;
+    pa.group = kGroup;
     pa.hdr = hdr;
     LORA_CUDA(launch_plan(pa, s));
 

@@ -1,6 +1,7 @@
 // Internal declarations shared by the kernel files and the C-ABI layer.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -53,6 +54,7 @@ struct PlanArgs {
     // groups
     Group *groups;
     int32_t max_groups;
+    int32_t group;            // tokens per group (kGroup for the CUDA-core kernels, 128 for tcgen05)
     WsHeader *hdr;
 };
 
@@ -167,6 +169,37 @@ size_t fused_smem_bytes(int32_t N, int32_t n_adapters, int32_t Wk);
 bool fused_bgmv_supported(int32_t N, int32_t n_adapters, int32_t d_in);
 cudaError_t launch_bgmv_fused(const FusedBgmvArgs &a, cudaStream_t s, bool pdl);
 bool pdl_enabled();
+
+// ------------------------------------------------------------ tcgen05 kernels
+constexpr int kTcGroup = 128;       // rows per tensor-core tile
+constexpr int kKMax = 128;          // stacked rank a tile may carry
+
+struct TcArgs {
+    CUtensorMap map_x;       // X [N, d_in], boxes 64 x 128, 128-byte swizzle (shrink)
+    CUtensorMap map_y;       // Y [N, d_out], same boxes (expand)
+    int32_t mode;            // kModeSgmv or kModeMulti
+    const Group *groups;     // tiles of <= kTcGroup rows, one item each
+    const WsHeader *hdr;
+    const int32_t *seg_ad;
+    const int32_t *ad_off;
+    const int32_t *ad_id;
+    const float *ad_scale;
+    int32_t max_ads;
+    float scale;
+    PoolDev pool;
+    float *V;                // fp32 intermediate, row stride ldv, stacked adapters slot_stride apart
+    int64_t ldv;
+    int32_t slot_stride;
+    __nv_bfloat16 *Y;
+    int64_t ldy;
+    uint32_t *err;
+};
+
+bool tc_encode_x(TcArgs &a, const void *X, int32_t N, int32_t d_in, int64_t ldx);
+bool tc_encode_y(TcArgs &a, const void *Y, int32_t N, int32_t d_out, int64_t ldy);
+cudaError_t launch_tc_shrink(const TcArgs &a, int max_tiles, cudaStream_t s);
+cudaError_t launch_tc_expand(const TcArgs &a, cudaStream_t s);
+bool tc_enabled();
 
 // Launchers (return the CUDA error of the launch).
 cudaError_t launch_plan(const PlanArgs &a, cudaStream_t s);

@@ -7,7 +7,7 @@
 // -> exclusive scan -> stable scatter).  Prefill segments and multi-adapter
 // requests arrive already grouped; the plan kernel only validates their
 // offsets.  In every mode it then cuts each item (segment / request) into
-// work groups of at most kGroup tokens.
+// work groups of at most `group` tokens.
 //
 // One CTA of 1024 threads does everything: the decode batches this serves
 // hold hundreds to a few thousand tokens, and one CTA keeps the histogram in
@@ -172,20 +172,21 @@ __global__ void __launch_bounds__(kPlanThreads) k_plan(PlanArgs p)
         }
     }
 
-    // cut every item into groups of at most kGroup tokens
+    // cut every item into groups of at most p.group tokens
     Group *groups = p.groups;
     const int32_t max_groups = p.max_groups;
+    const int32_t G = p.group;
     long long total = block_scan<long long>(
         n_items,
-        [&](int k) { return (long long)((item_off[k + 1] - item_off[k] + kGroup - 1) / kGroup); },
+        [&](int k) { return (long long)((item_off[k + 1] - item_off[k] + G - 1) / G); },
         [&](int k, long long pre, long long v) {
             const int32_t lo = item_off[k], hi = item_off[k + 1];
             for (int32_t i = 0; i < (int32_t)v; ++i) {
                 const long long g = pre + i;
                 if (g < max_groups) {
                     Group gr;
-                    gr.p0 = lo + i * kGroup;
-                    gr.cnt = min(kGroup, hi - gr.p0);
+                    gr.p0 = lo + i * G;
+                    gr.cnt = min(G, hi - gr.p0);
                     gr.item = k;
                     gr.pad = 0;
                     groups[g] = gr;

@@ -120,6 +120,7 @@ extern "C" lora_status lora_apply_multi_static(const void *X, int64_t ldx, void 
         pa.max_ads = max_ads_per_req;
         pa.groups = groups;
         pa.max_groups = max_groups;
+        pa.group = kGroup;
         pa.hdr = hdr;
         if (launch_plan(pa, s) != cudaSuccess)
             return LORA_ERR_CUDA;

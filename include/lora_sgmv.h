@@ -80,7 +80,8 @@ typedef enum {
     LORA_ERR_BAD_ADAPTER = 4,   /* device: adapter id, rank or pool offset out of range */
     LORA_ERR_BAD_SEGMENT = 8,   /* device: segment/request offsets decreasing or outside [0, N] */
     LORA_ERR_CUDA = 16,         /* host: a CUDA runtime call (launch, copy) failed */
-    LORA_ERR_WORKSPACE = 32     /* host: workspace null, misaligned or too small */
+    LORA_ERR_WORKSPACE = 32,    /* host: workspace null, misaligned or too small */
+    LORA_ERR_TIMEOUT = 64       /* device: a pipeline wait inside a kernel expired (work skipped) */
 } lora_status;
 
 /* One projection's resident adapter pool ("all LoRAs stay resident", same

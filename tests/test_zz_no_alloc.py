@@ -35,7 +35,9 @@ def test_static_scratch_matches_the_workspace_entry_point_on_two_calls():
         torch.cuda.synchronize()
         assert int(err.item()) == 0
         got, want = widen(to_host(y)), widen(to_host(y_ref))
-        check_parity(got, want, f"static scratch vs workspace, call seed {seed}")
+        # both sides are bf16 results (the workspace entry point may take the tensor-core
+        # path, whose rank-r intermediate is bf16), so both roundings are allowed for
+        check_parity(got, want, f"static scratch vs workspace, call seed {seed}", ref_rounded=True)
         assert np.max(np.abs(want - widen(to_host(c.Y)))) > 0   # the call did change y
 
 
