@@ -370,6 +370,7 @@ lora_status lora_sgmv_shrink(const void *X, int64_t ldx, float *V, int64_t ldv,
 
     if (long_items(N, n_seg) && aligned_v(V, ldv)) {
         TcArgs ta = {};
+        tc_encode_a(ta, pool->A, pool->A_elems, pool->d_in);
         if (tc_encode_x(ta, X, N, pool->d_in, ldx)) {
             PlanArgs pa = {};
             pa.mode = kModeSgmv;
@@ -538,6 +539,7 @@ lora_status lora_apply_multi(const void *X, int64_t ldx, void *Y, int64_t ldy,
 
     if (long_items(N, n_req) && max_ads_per_req * pool->max_rank <= kKMax) {
         TcArgs ta = {};
+        tc_encode_a(ta, pool->A, pool->A_elems, pool->d_in);
         if (tc_encode_x(ta, X, N, pool->d_in, ldx) && tc_encode_y(ta, Y, N, pool->d_out, ldy)) {
             PlanArgs pa = {};
             pa.mode = kModeMulti;

@@ -177,6 +177,8 @@ constexpr int kKMax = 128;          // stacked rank a tile may carry
 struct TcArgs {
     CUtensorMap map_x;       // X [N, d_in], boxes 64 x 128, 128-byte swizzle (shrink)
     CUtensorMap map_y;       // Y [N, d_out], same boxes (expand)
+    CUtensorMap map_a;       // A pool as [A_elems / d_in, d_in], boxes 64 x 8 (shrink), valid if a_tma
+    int32_t a_tma;
     int32_t mode;            // kModeSgmv or kModeMulti
     const Group *groups;     // tiles of <= kTcGroup rows, one item each
     const WsHeader *hdr;
@@ -197,6 +199,8 @@ struct TcArgs {
 
 bool tc_encode_x(TcArgs &a, const void *X, int32_t N, int32_t d_in, int64_t ldx);
 bool tc_encode_y(TcArgs &a, const void *Y, int32_t N, int32_t d_out, int64_t ldy);
+// optional: without it the shrink gathers A rows with cp.async
+bool tc_encode_a(TcArgs &a, const void *A, int64_t A_elems, int32_t d_in);
 cudaError_t launch_tc_shrink(const TcArgs &a, int max_tiles, cudaStream_t s);
 cudaError_t launch_tc_expand(const TcArgs &a, cudaStream_t s);
 bool tc_enabled();

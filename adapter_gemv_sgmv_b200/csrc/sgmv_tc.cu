@@ -43,9 +43,9 @@ constexpr int kBM = 128;            // rows per tile
 constexpr int kBN = 128;            // expand: outputs per unit
 constexpr int kBK = 64;             // shrink: d_in per k-block (one 128-byte swizzle atom)
 constexpr int kAtom = kBM * 128;    // bytes of a 128-row x 64-column bf16 swizzle atom
-constexpr int kShrinkStages = 4;
-constexpr int kExpandBStages = 3;
-constexpr int kExpandYStages = 2;
+constexpr int kShrinkStages = 6;
+constexpr int kExpandBStages = 2;
+constexpr int kExpandYStages = 3;
 constexpr unsigned long long kWaitNs = 2000000000ull;   // 2 s bound on any single wait
 
 // ------------------------------------------------------------------ PTX glue
@@ -121,11 +121,39 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, u
         : "memory");
 }
 
+// TMA store of a 2-D box from shared memory (bulk-group completion).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, const void *src, int x, int y)
+{
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];"
+                 ::"l"(map), "r"(smem_u32(src)), "r"(x), "r"(y)
+                 : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// the bulk groups committed by this thread, all but the newest one, have finished reading shared memory
+__device__ __forceinline__ void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// ... and have completed
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d)
+{
+    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
+__device__ __forceinline__ void ld_shared_v4(uint32_t addr, uint32_t (&w)[4])
+{
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]) : "r"(addr)
+                 : "memory");
+}
+
 // 16-byte async copy global -> shared; when !pred the destination is zero-filled
 // and nothing is read (the source must still be a valid address).
+// (No memory clobber: the copy lands asynchronously anyway, and the address
+// tables read around it in shared memory must stay free to be scheduled early.)
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool pred)
 {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(pred ? 16 : 0) : "memory");
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(pred ? 16 : 0));
 }
 
 // Arrive on `bar` once this thread's earlier cp.async copies have landed.
@@ -224,76 +252,101 @@ __device__ __forceinline__ bool adapter_ok(const PoolDev &P, int32_t a, int32_t 
     return true;
 }
 
-// The adapter stack of one tile: entry e covers ranks [kb[e], kb[e] + r[e]) of
-// the stacked axis and reads V columns slot[e] * slot_stride + j.
-struct Stack {
-    int n;
-    int kpad;                     // stacked rank rounded up to 16 (MMA N or K)
+// The adapter stack of one tile: entry i covers ranks [kb[i], kb[i] + r[i]) of
+// the stacked axis, reads V columns slot[i] * slot_stride + j and is scaled
+// by s[i].  The roles work on different tiles at any moment, so every warp
+// keeps its own copy in shared memory.
+struct StackSm {
+    int n;                                  // entries
+    int ktot;                               // stacked rank
+    int kpad;                               // stacked rank rounded up to 16 (MMA N or K)
+    int a_tma;                              // every entry's A offset is a multiple of d_in
     int r[LORA_MAX_ADS_PER_REQ];
     int kb[LORA_MAX_ADS_PER_REQ];
     int slot[LORA_MAX_ADS_PER_REQ];
     float s[LORA_MAX_ADS_PER_REQ];
-    int64_t aoff[LORA_MAX_ADS_PER_REQ];
-    int64_t boff[LORA_MAX_ADS_PER_REQ];
+    long long aoff[LORA_MAX_ADS_PER_REQ];
+    long long boff[LORA_MAX_ADS_PER_REQ];
 };
 
-// Build the stack of item `item`; adapters failing validation are left out
-// (and reported) -- the shrink and the expand leave out the same ones.
-__device__ void build_stack(const TcArgs &p, int item, Stack &st, bool report)
+// the entry holding stacked rank k (k < ktot)
+__device__ __forceinline__ int stack_entry(const StackSm &st, int k)
 {
+    int e = 0;
+    for (int i = 1; i < st.n; ++i)
+        if (k >= st.kb[i])
+            e = i;
+    return e;
+}
+
+// One warp builds the stack of item `item`; lane e looks at the item's adapter
+// e.  Adapters failing validation are left out (and reported when `report`);
+// the shrink and the expand leave out the same ones.  The host sends only
+// calls whose stacks fit in kKMax ranks; an entry that would not fit is left
+// out and reported as a bad segment.
+__device__ void warp_build_stack(const TcArgs &p, int item, StackSm &st, bool report)
+{
+    const int lane = threadIdx.x & 31;
+    __syncwarp();                           // this warp's readers of the previous stack are done
     int lo = 0, n = 1;
     if (p.mode == kModeMulti) {
         lo = p.ad_off[item];
         n = min(p.ad_off[item + 1] - lo, p.max_ads);
     }
-    st.n = 0;
-    int k = 0;
-    for (int e = 0; e < n; ++e) {
-        const int32_t a = p.mode == kModeMulti ? p.ad_id[lo + e] : p.seg_ad[item];
-        int32_t r;
-        int64_t ao, bo;
-        if (!adapter_ok(p.pool, a, &r, &ao, &bo)) {
-            if (report)
-                atomicOr(p.err, (uint32_t)LORA_ERR_BAD_ADAPTER);
-            continue;
-        }
-        if (k + r > kKMax) {     // the host only sends calls whose stacks fit
-            if (report)
-                atomicOr(p.err, (uint32_t)LORA_ERR_BAD_SEGMENT);
-            continue;
-        }
-        const int i = st.n++;
+    int32_t r = 0;
+    int64_t ao = 0, bo = 0;
+    float sc = 0.f;
+    bool ok = false;
+    if (lane < n) {
+        const int32_t a = p.mode == kModeMulti ? p.ad_id[lo + lane] : p.seg_ad[item];
+        ok = adapter_ok(p.pool, a, &r, &ao, &bo);
+        if (!ok && report)
+            atomicOr(p.err, (uint32_t)LORA_ERR_BAD_ADAPTER);
+        sc = p.mode == kModeMulti ? p.ad_scale[lo + lane] : p.scale;
+    }
+    if (!ok)
+        r = 0;
+    int incl = r;                           // inclusive prefix of the ranks over the item's adapters
+#pragma unroll
+    for (int d = 1; d < LORA_MAX_ADS_PER_REQ; d <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, d);
+        if (lane >= d)
+            incl += t;
+    }
+    const bool fits = ok && incl <= kKMax;
+    if (ok && !fits && report)
+        atomicOr(p.err, (uint32_t)LORA_ERR_BAD_SEGMENT);
+    const unsigned m = __ballot_sync(0xffffffffu, fits);
+    const int ktot = (int)__reduce_max_sync(0xffffffffu, fits ? (unsigned)incl : 0u);
+    const bool a_tma = __all_sync(0xffffffffu, !fits || (ao % p.pool.d_in) == 0);
+    if (fits) {
+        const int i = __popc(m & ((1u << lane) - 1u));
         st.r[i] = r;
-        st.kb[i] = k;
-        st.slot[i] = e;
-        st.s[i] = p.mode == kModeMulti ? p.ad_scale[lo + e] : p.scale;
+        st.kb[i] = incl - r;
+        st.slot[i] = lane;
+        st.s[i] = sc;
         st.aoff[i] = ao;
         st.boff[i] = bo;
-        k += r;
     }
-    st.kpad = (k + 15) & ~15;
+    if (lane == 0) {
+        st.n = __popc(m);
+        st.ktot = ktot;
+        st.kpad = (ktot + 15) & ~15;
+        st.a_tma = a_tma ? 1 : 0;
+    }
+    __syncwarp();
 }
-
-#ifdef LORA_TC_TRACE
-// Development aid: per-iteration %globaltimer stamps of CTA 0 (slot = role * 4096 + iter * 4 + point).
-__device__ unsigned long long g_tc_trace[3 * 4096];
-#define TCTRACE(role, iter, point)                                                           \
-    do {                                                                                     \
-        if (blockIdx.x == 0 && (threadIdx.x & 31) == 0 && (iter) < 1024)                     \
-            g_tc_trace[(role) * 4096 + (iter) * 4 + (point)] = now_ns();                     \
-    } while (0)
-#else
-#define TCTRACE(role, iter, point) \
-    do {                           \
-    } while (0)
-#endif
 
 // ============================================================ shrink kernel
 //
 // Unit = one tile of <= 128 rows of one item.  D[128 x kpad] = X_tile A_stack^T
-// over d_in in 64-column k-blocks; the epilogue writes V rows (fp32).
+// over d_in in 64-column k-blocks; the epilogue writes V rows (fp32).  The A
+// rows of a k-block come by TMA in 8-row boxes over the A pool seen as a
+// [A_elems / d_in, d_in] matrix (every adapter packed at a multiple of d_in),
+// else by cp.async, 16 bytes at a time.
 struct ShrinkSmem {
-    static constexpr int kStage = 2 * kAtom;   // x atom + A atom
+    static constexpr int kA = kKMax * 128;          // up to 128 stacked A rows x 64 columns
+    static constexpr int kStage = kAtom + kA;       // x atom + A rows
     static constexpr int kBytes = kShrinkStages * kStage;
 };
 
@@ -304,6 +357,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_shrink(const __grid_consta
     unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(sm_dyn) + 1023) & ~(uintptr_t)1023);
     __shared__ __align__(8) uint64_t full_bar[kShrinkStages], empty_bar[kShrinkStages];
     __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2];
+    __shared__ __align__(8) StackSm stk[kTcThreads / 32];
+    __shared__ long long arow[kKMax];        // producer, cp.async path: element offset of stacked row j's A row
+    __shared__ int vcol[4][kKMax / 4];       // epilogue warp q: V column of stacked columns 4g..4g+3 (-1: none)
     __shared__ uint32_t tmem_base;
     __shared__ int abort_flag;
 
@@ -335,66 +391,79 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_shrink(const __grid_consta
 
     if (warp == 0) {
         // ------------------------------------------------ producer
+        StackSm &st = stk[0];
         int it = 0;
         for (int u = u0; u < u1; ++u) {
             const Group gr = p.groups[u];
-            Stack st;
-            build_stack(p, gr.item, st, false);
+            warp_build_stack(p, gr.item, st, false);
+            const bool use_tma = st.a_tma && p.a_tma;
+            const int nbox = st.ktot >> 3;
+            int box_row = 0;                 // this lane's 8-row A box: its first row in the pool view
+            if (use_tma) {
+                if (lane < nbox) {
+                    const int e = stack_entry(st, lane * 8);
+                    box_row = (int)(st.aoff[e] / d_in) + (lane * 8 - st.kb[e]);
+                }
+            } else {
+                for (int j = lane; j < kKMax; j += 32) {
+                    long long o = -1;
+                    if (j < st.ktot) {
+                        const int e = stack_entry(st, j);
+                        o = st.aoff[e] + (long long)(j - st.kb[e]) * d_in;
+                    }
+                    arow[j] = o;
+                }
+                __syncwarp();
+            }
+            const uint32_t tx = (uint32_t)kAtom + (use_tma ? (uint32_t)nbox * 1024u : 0u);
             for (int kb = 0; kb < n_kb; ++kb, ++it) {
                 const int s = it % kShrinkStages;
                 const uint32_t ph = (it / kShrinkStages) & 1;
-                TCTRACE(0, it, 0);
                 if (!warp_wait(&empty_bar[s], ph ^ 1, &abort_flag, p.err))
                     goto done;
-                TCTRACE(0, it, 1);
                 unsigned char *xs = sm + s * ShrinkSmem::kStage;
                 unsigned char *as = xs + kAtom;
                 if (lane == 0) {
-                    mbar_arrive_expect_tx(&full_bar[s], kAtom);
+                    mbar_arrive_expect_tx(&full_bar[s], tx);
                     tma_load_2d(xs, &p.map_x, &full_bar[s], kb * kBK, gr.p0);
                 }
-                // A rows of the stacked adapters: row j of the stack, chunk c of the k-block
-                const uint32_t abase = smem_u32(as);
-                for (int idx = lane; idx < kBM * 8; idx += 32) {
-                    const int j = idx >> 3, c = idx & 7;
-                    const int col = kb * kBK + c * 8;
-                    const void *src = p.pool.A;
-                    bool ok = false;
-                    for (int e = 0; e < st.n; ++e) {
-                        if (j >= st.kb[e] && j < st.kb[e] + st.r[e] && col < d_in) {
-                            src = p.pool.A + st.aoff[e] + (int64_t)(j - st.kb[e]) * d_in + col;
-                            ok = true;
-                        }
-                    }
-                    if (j < st.kpad || ok)
-                        cp_async16(abase + sw128_off(j, c), src, ok);
+                __syncwarp();
+                if (use_tma) {
+                    if (lane < nbox)
+                        tma_load_2d(as + lane * 1024, &p.map_a, &full_bar[s], kb * kBK, box_row);
+                } else {
+                    // stacked row j, 16-byte chunk c; rows past the stack feed only
+                    // accumulator columns that are never stored
+                    const int c = lane & 7, col = kb * kBK + c * 8;
+                    const bool in = col < d_in;
+                    const uint32_t abase = smem_u32(as);
+                    for (int j = lane >> 3; j < st.ktot; j += 4)
+                        cp_async16(abase + sw128_off(j, c), in ? p.pool.A + arow[j] + col : p.pool.A, in);
                 }
                 cp_async_arrive(&full_bar[s]);
-                TCTRACE(0, it, 2);
             }
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
+        StackSm &st = stk[1];
         int it = 0, t = 0;
         for (int u = u0; u < u1; ++u, ++t) {
             const Group gr = p.groups[u];
-            Stack st;
-            build_stack(p, gr.item, st, false);
+            warp_build_stack(p, gr.item, st, false);
+            const int kpad = st.kpad;
             const int b = t & 1;
             if (!warp_wait(&acc_empty[b], ((t >> 1) & 1) ^ 1, &abort_flag, p.err))
                 goto done;
             tc_fence_after();
-            const uint32_t idesc = idesc_bf16(kBM, st.kpad > 0 ? st.kpad : 16);
+            const uint32_t idesc = idesc_bf16(kBM, kpad > 0 ? kpad : 16);
             for (int kb = 0; kb < n_kb; ++kb, ++it) {
                 const int s = it % kShrinkStages;
                 const uint32_t ph = (it / kShrinkStages) & 1;
-                TCTRACE(1, it, 0);
                 if (!warp_wait(&full_bar[s], ph, &abort_flag, p.err))
                     goto done;
-                TCTRACE(1, it, 1);
                 fence_async_smem();
                 tc_fence_after();
-                if (lane == 0 && st.kpad > 0) {
+                if (lane == 0 && kpad > 0) {
                     const uint32_t xa = smem_u32(sm + s * ShrinkSmem::kStage);
                     const uint32_t aa = xa + kAtom;
 #pragma unroll
@@ -415,11 +484,22 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_shrink(const __grid_consta
         // ------------------------------------------------ epilogue: D -> V rows
         const int q = warp & 3;                 // TMEM lane quarter owned by this warp
         const int row = q * 32 + lane;
+        StackSm &st = stk[warp];
+        int *vc = vcol[q];
         int t = 0;
         for (int u = u0; u < u1; ++u, ++t) {
             const Group gr = p.groups[u];
-            Stack st;
-            build_stack(p, gr.item, st, tid == 64);
+            warp_build_stack(p, gr.item, st, warp == 2);
+            {
+                const int k = lane * 4;
+                int c = -1;
+                if (k < st.ktot) {
+                    const int e = stack_entry(st, k);
+                    c = st.slot[e] * p.slot_stride + (k - st.kb[e]);
+                }
+                vc[lane] = c;
+            }
+            __syncwarp();
             const int b = t & 1;
             if (!warp_wait(&acc_full[b], (t >> 1) & 1, &abort_flag, p.err))
                 goto done;
@@ -430,16 +510,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_shrink(const __grid_consta
                 float v[32];
                 tmem_ld32(tmem + b * 128 + ((uint32_t)(q * 32) << 16) + c0, v);
                 if (valid) {
-                    // stacked column c0 + jj belongs to entry e: V[row][slot_e * stride + (c0 + jj - kb_e)]
 #pragma unroll
-                    for (int jj = 0; jj < 32; jj += 4) {
-                        const int col = c0 + jj;
-                        for (int e = 0; e < st.n; ++e) {
-                            if (col >= st.kb[e] && col < st.kb[e] + st.r[e]) {
-                                *reinterpret_cast<float4 *>(vrow + st.slot[e] * p.slot_stride + (col - st.kb[e])) =
-                                    make_float4(v[jj], v[jj + 1], v[jj + 2], v[jj + 3]);
-                            }
-                        }
+                    for (int g = 0; g < 8; ++g) {
+                        const int col = vc[(c0 >> 2) + g];
+                        if (col >= 0)
+                            *reinterpret_cast<float4 *>(vrow + col) =
+                                make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
                     }
                 }
             }
@@ -461,7 +537,8 @@ done:
 //
 // Unit = (tile, 128-output slice).  D[128 x 128] = V_tile B_stack[slice]^T over
 // the stacked rank (V staged once per tile as bf16 with the scales folded in);
-// the epilogue adds D to the y tile (TMA-loaded) and stores the tile's rows.
+// the epilogue adds D to the y tile (TMA-loaded) in shared memory and a TMA
+// store writes the tile back (a ragged tile: plain coalesced stores of its rows).
 struct ExpandSmem {
     static constexpr int kV = 2 * kAtom;                 // V: 128 rows x up to 128 ranks
     static constexpr int kB = 2 * kAtom;                 // B: 128 outputs x up to 128 ranks
@@ -478,7 +555,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_expand(const __grid_consta
     __shared__ __align__(8) uint64_t b_full[kExpandBStages], b_empty[kExpandBStages];
     __shared__ __align__(8) uint64_t y_full[kExpandYStages], y_empty[kExpandYStages];
     __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2];
-    __shared__ __align__(8) uint64_t v_full, v_empty;
+    __shared__ __align__(8) uint64_t v_full, v_empty, ep_bar;
+    __shared__ __align__(8) StackSm stk[kTcThreads / 32];
+    __shared__ long long cb_off[kKMax / 8];  // producer: B element offset of stacked 8-rank chunk c in output row 0
+    __shared__ int cb_r[kKMax / 8];          // its row stride (the adapter's rank); 0 = padding chunk
+    __shared__ int vsrc[4][kKMax / 8];       // epilogue warp q: V column of stacked chunk c (-1: zero)
+    __shared__ float vsc[4][kKMax / 8];      // and its adapter's scale
     __shared__ uint32_t tmem_base;
     __shared__ int abort_flag;
 
@@ -496,7 +578,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_expand(const __grid_consta
         }
         for (int s = 0; s < kExpandYStages; ++s) {
             mbar_init(&y_full[s], 1);        // expect_tx
-            mbar_init(&y_empty[s], 4);       // epilogue warps
+            mbar_init(&y_empty[s], 1);       // the epilogue thread that stored the tile
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&acc_full[b], 1);
@@ -504,6 +586,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_expand(const __grid_consta
         }
         mbar_init(&v_full, 4);               // epilogue warps, after staging V
         mbar_init(&v_empty, 1);              // MMA commit after a tile's last unit
+        mbar_init(&ep_bar, 4);               // the epilogue warps meet (y tile complete in shared memory)
         abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -515,18 +598,40 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_expand(const __grid_consta
     const uint32_t tmem = tmem_base;
 
     if (warp == 0) {
-        // ------------------------------------------------ producer: B slices (cp.async), y tiles (TMA)
+        // ------------------------------------------------ producer: y tiles (TMA), B slices (cp.async)
+        StackSm &st = stk[0];
         int it = 0;
         int64_t prev_tile = -1;
-        Stack st;
-        st.n = 0;
-        st.kpad = 0;
+        int nch = 0, o_l = 0, c_l = 0, dq = 0, dr = 0;
+        int p0 = 0;
         for (int64_t u = u0; u < u1; ++u, ++it) {
             const int tile = (int)(u / n_ns), ns = (int)(u - (int64_t)tile * n_ns);
-            const Group gr = p.groups[tile];
             if (tile != prev_tile) {
-                build_stack(p, gr.item, st, false);
+                const Group gr = p.groups[tile];
+                p0 = gr.p0;
+                warp_build_stack(p, gr.item, st, false);
                 prev_tile = tile;
+                if (lane < kKMax / 8) {
+                    const int k = lane * 8;
+                    long long o = 0;
+                    int rr = 0;
+                    if (k < st.ktot) {
+                        const int e = stack_entry(st, k);
+                        o = st.boff[e] + (k - st.kb[e]);
+                        rr = st.r[e];
+                    }
+                    cb_off[lane] = o;
+                    cb_r[lane] = rr;
+                }
+                __syncwarp();
+                // this lane walks chunk indices lane, lane + 32, ... of the (output, chunk) grid
+                nch = st.kpad >> 3;
+                if (nch > 0) {
+                    o_l = lane / nch;
+                    c_l = lane - o_l * nch;
+                    dq = 32 / nch;
+                    dr = 32 - dq * nch;
+                }
             }
             const int o0 = ns * kBN;
             const int sy = it % kExpandYStages;
@@ -535,41 +640,39 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_expand(const __grid_consta
             unsigned char *ys = sm + ExpandSmem::kOffY + sy * ExpandSmem::kY;
             if (lane == 0) {
                 mbar_arrive_expect_tx(&y_full[sy], ExpandSmem::kY);
-                tma_load_2d(ys, &p.map_y, &y_full[sy], o0, gr.p0);
-                tma_load_2d(ys + kAtom, &p.map_y, &y_full[sy], o0 + 64, gr.p0);
+                tma_load_2d(ys, &p.map_y, &y_full[sy], o0, p0);
+                tma_load_2d(ys + kAtom, &p.map_y, &y_full[sy], o0 + 64, p0);
             }
             const int sb = it % kExpandBStages;
             if (!warp_wait(&b_empty[sb], ((it / kExpandBStages) & 1) ^ 1, &abort_flag, p.err))
                 goto done;
             const uint32_t bbase = smem_u32(sm + ExpandSmem::kOffB + sb * ExpandSmem::kB);
-            // row o of the slice, 16-byte chunk c of the stacked rank axis (atom c / 8)
-            const int nch = st.kpad >> 3;
+            // output o of the slice, 16-byte chunk c of the stacked rank axis (atom c / 8);
+            // padding chunks and outputs past d_out are zero-filled
+            int o = o_l, c = c_l;
             for (int idx = lane; idx < kBN * nch; idx += 32) {
-                const int o = idx / nch, c = idx - o * nch;
-                const int k = c * 8;
-                const void *src = p.pool.B;
-                bool ok = false;
-                for (int e = 0; e < st.n; ++e) {
-                    if (k >= st.kb[e] && k < st.kb[e] + st.r[e] && o0 + o < d_out) {
-                        src = p.pool.B + st.boff[e] + (int64_t)(o0 + o) * st.r[e] + (k - st.kb[e]);
-                        ok = true;
-                    }
-                }
+                const int rr = cb_r[c];
+                const bool ok = rr > 0 && o0 + o < d_out;
+                const __nv_bfloat16 *src = ok ? p.pool.B + cb_off[c] + (long long)(o0 + o) * rr : p.pool.B;
                 cp_async16(bbase + (c >> 3) * kAtom + sw128_off(o, c & 7), src, ok);
+                c += dr;
+                o += dq;
+                if (c >= nch) {
+                    c -= nch;
+                    ++o;
+                }
             }
             cp_async_arrive(&b_full[sb]);
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
+        StackSm &st = stk[1];
         int it = 0, vt = 0;
         int64_t prev_tile = -1;
-        Stack st;
-        st.n = 0;
-        st.kpad = 0;
         for (int64_t u = u0; u < u1; ++u, ++it) {
             const int tile = (int)(u / n_ns);
             if (tile != prev_tile) {
-                build_stack(p, p.groups[tile].item, st, false);
+                warp_build_stack(p, p.groups[tile].item, st, false);
                 prev_tile = tile;
                 if (!warp_wait(&v_full, vt & 1, &abort_flag, p.err))
                     goto done;
@@ -600,54 +703,58 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_expand(const __grid_consta
             __syncwarp();
         }
     } else {
-        // ------------------------------------------------ epilogue: V staging, y += D
+        // ------------------------------------------------ epilogue: V staging, y += D, store
         const int q = warp & 3;
         const int row = q * 32 + lane;
         const int et = tid - 64;                // 0..127 over the epilogue warps
-        int it = 0, vt = 0;
+        StackSm &st = stk[warp];
+        int it = 0, vt = 0, pending = -1;
+        uint32_t ep_uses = 0;
         int64_t prev_tile = -1;
-        Stack st;
-        st.n = 0;
-        st.kpad = 0;
         Group gr = {0, 0, 0, 0};
         for (int64_t u = u0; u < u1; ++u, ++it) {
             const int tile = (int)(u / n_ns), ns = (int)(u - (int64_t)tile * n_ns);
             if (tile != prev_tile) {
                 gr = p.groups[tile];
-                build_stack(p, gr.item, st, false);   // the shrink kernel reports bad adapters
+                warp_build_stack(p, gr.item, st, false);   // the shrink kernel reports bad adapters
                 prev_tile = tile;
+                if (lane < kKMax / 8) {
+                    const int k = lane * 8;
+                    int c = -1;
+                    float sc = 0.f;
+                    if (k < st.ktot) {
+                        const int e = stack_entry(st, k);
+                        c = st.slot[e] * p.slot_stride + (k - st.kb[e]);
+                        sc = st.s[e];
+                    }
+                    vsrc[q][lane] = c;
+                    vsc[q][lane] = sc;
+                }
+                __syncwarp();
                 // wait until the MMAs of the previous tile stopped reading V
                 if (vt > 0 && !warp_wait(&v_empty, (vt - 1) & 1, &abort_flag, p.err))
                     goto done;
-                // V[row][stacked k] = bf16(s_e * V_e[row][k - kb_e]), zero outside the tile's rows
+                // V[row][stacked k] = bf16(s_e * V_e[row][k - kb_e]), zero outside the tile's rows and the stack
                 const bool valid = et < gr.cnt;
                 const float *vrow = p.V + (int64_t)(gr.p0 + (valid ? et : 0)) * p.ldv;
                 const uint32_t vbase = smem_u32(sm);
                 for (int c = 0; c < st.kpad / 8; ++c) {
-                    const int k = c * 8;
+                    const int col = vsrc[q][c];
                     uint32_t w[4] = {0u, 0u, 0u, 0u};
-                    if (valid) {
-                        for (int e = 0; e < st.n; ++e) {
-                            if (k >= st.kb[e] && k < st.kb[e] + st.r[e]) {
-                                const float *src = vrow + st.slot[e] * p.slot_stride + (k - st.kb[e]);
-                                const float4 a = *reinterpret_cast<const float4 *>(src);
-                                const float4 bq = *reinterpret_cast<const float4 *>(src + 4);
-                                const float sc = st.s[e];
-                                const __nv_bfloat162 h0 = __floats2bfloat162_rn(sc * a.x, sc * a.y);
-                                const __nv_bfloat162 h1 = __floats2bfloat162_rn(sc * a.z, sc * a.w);
-                                const __nv_bfloat162 h2 = __floats2bfloat162_rn(sc * bq.x, sc * bq.y);
-                                const __nv_bfloat162 h3 = __floats2bfloat162_rn(sc * bq.z, sc * bq.w);
-                                w[0] = *reinterpret_cast<const uint32_t *>(&h0);
-                                w[1] = *reinterpret_cast<const uint32_t *>(&h1);
-                                w[2] = *reinterpret_cast<const uint32_t *>(&h2);
-                                w[3] = *reinterpret_cast<const uint32_t *>(&h3);
-                            }
-                        }
+                    if (valid && col >= 0) {
+                        const float sc = vsc[q][c];
+                        const float4 a = *reinterpret_cast<const float4 *>(vrow + col);
+                        const float4 bq = *reinterpret_cast<const float4 *>(vrow + col + 4);
+                        const __nv_bfloat162 h0 = __floats2bfloat162_rn(sc * a.x, sc * a.y);
+                        const __nv_bfloat162 h1 = __floats2bfloat162_rn(sc * a.z, sc * a.w);
+                        const __nv_bfloat162 h2 = __floats2bfloat162_rn(sc * bq.x, sc * bq.y);
+                        const __nv_bfloat162 h3 = __floats2bfloat162_rn(sc * bq.z, sc * bq.w);
+                        w[0] = *reinterpret_cast<const uint32_t *>(&h0);
+                        w[1] = *reinterpret_cast<const uint32_t *>(&h1);
+                        w[2] = *reinterpret_cast<const uint32_t *>(&h2);
+                        w[3] = *reinterpret_cast<const uint32_t *>(&h3);
                     }
-                    const uint32_t dst = vbase + (c >> 3) * kAtom + sw128_off(et, c & 7);
-                    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(dst), "r"(w[0]), "r"(w[1]), "r"(w[2]),
-                                 "r"(w[3])
-                                 : "memory");
+                    st_shared_v4(vbase + (c >> 3) * kAtom + sw128_off(et, c & 7), w[0], w[1], w[2], w[3]);
                 }
                 fence_async_smem();
                 __syncwarp();
@@ -662,10 +769,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_expand(const __grid_consta
             if (!warp_wait(&y_full[sy], (it / kExpandYStages) & 1, &abort_flag, p.err))
                 goto done;
             tc_fence_after();
-            const bool valid = row < gr.cnt;
             const int o0 = ns * kBN;
-            const unsigned char *ys = sm + ExpandSmem::kOffY + sy * ExpandSmem::kY;
-            __nv_bfloat16 *yrow = p.Y + (int64_t)(gr.p0 + (valid ? row : 0)) * p.ldy;
+            unsigned char *ys = sm + ExpandSmem::kOffY + sy * ExpandSmem::kY;
+            const uint32_t ysa = smem_u32(ys);
 #pragma unroll 1
             for (int c0 = 0; c0 < kBN; c0 += 32) {
                 float d[32];
@@ -676,35 +782,75 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_expand(const __grid_consta
                         d[i] = 0.f;
                 }
                 // four 16-byte chunks of this row's y: atom c0 / 64, chunks (c0 % 64) / 8 ..
-                const unsigned char *atom = ys + (c0 >> 6) * kAtom;
+                const uint32_t atom = ysa + (c0 >> 6) * kAtom;
 #pragma unroll
                 for (int h = 0; h < 4; ++h) {
-                    const int c = ((c0 & 63) >> 3) + h;
-                    const uint4 yv = *reinterpret_cast<const uint4 *>(atom + sw128_off(row, c));
-                    const __nv_bfloat162 *y2 = reinterpret_cast<const __nv_bfloat162 *>(&yv);
-                    uint4 out;
-                    uint32_t *o32 = reinterpret_cast<uint32_t *>(&out);
+                    const uint32_t addr = atom + sw128_off(row, ((c0 & 63) >> 3) + h);
+                    uint32_t yw[4];
+                    ld_shared_v4(addr, yw);
+                    uint32_t ow[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const float2 yf = __bfloat1622float2(y2[e]);
+                        const float2 yf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&yw[e]));
                         const __nv_bfloat162 r2 =
                             __floats2bfloat162_rn(yf.x + d[h * 8 + 2 * e], yf.y + d[h * 8 + 2 * e + 1]);
-                        o32[e] = *reinterpret_cast<const uint32_t *>(&r2);
+                        ow[e] = *reinterpret_cast<const uint32_t *>(&r2);
                     }
-                    const int o = o0 + c0 + h * 8;
-                    if (valid && o < d_out)
-                        *reinterpret_cast<uint4 *>(yrow + o) = out;
+                    st_shared_v4(addr, ow[0], ow[1], ow[2], ow[3]);
                 }
             }
             tc_fence_before();
+            fence_async_smem();                 // this thread's y writes, before the TMA store reads them
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive(&acc_empty[b]);
-                mbar_arrive(&y_empty[sy]);
+                mbar_arrive(&ep_bar);
+            }
+            if (!warp_wait(&ep_bar, ep_uses & 1, &abort_flag, p.err))
+                goto done;
+            ++ep_uses;
+            if (gr.cnt == kBM) {
+                // full tile: one thread stores it; the stage is released once the store has read it
+                if (et == 0) {
+                    tma_store_2d(&p.map_y, ys, o0, gr.p0);
+                    tma_store_2d(&p.map_y, ys + kAtom, o0 + 64, gr.p0);
+                    bulk_commit();
+                    bulk_wait_read_1();
+                    if (pending >= 0)
+                        mbar_arrive(&y_empty[pending]);
+                    pending = sy;
+                }
+            } else {
+                // ragged tile: the valid rows, 16 bytes per thread, 256 contiguous bytes per row
+                for (int idx = et; idx < gr.cnt * 16; idx += 128) {
+                    const int r = idx >> 4, ch = idx & 15;
+                    const int o = o0 + ch * 8;
+                    if (o < d_out) {
+                        uint32_t w[4];
+                        ld_shared_v4(ysa + (ch >> 3) * kAtom + sw128_off(r, ch & 7), w);
+                        *reinterpret_cast<uint4 *>(p.Y + (int64_t)(gr.p0 + r) * p.ldy + o) =
+                            make_uint4(w[0], w[1], w[2], w[3]);
+                    }
+                }
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(&ep_bar);
+                if (!warp_wait(&ep_bar, ep_uses & 1, &abort_flag, p.err))
+                    goto done;
+                ++ep_uses;
+                if (et == 0) {
+                    bulk_wait_read_0();
+                    if (pending >= 0)
+                        mbar_arrive(&y_empty[pending]);
+                    pending = -1;
+                    mbar_arrive(&y_empty[sy]);
+                }
             }
         }
     }
 done:
+    if (tid == 64)
+        bulk_wait_all();                        // the last TMA stores have landed
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
@@ -783,6 +929,28 @@ cudaError_t launch_tc(void (*kernel)(TcArgs), bool *attr_set, const TcArgs &a, i
 
 }  // namespace
 
+bool tc_encode_a(TcArgs &a, const void *A, int64_t A_elems, int32_t d_in)
+{
+    // the A pool as a [A_elems / d_in, d_in] matrix, boxes of 64 columns x 8 rows
+    a.a_tma = 0;
+    const int64_t rows = A_elems / d_in;
+    if (rows < 1 || rows > 0x7fffffffLL)
+        return false;
+    EncodeTiledFn fn = encode_fn();
+    if (!fn)
+        return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)d_in, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)d_in * 2};
+    const cuuint32_t box[2] = {64, 8};
+    const cuuint32_t estr[2] = {1, 1};
+    if (fn(&a.map_a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(A), dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return false;
+    a.a_tma = 1;
+    return true;
+}
+
 bool tc_encode_x(TcArgs &a, const void *X, int32_t N, int32_t d_in, int64_t ldx)
 {
     return encode_rows(&a.map_x, X, N, d_in, ldx);
@@ -807,9 +975,3 @@ cudaError_t launch_tc_expand(const TcArgs &a, cudaStream_t s)
 
 }  // namespace lora
 
-#ifdef LORA_TC_TRACE
-extern "C" LORA_API int lora_debug_tc_trace(unsigned long long *host, int n)
-{
-    return (int)cudaMemcpyFromSymbol(host, lora::g_tc_trace, sizeof(unsigned long long) * (size_t)n);
-}
-#endif

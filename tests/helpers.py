@@ -39,6 +39,29 @@ def rand_host_pool(rng: np.random.Generator, ranks, d_in: int, d_out: int,
     return HostPool(A=A, B=B, A_off=A_off, B_off=B_off, rank=ranks, d_in=d_in, d_out=d_out)
 
 
+def scatter_pool(hp: HostPool, gap: int = 8) -> HostPool:
+    """The same adapters stored in reverse order with `gap` spare elements before
+    each one: offsets stay multiples of 8 but are no longer multiples of d_in."""
+    n = len(hp.rank)
+    A_off = np.zeros(n, np.int64)
+    B_off = np.zeros(n, np.int64)
+    a_pos = b_pos = 0
+    for a in reversed(range(n)):
+        r = int(hp.rank[a])
+        a_pos += gap
+        b_pos += gap
+        A_off[a], B_off[a] = a_pos, b_pos
+        a_pos += r * hp.d_in
+        b_pos += r * hp.d_out
+    A = np.full(a_pos + gap, 0x7FC0, np.uint16)       # NaN between adapters: a stray read shows
+    B = np.full(b_pos + gap, 0x7FC0, np.uint16)
+    for a in range(n):
+        r = int(hp.rank[a])
+        A[A_off[a]:A_off[a] + r * hp.d_in] = hp.A[hp.A_off[a]:hp.A_off[a] + r * hp.d_in]
+        B[B_off[a]:B_off[a] + r * hp.d_out] = hp.B[hp.B_off[a]:hp.B_off[a] + r * hp.d_out]
+    return HostPool(A=A, B=B, A_off=A_off, B_off=B_off, rank=hp.rank.copy(), d_in=hp.d_in, d_out=hp.d_out)
+
+
 def rand_x(rng: np.random.Generator, N: int, d: int) -> np.ndarray:
     return bf16_bits(rng.standard_normal((N, d)).astype(np.float32))
 

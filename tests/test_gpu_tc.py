@@ -10,7 +10,8 @@ import torch
 
 import adapter_gemv_sgmv_b200 as L
 import oracle
-from helpers import DevPool, check_close_f32, check_parity, dev_bf16, rand_host_pool, rand_x, widen
+from helpers import (DevPool, check_close_f32, check_parity, dev_bf16, rand_host_pool, rand_x,
+                     scatter_pool, widen)
 from workloads import to_host
 
 pytestmark = pytest.mark.gpu
@@ -21,11 +22,16 @@ def _i32(a):
     return torch.tensor(np.asarray(a, np.int32), device=DEV)
 
 
+@pytest.mark.parametrize("packed", [True, False])
 @pytest.mark.parametrize("d_in,d_out", [(264, 200), (4096, 384), (128, 1000)])
-def test_tc_sgmv_ragged(d_in, d_out):
+def test_tc_sgmv_ragged(d_in, d_out, packed):
+    """packed: adapters back to back (A rows fetched by TMA); else scattered with
+    gaps, offsets not multiples of d_in (A rows gathered 16 bytes at a time)."""
     rng = np.random.default_rng(d_in + d_out)
     ranks = [8, 24, 128, 40, 64]
     hp = rand_host_pool(rng, ranks, d_in, d_out)
+    if not packed:
+        hp = scatter_pool(hp)
     lens = [130, 1, 255, 0, 128, 37, 300]
     ads = [2, 0, 4, 1, 3, 2, 1]
     start = 5
@@ -52,11 +58,14 @@ def test_tc_sgmv_ragged(d_in, d_out):
     assert np.array_equal(got[outside], widen(Y0)[outside])
 
 
-def test_tc_multi_stacked_adapters():
+@pytest.mark.parametrize("packed", [True, False])
+def test_tc_multi_stacked_adapters(packed):
     rng = np.random.default_rng(7)
     d_in, d_out = 320, 272
     ranks = [8, 16, 32, 24, 32, 8]
     hp = rand_host_pool(rng, ranks, d_in, d_out)
+    if not packed:
+        hp = scatter_pool(hp)
     lens = [300, 0, 129, 64, 200]
     req_off = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
     N = int(req_off[-1]) + 7                      # a few rows outside every request
