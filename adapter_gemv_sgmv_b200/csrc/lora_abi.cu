@@ -393,7 +393,7 @@ lora_status lora_sgmv_shrink(const void *X, int64_t ldx, float *V, int64_t ldv,
             ta.ldv = ldv;
             ta.slot_stride = 0;
             ta.err = &hdr->err;
-            LORA_CUDA(launch_tc_shrink(ta, N / kTcGroup + n_seg + 1, s));
+            LORA_CUDA(launch_tc_shrink(ta, N / kTcGroup + n_seg + 1, pool->max_rank, s));
             return LORA_OK;
         }
     }
@@ -451,6 +451,7 @@ lora_status lora_sgmv_expand(const float *V, int64_t ldv, void *Y, int64_t ldy,
 
     if (long_items(N, n_seg) && aligned_v(V, ldv)) {
         TcArgs ta = {};
+        tc_encode_b(ta, pool->B, pool->B_elems);
         if (tc_encode_y(ta, Y, N, pool->d_out, ldy)) {
             PlanArgs pa = {};
             pa.mode = kModeSgmv;
@@ -475,7 +476,7 @@ lora_status lora_sgmv_expand(const float *V, int64_t ldv, void *Y, int64_t ldy,
             ta.Y = static_cast<__nv_bfloat16 *>(Y);
             ta.ldy = ldy;
             ta.err = &hdr->err;
-            LORA_CUDA(launch_tc_expand(ta, s));
+            LORA_CUDA(launch_tc_expand(ta, pool->max_rank, s));
             return LORA_OK;
         }
     }
@@ -540,6 +541,7 @@ lora_status lora_apply_multi(const void *X, int64_t ldx, void *Y, int64_t ldy,
     if (long_items(N, n_req) && max_ads_per_req * pool->max_rank <= kKMax) {
         TcArgs ta = {};
         tc_encode_a(ta, pool->A, pool->A_elems, pool->d_in);
+        tc_encode_b(ta, pool->B, pool->B_elems);
         if (tc_encode_x(ta, X, N, pool->d_in, ldx) && tc_encode_y(ta, Y, N, pool->d_out, ldy)) {
             PlanArgs pa = {};
             pa.mode = kModeMulti;
@@ -568,8 +570,8 @@ lora_status lora_apply_multi(const void *X, int64_t ldx, void *Y, int64_t ldy,
             ta.Y = static_cast<__nv_bfloat16 *>(Y);
             ta.ldy = ldy;
             ta.err = &hdr->err;
-            LORA_CUDA(launch_tc_shrink(ta, N / kTcGroup + n_req + 1, s));
-            LORA_CUDA(launch_tc_expand(ta, s));
+            LORA_CUDA(launch_tc_shrink(ta, N / kTcGroup + n_req + 1, max_ads_per_req * pool->max_rank, s));
+            LORA_CUDA(launch_tc_expand(ta, max_ads_per_req * pool->max_rank, s));
             return LORA_OK;
         }
     }

@@ -177,8 +177,14 @@ constexpr int kKMax = 128;          // stacked rank a tile may carry
 struct TcArgs {
     CUtensorMap map_x;       // X [N, d_in], boxes 64 x 128, 128-byte swizzle (shrink)
     CUtensorMap map_y;       // Y [N, d_out], same boxes (expand)
-    CUtensorMap map_a;       // A pool as [A_elems / d_in, d_in], boxes 64 x 8 (shrink), valid if a_tma
-    int32_t a_tma;
+    CUtensorMap map_a[3];    // A pool as [A_elems / d_in, d_in], boxes of 64 columns x 64 / 32 / 8 rows
+    int32_t a_tma;           // map_a valid (shrink)
+    CUtensorMap map_b[4];    // B pool as [B_elems / r, r], r = 16 << m, boxes of min(r, 64) x 128 rows
+    int32_t b_tma;           // bit m: map_b[m] valid (expand)
+    int32_t e_natoms;        // expand: 16 KB atoms per V / B stage (1 or 2; set by the launcher)
+    int32_t e_ystages;       // expand: y stages (set by the launcher)
+    int32_t s_stages;        // shrink: pipeline stages (set by the launcher)
+    int32_t s_stage;         // shrink: bytes per stage (set by the launcher)
     int32_t mode;            // kModeSgmv or kModeMulti
     const Group *groups;     // tiles of <= kTcGroup rows, one item each
     const WsHeader *hdr;
@@ -201,8 +207,11 @@ bool tc_encode_x(TcArgs &a, const void *X, int32_t N, int32_t d_in, int64_t ldx)
 bool tc_encode_y(TcArgs &a, const void *Y, int32_t N, int32_t d_out, int64_t ldy);
 // optional: without it the shrink gathers A rows with cp.async
 bool tc_encode_a(TcArgs &a, const void *A, int64_t A_elems, int32_t d_in);
-cudaError_t launch_tc_shrink(const TcArgs &a, int max_tiles, cudaStream_t s);
-cudaError_t launch_tc_expand(const TcArgs &a, cudaStream_t s);
+// optional: without it the expand gathers B rows with cp.async
+bool tc_encode_b(TcArgs &a, const void *B, int64_t B_elems);
+cudaError_t launch_tc_shrink(const TcArgs &a, int max_tiles, int kk, cudaStream_t s);
+// kk: the largest stacked rank of any item (max_rank, or max_ads * max_rank)
+cudaError_t launch_tc_expand(const TcArgs &a, int kk, cudaStream_t s);
 bool tc_enabled();
 
 // Launchers (return the CUDA error of the launch).

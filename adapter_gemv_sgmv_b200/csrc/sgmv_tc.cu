@@ -38,14 +38,19 @@
 namespace lora {
 namespace {
 
-constexpr int kTcThreads = 192;
+constexpr int kTcThreads = 192;       // shrink: producer, MMA, 4 epilogue warps
+constexpr int kExpandThreads = 320;   // expand: producer, MMA, 8 epilogue warps
+// heights of the A-pool TMA boxes (map_a[m])
+__host__ __device__ constexpr int abox_rows(int m) { return m == 0 ? 64 : (m == 1 ? 32 : 8); }
+// B-pool TMA views: map_b[m] sees the pool as [B_elems / r, r] for r = 16 << m, so
+// adapter a's output o is row B_off[a] / r + o when B_off[a] is a multiple of r
+__host__ __device__ constexpr int b_map(int r) { return r == 16 ? 0 : (r == 32 ? 1 : (r == 64 ? 2 : (r == 128 ? 3 : -1))); }
 constexpr int kBM = 128;            // rows per tile
 constexpr int kBN = 128;            // expand: outputs per unit
 constexpr int kBK = 64;             // shrink: d_in per k-block (one 128-byte swizzle atom)
 constexpr int kAtom = kBM * 128;    // bytes of a 128-row x 64-column bf16 swizzle atom
-constexpr int kShrinkStages = 6;
+constexpr int kMaxShrinkStages = 4;
 constexpr int kExpandBStages = 2;
-constexpr int kExpandYStages = 3;
 constexpr unsigned long long kWaitNs = 2000000000ull;   // 2 s bound on any single wait
 
 // ------------------------------------------------------------------ PTX glue
@@ -120,21 +125,6 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, u
         ::"r"(smem_u32(dst)), "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y)
         : "memory");
 }
-
-// TMA store of a 2-D box from shared memory (bulk-group completion).
-__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, const void *src, int x, int y)
-{
-    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];"
-                 ::"l"(map), "r"(smem_u32(src)), "r"(x), "r"(y)
-                 : "memory");
-}
-
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-// the bulk groups committed by this thread, all but the newest one, have finished reading shared memory
-__device__ __forceinline__ void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_read_0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-// ... and have completed
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d)
 {
@@ -216,12 +206,48 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
         v[i] = __uint_as_float(r[i]);
 }
 
+// 64 consecutive fp32 columns of this thread's TMEM lane (one load, then the wait).
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x64.b32 {"
+        "%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
+        "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+        "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63"
+        "}, [%64];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
+          "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]),
+          "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]),
+          "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
+          "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+        : "r"(taddr)
+        : "memory");
+}
+
 // Shared-memory matrix descriptor of a K-major operand in 128-byte-swizzled
 // atoms (8 rows x 128 bytes; 8-row groups 1024 bytes apart).
 __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr)
 {
     return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
            ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// The same for the 64- and 32-byte swizzles (8-row groups 512 / 256 bytes apart).
+__device__ __forceinline__ uint64_t sw64_desc(uint32_t saddr)
+{
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(512 >> 4) << 32) |
+           ((uint64_t)1 << 46) | ((uint64_t)4 << 61);
+}
+
+__device__ __forceinline__ uint64_t sw32_desc(uint32_t saddr)
+{
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(256 >> 4) << 32) |
+           ((uint64_t)1 << 46) | ((uint64_t)6 << 61);
 }
 
 // Instruction descriptor: bf16 A and B, fp32 D, both K-major, M x N.
@@ -261,6 +287,7 @@ struct StackSm {
     int ktot;                               // stacked rank
     int kpad;                               // stacked rank rounded up to 16 (MMA N or K)
     int a_tma;                              // every entry's A offset is a multiple of d_in
+    int b_tma;                              // every entry's B slice can come by TMA (see b_map)
     int r[LORA_MAX_ADS_PER_REQ];
     int kb[LORA_MAX_ADS_PER_REQ];
     int slot[LORA_MAX_ADS_PER_REQ];
@@ -319,6 +346,8 @@ __device__ void warp_build_stack(const TcArgs &p, int item, StackSm &st, bool re
     const unsigned m = __ballot_sync(0xffffffffu, fits);
     const int ktot = (int)__reduce_max_sync(0xffffffffu, fits ? (unsigned)incl : 0u);
     const bool a_tma = __all_sync(0xffffffffu, !fits || (ao % p.pool.d_in) == 0);
+    const int bm = b_map(r);
+    const bool b_tma = __all_sync(0xffffffffu, !fits || (bm >= 0 && ((p.b_tma >> bm) & 1) && (bo % r) == 0));
     if (fits) {
         const int i = __popc(m & ((1u << lane) - 1u));
         st.r[i] = r;
@@ -333,9 +362,24 @@ __device__ void warp_build_stack(const TcArgs &p, int item, StackSm &st, bool re
         st.ktot = ktot;
         st.kpad = (ktot + 15) & ~15;
         st.a_tma = a_tma ? 1 : 0;
+        st.b_tma = b_tma ? 1 : 0;
     }
     __syncwarp();
 }
+
+#ifdef LORA_TC_TRACE
+// Development aid: %globaltimer stamps of the last CTA, [role][unit][point].
+__device__ unsigned long long g_tc_trace[3 * 1024 * 8];
+#define TC_STAMP(role, iter, point)                                                          \
+    do {                                                                                     \
+        if (blockIdx.x == gridDim.x - 1 && (threadIdx.x & 31) == 0 && (iter) < 1024)         \
+            g_tc_trace[((role) * 1024 + (iter)) * 8 + (point)] = now_ns();                   \
+    } while (0)
+#else
+#define TC_STAMP(role, iter, point) \
+    do {                            \
+    } while (0)
+#endif
 
 // ============================================================ shrink kernel
 //
@@ -343,22 +387,20 @@ __device__ void warp_build_stack(const TcArgs &p, int item, StackSm &st, bool re
 // over d_in in 64-column k-blocks; the epilogue writes V rows (fp32).  The A
 // rows of a k-block come by TMA in 8-row boxes over the A pool seen as a
 // [A_elems / d_in, d_in] matrix (every adapter packed at a multiple of d_in),
-// else by cp.async, 16 bytes at a time.
-struct ShrinkSmem {
-    static constexpr int kA = kKMax * 128;          // up to 128 stacked A rows x 64 columns
-    static constexpr int kStage = kAtom + kA;       // x atom + A rows
-    static constexpr int kBytes = kShrinkStages * kStage;
-};
+// else by cp.async, 16 bytes at a time.  A stage holds the x atom and as many A
+// rows as the call's largest stacked rank (rounded to 16): at rank 64, 24 KB, and
+// four stages fit twice per SM, so two tiles can stream through one SM at once.
 
-__global__ void __launch_bounds__(kTcThreads, 1) k_tc_shrink(const __grid_constant__ TcArgs p)
+__global__ void __launch_bounds__(kTcThreads, 2) k_tc_shrink(const __grid_constant__ TcArgs p)
 {
     extern __shared__ __align__(1024) unsigned char sm_dyn[];
     // 1024-byte alignment for the swizzle atoms
     unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(sm_dyn) + 1023) & ~(uintptr_t)1023);
-    __shared__ __align__(8) uint64_t full_bar[kShrinkStages], empty_bar[kShrinkStages];
+    __shared__ __align__(8) uint64_t full_bar[kMaxShrinkStages], empty_bar[kMaxShrinkStages];
     __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2];
     __shared__ __align__(8) StackSm stk[kTcThreads / 32];
     __shared__ long long arow[kKMax];        // producer, cp.async path: element offset of stacked row j's A row
+    __shared__ int4 abox[kKMax / 8];         // producer, TMA path: (stacked row, pool row, map) of each A box
     __shared__ int vcol[4][kKMax / 4];       // epilogue warp q: V column of stacked columns 4g..4g+3 (-1: none)
     __shared__ uint32_t tmem_base;
     __shared__ int abort_flag;
@@ -369,9 +411,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_shrink(const __grid_consta
     const int u0 = (int)((int64_t)blockIdx.x * n_units / G), u1 = (int)((int64_t)(blockIdx.x + 1) * n_units / G);
     const int d_in = p.pool.d_in;
     const int n_kb = (d_in + kBK - 1) / kBK;
+    const int n_st = p.s_stages;
 
     if (tid == 0) {
-        for (int s = 0; s < kShrinkStages; ++s) {
+        for (int s = 0; s < kMaxShrinkStages; ++s) {
             mbar_init(&full_bar[s], 33);     // producer lane 0's expect_tx + 32 cp.async arrivals
             mbar_init(&empty_bar[s], 1);     // MMA commit
         }
@@ -397,12 +440,28 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_shrink(const __grid_consta
             const Group gr = p.groups[u];
             warp_build_stack(p, gr.item, st, false);
             const bool use_tma = st.a_tma && p.a_tma;
-            const int nbox = st.ktot >> 3;
-            int box_row = 0;                 // this lane's 8-row A box: its first row in the pool view
+            // A boxes: each entry's rows cut into 64-, 32- and 8-row boxes (at most 16 boxes)
+            int nbox = 0;
+            int box_j = 0, box_row = 0, box_m = 0;   // this lane's box: stacked row, pool row, map
             if (use_tma) {
+                if (lane == 0) {
+                    for (int e = 0; e < st.n; ++e) {
+                        const int row0 = (int)(st.aoff[e] / d_in);
+                        for (int j = 0; j < st.r[e];) {
+                            const int m = st.r[e] - j >= 64 ? 0 : (st.r[e] - j >= 32 ? 1 : 2);
+                            abox[nbox] = make_int4(st.kb[e] + j, row0 + j, m, 0);
+                            ++nbox;
+                            j += abox_rows(m);
+                        }
+                    }
+                }
+                nbox = __shfl_sync(0xffffffffu, nbox, 0);
+                __syncwarp();
                 if (lane < nbox) {
-                    const int e = stack_entry(st, lane * 8);
-                    box_row = (int)(st.aoff[e] / d_in) + (lane * 8 - st.kb[e]);
+                    const int4 bx = abox[lane];
+                    box_j = bx.x;
+                    box_row = bx.y;
+                    box_m = bx.z;
                 }
             } else {
                 for (int j = lane; j < kKMax; j += 32) {
@@ -415,13 +474,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_shrink(const __grid_consta
                 }
                 __syncwarp();
             }
-            const uint32_t tx = (uint32_t)kAtom + (use_tma ? (uint32_t)nbox * 1024u : 0u);
+            const uint32_t tx = (uint32_t)kAtom + (use_tma ? (uint32_t)st.ktot * 128u : 0u);
             for (int kb = 0; kb < n_kb; ++kb, ++it) {
-                const int s = it % kShrinkStages;
-                const uint32_t ph = (it / kShrinkStages) & 1;
+                const int s = it % n_st;
+                const uint32_t ph = (it / n_st) & 1;
+                TC_STAMP(0, it, 0);
                 if (!warp_wait(&empty_bar[s], ph ^ 1, &abort_flag, p.err))
                     goto done;
-                unsigned char *xs = sm + s * ShrinkSmem::kStage;
+                TC_STAMP(0, it, 1);
+                unsigned char *xs = sm + s * p.s_stage;
                 unsigned char *as = xs + kAtom;
                 if (lane == 0) {
                     mbar_arrive_expect_tx(&full_bar[s], tx);
@@ -430,7 +491,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_shrink(const __grid_consta
                 __syncwarp();
                 if (use_tma) {
                     if (lane < nbox)
-                        tma_load_2d(as + lane * 1024, &p.map_a, &full_bar[s], kb * kBK, box_row);
+                        tma_load_2d(as + box_j * 128, &p.map_a[box_m], &full_bar[s], kb * kBK, box_row);
                 } else {
                     // stacked row j, 16-byte chunk c; rows past the stack feed only
                     // accumulator columns that are never stored
@@ -441,6 +502,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_shrink(const __grid_consta
                         cp_async16(abase + sw128_off(j, c), in ? p.pool.A + arow[j] + col : p.pool.A, in);
                 }
                 cp_async_arrive(&full_bar[s]);
+                TC_STAMP(0, it, 2);
             }
         }
     } else if (warp == 1) {
@@ -451,29 +513,35 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_shrink(const __grid_consta
             const Group gr = p.groups[u];
             warp_build_stack(p, gr.item, st, false);
             const int kpad = st.kpad;
+            const bool a_tma = st.a_tma && p.a_tma;
             const int b = t & 1;
             if (!warp_wait(&acc_empty[b], ((t >> 1) & 1) ^ 1, &abort_flag, p.err))
                 goto done;
             tc_fence_after();
             const uint32_t idesc = idesc_bf16(kBM, kpad > 0 ? kpad : 16);
             for (int kb = 0; kb < n_kb; ++kb, ++it) {
-                const int s = it % kShrinkStages;
-                const uint32_t ph = (it / kShrinkStages) & 1;
+                const int s = it % n_st;
+                const uint32_t ph = (it / n_st) & 1;
+                TC_STAMP(1, it, 0);
                 if (!warp_wait(&full_bar[s], ph, &abort_flag, p.err))
                     goto done;
-                fence_async_smem();
+                TC_STAMP(1, it, 1);
+                if (!a_tma)
+                    fence_async_smem();         // A written by cp.async (generic proxy)
                 tc_fence_after();
                 if (lane == 0 && kpad > 0) {
-                    const uint32_t xa = smem_u32(sm + s * ShrinkSmem::kStage);
+                    const uint32_t xa = smem_u32(sm + s * p.s_stage);
                     const uint32_t aa = xa + kAtom;
 #pragma unroll
                     for (int k = 0; k < kBK / 16; ++k)
                         tc_mma(tmem + b * 128, sw128_desc(xa + k * 32), sw128_desc(aa + k * 32), idesc,
                                (kb > 0 || k > 0) ? 1u : 0u);
+                    TC_STAMP(1, it, 2);
                 }
                 __syncwarp();
                 if (lane == 0)
                     tc_commit(&empty_bar[s]);
+                TC_STAMP(1, it, 3);
                 __syncwarp();
             }
             if (lane == 0)
@@ -533,34 +601,36 @@ done:
     }
 }
 
+
 // ============================================================ expand kernel
 //
 // Unit = (tile, 128-output slice).  D[128 x 128] = V_tile B_stack[slice]^T over
 // the stacked rank (V staged once per tile as bf16 with the scales folded in);
-// the epilogue adds D to the y tile (TMA-loaded) in shared memory and a TMA
-// store writes the tile back (a ragged tile: plain coalesced stores of its rows).
-struct ExpandSmem {
-    static constexpr int kV = 2 * kAtom;                 // V: 128 rows x up to 128 ranks
-    static constexpr int kB = 2 * kAtom;                 // B: 128 outputs x up to 128 ranks
-    static constexpr int kY = kBM * kBN * 2;             // y: 128 rows x 128 outputs (two 64-column atoms)
-    static constexpr int kOffB = kV;
-    static constexpr int kOffY = kOffB + kExpandBStages * kB;
-    static constexpr int kBytes = kOffY + kExpandYStages * kY;
-};
+// the epilogue adds D to the y tile (TMA-loaded; threads only read it, so a
+// stage goes back to the producer as soon as it is read) and each epilogue
+// warp stores its rows through a small staging area with coalesced 16-byte
+// stores.
+//
+// Shared memory is laid out at run time: V and every B stage take one 16 KB
+// atom per 64 stacked ranks the call can carry (1 or 2), and the y stages fill
+// the rest (up to kMaxYStages), so a rank-64 call keeps five 32 KB y tiles in flight.
+constexpr int kY = kBM * kBN * 2;                  // y: 128 rows x 128 outputs (two 64-column atoms)
+constexpr int kMaxYStages = 6;
+constexpr int kStaging = 8 * 2048;                 // per epilogue warp: 32 rows x 32 outputs of bf16
 
-__global__ void __launch_bounds__(kTcThreads, 1) k_tc_expand(const __grid_constant__ TcArgs p)
+__global__ void __launch_bounds__(kExpandThreads, 1) k_tc_expand(const __grid_constant__ TcArgs p)
 {
     extern __shared__ __align__(1024) unsigned char sm_dyn[];
     unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(sm_dyn) + 1023) & ~(uintptr_t)1023);
     __shared__ __align__(8) uint64_t b_full[kExpandBStages], b_empty[kExpandBStages];
-    __shared__ __align__(8) uint64_t y_full[kExpandYStages], y_empty[kExpandYStages];
+    __shared__ __align__(8) uint64_t y_full[kMaxYStages], y_empty[kMaxYStages];
     __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2];
-    __shared__ __align__(8) uint64_t v_full, v_empty, ep_bar;
-    __shared__ __align__(8) StackSm stk[kTcThreads / 32];
+    __shared__ __align__(8) uint64_t v_full, v_empty;
+    __shared__ __align__(8) StackSm stk[kExpandThreads / 32];
     __shared__ long long cb_off[kKMax / 8];  // producer: B element offset of stacked 8-rank chunk c in output row 0
     __shared__ int cb_r[kKMax / 8];          // its row stride (the adapter's rank); 0 = padding chunk
-    __shared__ int vsrc[4][kKMax / 8];       // epilogue warp q: V column of stacked chunk c (-1: zero)
-    __shared__ float vsc[4][kKMax / 8];      // and its adapter's scale
+    __shared__ int vsrc[8][kKMax / 8];       // epilogue warp e: V column of stacked chunk c (-1: zero)
+    __shared__ float vsc[8][kKMax / 8];      // and its adapter's scale
     __shared__ uint32_t tmem_base;
     __shared__ int abort_flag;
 
@@ -570,23 +640,28 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_expand(const __grid_consta
     const int64_t n_units = (int64_t)p.hdr->n_groups * n_ns;
     const int G = gridDim.x;
     const int64_t u0 = (int64_t)blockIdx.x * n_units / G, u1 = (int64_t)(blockIdx.x + 1) * n_units / G;
+    const int n_ys = p.e_ystages;
+    const int szB = p.e_natoms * kAtom;                 // one B stage (and V)
+    unsigned char *const smV = sm;
+    unsigned char *const smB = sm + szB;
+    unsigned char *const smS = smB + kExpandBStages * szB;   // epilogue warps' output staging
+    unsigned char *const smY = smS + kStaging;
 
     if (tid == 0) {
         for (int s = 0; s < kExpandBStages; ++s) {
-            mbar_init(&b_full[s], 32);       // 32 cp.async arrivals
+            mbar_init(&b_full[s], 33);       // lane 0 (expect_tx or plain) + 32 cp.async arrivals
             mbar_init(&b_empty[s], 1);       // MMA commit
         }
-        for (int s = 0; s < kExpandYStages; ++s) {
+        for (int s = 0; s < kMaxYStages; ++s) {
             mbar_init(&y_full[s], 1);        // expect_tx
-            mbar_init(&y_empty[s], 1);       // the epilogue thread that stored the tile
+            mbar_init(&y_empty[s], 8);       // epilogue warps: the tile is stored
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&acc_full[b], 1);
-            mbar_init(&acc_empty[b], 4);
+            mbar_init(&acc_empty[b], 8);     // epilogue warps
         }
-        mbar_init(&v_full, 4);               // epilogue warps, after staging V
+        mbar_init(&v_full, 8);               // epilogue warps, after staging V
         mbar_init(&v_empty, 1);              // MMA commit after a tile's last unit
-        mbar_init(&ep_bar, 4);               // the epilogue warps meet (y tile complete in shared memory)
         abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -598,12 +673,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_expand(const __grid_consta
     const uint32_t tmem = tmem_base;
 
     if (warp == 0) {
-        // ------------------------------------------------ producer: y tiles (TMA), B slices (cp.async)
+        // ------------------------------------------------ producer: y tiles and B slices
         StackSm &st = stk[0];
         int it = 0;
         int64_t prev_tile = -1;
         int nch = 0, o_l = 0, c_l = 0, dq = 0, dr = 0;
         int p0 = 0;
+        int bx_m = 0, bx_y = 0, bx_dst = 0, bx_two = 0;   // this lane's B box (TMA path, lane < n)
         for (int64_t u = u0; u < u1; ++u, ++it) {
             const int tile = (int)(u / n_ns), ns = (int)(u - (int64_t)tile * n_ns);
             if (tile != prev_tile) {
@@ -611,105 +687,171 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_expand(const __grid_consta
                 p0 = gr.p0;
                 warp_build_stack(p, gr.item, st, false);
                 prev_tile = tile;
-                if (lane < kKMax / 8) {
-                    const int k = lane * 8;
-                    long long o = 0;
-                    int rr = 0;
-                    if (k < st.ktot) {
-                        const int e = stack_entry(st, k);
-                        o = st.boff[e] + (k - st.kb[e]);
-                        rr = st.r[e];
+                if (st.b_tma) {
+                    if (lane < st.n) {
+                        const int r = st.r[lane];
+                        bx_m = b_map(r);
+                        bx_y = (int)(st.boff[lane] / r);
+                        bx_dst = st.kb[lane] * 256;
+                        bx_two = r == 128;
                     }
-                    cb_off[lane] = o;
-                    cb_r[lane] = rr;
-                }
-                __syncwarp();
-                // this lane walks chunk indices lane, lane + 32, ... of the (output, chunk) grid
-                nch = st.kpad >> 3;
-                if (nch > 0) {
-                    o_l = lane / nch;
-                    c_l = lane - o_l * nch;
-                    dq = 32 / nch;
-                    dr = 32 - dq * nch;
+                } else {
+                    if (lane < kKMax / 8) {
+                        const int k = lane * 8;
+                        long long o = 0;
+                        int rr = 0;
+                        if (k < st.ktot) {
+                            const int e = stack_entry(st, k);
+                            o = st.boff[e] + (k - st.kb[e]);
+                            rr = st.r[e];
+                        }
+                        cb_off[lane] = o;
+                        cb_r[lane] = rr;
+                    }
+                    __syncwarp();
+                    // this lane walks chunk indices lane, lane + 32, ... of the (output, chunk) grid
+                    nch = st.kpad >> 3;
+                    if (nch > 0) {
+                        o_l = lane / nch;
+                        c_l = lane - o_l * nch;
+                        dq = 32 / nch;
+                        dr = 32 - dq * nch;
+                    }
                 }
             }
             const int o0 = ns * kBN;
-            const int sy = it % kExpandYStages;
-            if (!warp_wait(&y_empty[sy], ((it / kExpandYStages) & 1) ^ 1, &abort_flag, p.err))
+            const int sy = it % n_ys;
+            TC_STAMP(0, it, 0);
+            if (!warp_wait(&y_empty[sy], ((it / n_ys) & 1) ^ 1, &abort_flag, p.err))
                 goto done;
-            unsigned char *ys = sm + ExpandSmem::kOffY + sy * ExpandSmem::kY;
+            TC_STAMP(0, it, 1);
+            unsigned char *ys = smY + sy * kY;
             if (lane == 0) {
-                mbar_arrive_expect_tx(&y_full[sy], ExpandSmem::kY);
+                mbar_arrive_expect_tx(&y_full[sy], kY);
                 tma_load_2d(ys, &p.map_y, &y_full[sy], o0, p0);
                 tma_load_2d(ys + kAtom, &p.map_y, &y_full[sy], o0 + 64, p0);
             }
             const int sb = it % kExpandBStages;
             if (!warp_wait(&b_empty[sb], ((it / kExpandBStages) & 1) ^ 1, &abort_flag, p.err))
                 goto done;
-            const uint32_t bbase = smem_u32(sm + ExpandSmem::kOffB + sb * ExpandSmem::kB);
-            // output o of the slice, 16-byte chunk c of the stacked rank axis (atom c / 8);
-            // padding chunks and outputs past d_out are zero-filled
-            int o = o_l, c = c_l;
-            for (int idx = lane; idx < kBN * nch; idx += 32) {
-                const int rr = cb_r[c];
-                const bool ok = rr > 0 && o0 + o < d_out;
-                const __nv_bfloat16 *src = ok ? p.pool.B + cb_off[c] + (long long)(o0 + o) * rr : p.pool.B;
-                cp_async16(bbase + (c >> 3) * kAtom + sw128_off(o, c & 7), src, ok);
-                c += dr;
-                o += dq;
-                if (c >= nch) {
-                    c -= nch;
-                    ++o;
+            TC_STAMP(0, it, 2);
+            unsigned char *bs = smB + sb * szB;
+            if (st.b_tma) {
+                // one box per entry (two for rank 128): outputs o0 .. o0 + 127 of its B, in the
+                // entry's own region (kb * 256 bytes in), swizzled to its row width; rows past
+                // d_out feed only accumulator columns that are never stored
+                if (lane == 0)
+                    mbar_arrive_expect_tx(&b_full[sb], (uint32_t)st.ktot * 256u);
+                __syncwarp();
+                if (lane < st.n) {
+                    tma_load_2d(bs + bx_dst, &p.map_b[bx_m], &b_full[sb], 0, bx_y + o0);
+                    if (bx_two)
+                        tma_load_2d(bs + bx_dst + kAtom, &p.map_b[bx_m], &b_full[sb], 64, bx_y + o0);
+                }
+            } else {
+                if (lane == 0)
+                    mbar_arrive(&b_full[sb]);
+                // cp.async: output o of the slice, 16-byte chunk c of the stacked rank axis
+                // (atom c / 8); padding chunks and outputs past d_out are zero-filled
+                const uint32_t bbase = smem_u32(bs);
+                int o = o_l, c = c_l;
+                for (int idx = lane; idx < kBN * nch; idx += 32) {
+                    const int rr = cb_r[c];
+                    const bool ok = rr > 0 && o0 + o < d_out;
+                    const __nv_bfloat16 *src = ok ? p.pool.B + cb_off[c] + (long long)(o0 + o) * rr : p.pool.B;
+                    cp_async16(bbase + (c >> 3) * kAtom + sw128_off(o, c & 7), src, ok);
+                    c += dr;
+                    o += dq;
+                    if (c >= nch) {
+                        c -= nch;
+                        ++o;
+                    }
                 }
             }
             cp_async_arrive(&b_full[sb]);
+            TC_STAMP(0, it, 3);
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
+        // Per tile, the operand descriptors of every 16-rank step (at most 8) are worked
+        // out once: V's are absolute, B's relative to the stage (the stage base, >> 4, is
+        // added to the start-address field per unit).
         StackSm &st = stk[1];
         int it = 0, vt = 0;
         int64_t prev_tile = -1;
+        int nsteps = 0;
+        bool b_tma = false;
+        uint64_t ad[kKMax / 16], bd[kKMax / 16];
+        const uint32_t va = smem_u32(smV);
         for (int64_t u = u0; u < u1; ++u, ++it) {
             const int tile = (int)(u / n_ns);
             if (tile != prev_tile) {
                 warp_build_stack(p, p.groups[tile].item, st, false);
                 prev_tile = tile;
+                b_tma = st.b_tma;
+                nsteps = st.kpad / 16;
+                int e = 0;
+#pragma unroll
+                for (int k16 = 0; k16 < kKMax / 16; ++k16) {
+                    const int k = k16 * 16;
+                    ad[k16] = sw128_desc(va + (k >> 6) * kAtom + ((k & 63) >> 4) * 32);
+                    if (b_tma) {
+                        // B: entry e's region at kb_e * 256 bytes, swizzled to its rank
+                        while (e + 1 < st.n && k >= st.kb[e + 1])
+                            ++e;
+                        const int kl = k - st.kb[e];
+                        const int re = st.r[e];
+                        const uint32_t reg = st.kb[e] * 256;
+                        bd[k16] = re >= 64 ? sw128_desc(reg + (kl >> 6) * kAtom + ((kl & 63) >> 4) * 32)
+                                           : (re == 32 ? sw64_desc(reg + (kl >> 4) * 32) : sw32_desc(reg));
+                    } else {
+                        bd[k16] = sw128_desc((k >> 6) * kAtom + ((k & 63) >> 4) * 32);
+                    }
+                }
                 if (!warp_wait(&v_full, vt & 1, &abort_flag, p.err))
                     goto done;
                 ++vt;
             }
             const int b = it & 1;
+            TC_STAMP(1, it, 0);
             if (!warp_wait(&acc_empty[b], ((it >> 1) & 1) ^ 1, &abort_flag, p.err))
                 goto done;
+            TC_STAMP(1, it, 1);
             const int sb = it % kExpandBStages;
             if (!warp_wait(&b_full[sb], (it / kExpandBStages) & 1, &abort_flag, p.err))
                 goto done;
-            fence_async_smem();
+            TC_STAMP(1, it, 2);
+            if (!b_tma)
+                fence_async_smem();             // B written by cp.async (generic proxy)
             tc_fence_after();
             if (lane == 0) {
-                const uint32_t va = smem_u32(sm);
-                const uint32_t ba = smem_u32(sm + ExpandSmem::kOffB + sb * ExpandSmem::kB);
+                const uint64_t bbase = (smem_u32(smB + sb * szB) >> 4) & 0x3FFFu;
                 const uint32_t idesc = idesc_bf16(kBM, kBN);
-                for (int k = 0; k < st.kpad / 16; ++k) {
-                    const uint32_t off = (k >> 2) * kAtom + (k & 3) * 32;
-                    tc_mma(tmem + b * 128, sw128_desc(va + off), sw128_desc(ba + off), idesc, k > 0 ? 1u : 0u);
-                }
+#pragma unroll
+                for (int k16 = 0; k16 < kKMax / 16; ++k16)
+                    if (k16 < nsteps)
+                        tc_mma(tmem + b * 128, ad[k16], bd[k16] + bbase, idesc, k16 > 0 ? 1u : 0u);
+                TC_STAMP(1, it, 3);
                 tc_commit(&b_empty[sb]);
                 tc_commit(&acc_full[b]);
                 const bool last_of_tile = u + 1 >= u1 || (int)((u + 1) / n_ns) != tile;
                 if (last_of_tile)
                     tc_commit(&v_empty);
+                TC_STAMP(1, it, 4);
             }
             __syncwarp();
         }
     } else {
         // ------------------------------------------------ epilogue: V staging, y += D, store
+        // Eight warps: warp w reads TMEM lane quarter w % 4 (rows 32 (w % 4) ..) and
+        // owns output half h (one 64-column y atom) of every unit.
+        const int e8 = warp - 2;                // 0..7
         const int q = warp & 3;
+        const int h = e8 >> 2;
         const int row = q * 32 + lane;
-        const int et = tid - 64;                // 0..127 over the epilogue warps
+        const int et = tid - 64;                // 0..255 over the epilogue warps
         StackSm &st = stk[warp];
-        int it = 0, vt = 0, pending = -1;
-        uint32_t ep_uses = 0;
+        int it = 0, vt = 0;
         int64_t prev_tile = -1;
         Group gr = {0, 0, 0, 0};
         for (int64_t u = u0; u < u1; ++u, ++it) {
@@ -727,22 +869,25 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_expand(const __grid_consta
                         c = st.slot[e] * p.slot_stride + (k - st.kb[e]);
                         sc = st.s[e];
                     }
-                    vsrc[q][lane] = c;
-                    vsc[q][lane] = sc;
+                    vsrc[e8][lane] = c;
+                    vsc[e8][lane] = sc;
                 }
                 __syncwarp();
                 // wait until the MMAs of the previous tile stopped reading V
                 if (vt > 0 && !warp_wait(&v_empty, (vt - 1) & 1, &abort_flag, p.err))
                     goto done;
-                // V[row][stacked k] = bf16(s_e * V_e[row][k - kb_e]), zero outside the tile's rows and the stack
-                const bool valid = et < gr.cnt;
-                const float *vrow = p.V + (int64_t)(gr.p0 + (valid ? et : 0)) * p.ldv;
-                const uint32_t vbase = smem_u32(sm);
-                for (int c = 0; c < st.kpad / 8; ++c) {
-                    const int col = vsrc[q][c];
+                // V[vr][stacked k] = bf16(s_e * V_e[vr][k - kb_e]), zero outside the tile's rows and
+                // the stack; thread et stages row et % 128, stacked ranks 64 (et / 128) .. + 63
+                const int vr = et & 127, vh = et >> 7;
+                const bool valid = vr < gr.cnt;
+                const float *vrow = p.V + (int64_t)(gr.p0 + (valid ? vr : 0)) * p.ldv;
+                const uint32_t vbase = smem_u32(smV) + vh * kAtom;
+                const int c_end = min(st.kpad / 8, vh * 8 + 8);
+                for (int c = vh * 8; c < c_end; ++c) {
+                    const int col = vsrc[e8][c];
                     uint32_t w[4] = {0u, 0u, 0u, 0u};
                     if (valid && col >= 0) {
-                        const float sc = vsc[q][c];
+                        const float sc = vsc[e8][c];
                         const float4 a = *reinterpret_cast<const float4 *>(vrow + col);
                         const float4 bq = *reinterpret_cast<const float4 *>(vrow + col + 4);
                         const __nv_bfloat162 h0 = __floats2bfloat162_rn(sc * a.x, sc * a.y);
@@ -754,7 +899,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_expand(const __grid_consta
                         w[2] = *reinterpret_cast<const uint32_t *>(&h2);
                         w[3] = *reinterpret_cast<const uint32_t *>(&h3);
                     }
-                    st_shared_v4(vbase + (c >> 3) * kAtom + sw128_off(et, c & 7), w[0], w[1], w[2], w[3]);
+                    st_shared_v4(vbase + sw128_off(vr, c & 7), w[0], w[1], w[2], w[3]);
                 }
                 fence_async_smem();
                 __syncwarp();
@@ -763,94 +908,87 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_expand(const __grid_consta
                 ++vt;
             }
             const int b = it & 1;
-            const int sy = it % kExpandYStages;
+            const int sy = it % n_ys;
+            if (warp == 2)
+                TC_STAMP(2, it, 0);
             if (!warp_wait(&acc_full[b], (it >> 1) & 1, &abort_flag, p.err))
                 goto done;
-            if (!warp_wait(&y_full[sy], (it / kExpandYStages) & 1, &abort_flag, p.err))
+            if (warp == 2)
+                TC_STAMP(2, it, 1);
+            if (!warp_wait(&y_full[sy], (it / n_ys) & 1, &abort_flag, p.err))
                 goto done;
+            if (warp == 2)
+                TC_STAMP(2, it, 2);
             tc_fence_after();
             const int o0 = ns * kBN;
-            unsigned char *ys = sm + ExpandSmem::kOffY + sy * ExpandSmem::kY;
-            const uint32_t ysa = smem_u32(ys);
-#pragma unroll 1
-            for (int c0 = 0; c0 < kBN; c0 += 32) {
-                float d[32];
-                tmem_ld32(tmem + b * 128 + ((uint32_t)(q * 32) << 16) + c0, d);
-                if (st.kpad == 0) {   // no valid adapter: no MMA ran, y is stored unchanged
+            const uint32_t atom = smem_u32(smY + sy * kY) + h * kAtom;
+            // this row's 64 y values (eight 16-byte chunks); the stage is then free again:
+            // threads only read the TMA-loaded tiles, never write them
+            uint32_t yw[8][4];
 #pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        d[i] = 0.f;
-                }
-                // four 16-byte chunks of this row's y: atom c0 / 64, chunks (c0 % 64) / 8 ..
-                const uint32_t atom = ysa + (c0 >> 6) * kAtom;
-#pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                    const uint32_t addr = atom + sw128_off(row, ((c0 & 63) >> 3) + h);
-                    uint32_t yw[4];
-                    ld_shared_v4(addr, yw);
-                    uint32_t ow[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 yf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&yw[e]));
-                        const __nv_bfloat162 r2 =
-                            __floats2bfloat162_rn(yf.x + d[h * 8 + 2 * e], yf.y + d[h * 8 + 2 * e + 1]);
-                        ow[e] = *reinterpret_cast<const uint32_t *>(&r2);
-                    }
-                    st_shared_v4(addr, ow[0], ow[1], ow[2], ow[3]);
-                }
-            }
-            tc_fence_before();
-            fence_async_smem();                 // this thread's y writes, before the TMA store reads them
+            for (int c = 0; c < 8; ++c)
+                ld_shared_v4(atom + sw128_off(row, c), yw[c]);
             __syncwarp();
-            if (lane == 0) {
+            if (lane == 0)
+                mbar_arrive(&y_empty[sy]);
+            if (warp == 2)
+                TC_STAMP(2, it, 3);
+            uint32_t d[64];
+            tmem_ld64(tmem + b * 128 + ((uint32_t)(q * 32) << 16) + h * 64, d);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
                 mbar_arrive(&acc_empty[b]);
-                mbar_arrive(&ep_bar);
-            }
-            if (!warp_wait(&ep_bar, ep_uses & 1, &abort_flag, p.err))
-                goto done;
-            ++ep_uses;
-            if (gr.cnt == kBM) {
-                // full tile: one thread stores it; the stage is released once the store has read it
-                if (et == 0) {
-                    tma_store_2d(&p.map_y, ys, o0, gr.p0);
-                    tma_store_2d(&p.map_y, ys + kAtom, o0 + 64, gr.p0);
-                    bulk_commit();
-                    bulk_wait_read_1();
-                    if (pending >= 0)
-                        mbar_arrive(&y_empty[pending]);
-                    pending = sy;
+            if (warp == 2)
+                TC_STAMP(2, it, 4);
+            const bool none = st.kpad == 0;     // no valid adapter: no MMA ran, y is stored unchanged
+            uint32_t ow[8][4];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 yf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&yw[c][e]));
+                    const float d0 = none ? 0.f : __uint_as_float(d[c * 8 + 2 * e]);
+                    const float d1 = none ? 0.f : __uint_as_float(d[c * 8 + 2 * e + 1]);
+                    const __nv_bfloat162 r2 = __floats2bfloat162_rn(yf.x + d0, yf.y + d1);
+                    ow[c][e] = *reinterpret_cast<const uint32_t *>(&r2);
                 }
-            } else {
-                // ragged tile: the valid rows, 16 bytes per thread, 256 contiguous bytes per row
-                for (int idx = et; idx < gr.cnt * 16; idx += 128) {
-                    const int r = idx >> 4, ch = idx & 15;
-                    const int o = o0 + ch * 8;
-                    if (o < d_out) {
-                        uint32_t w[4];
-                        ld_shared_v4(ysa + (ch >> 3) * kAtom + sw128_off(r, ch & 7), w);
-                        *reinterpret_cast<uint4 *>(p.Y + (int64_t)(gr.p0 + r) * p.ldy + o) =
-                            make_uint4(w[0], w[1], w[2], w[3]);
+            }
+            if (warp == 2)
+                TC_STAMP(2, it, 5);
+            // store through this warp's 2 KB staging area, 32 columns at a time: rows of 64
+            // bytes (4 chunks, XOR-swizzled by row / 2), read back 4 lanes per row so every
+            // store instruction writes 8 rows x 64 contiguous bytes
+            const uint32_t stg = smem_u32(smS) + e8 * 2048;
+            const int n_rows = min(gr.cnt - q * 32, 32);
+#pragma unroll
+            for (int pass = 0; pass < 2; ++pass) {
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    st_shared_v4(stg + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4), ow[4 * pass + c][0],
+                                 ow[4 * pass + c][1], ow[4 * pass + c][2], ow[4 * pass + c][3]);
+                __syncwarp();
+                const int cc = lane & 3;
+                const int o = o0 + h * 64 + pass * 32 + cc * 8;
+                if (o < d_out) {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int rl = 8 * j + (lane >> 2);
+                        if (rl < n_rows) {
+                            uint32_t w[4];
+                            ld_shared_v4(stg + rl * 64 + ((cc ^ ((rl >> 1) & 3)) << 4), w);
+                            *reinterpret_cast<uint4 *>(p.Y + (int64_t)(gr.p0 + q * 32 + rl) * p.ldy + o) =
+                                make_uint4(w[0], w[1], w[2], w[3]);
+                        }
                     }
                 }
                 __syncwarp();
-                if (lane == 0)
-                    mbar_arrive(&ep_bar);
-                if (!warp_wait(&ep_bar, ep_uses & 1, &abort_flag, p.err))
-                    goto done;
-                ++ep_uses;
-                if (et == 0) {
-                    bulk_wait_read_0();
-                    if (pending >= 0)
-                        mbar_arrive(&y_empty[pending]);
-                    pending = -1;
-                    mbar_arrive(&y_empty[sy]);
-                }
             }
+            if (warp == 2)
+                TC_STAMP(2, it, 6);
         }
     }
 done:
-    if (tid == 64)
-        bulk_wait_all();                        // the last TMA stores have landed
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
@@ -902,7 +1040,7 @@ int sm_count()
 
 // attr_set: this kernel's per-device "shared-memory opt-in done" flags (one
 // array per kernel: the kernels share a type, so they cannot share the flags)
-cudaError_t launch_tc(void (*kernel)(TcArgs), bool *attr_set, const TcArgs &a, int smem, int units_hint,
+cudaError_t launch_tc(void (*kernel)(TcArgs), bool *attr_set, const TcArgs &a, int threads, int smem, int grid,
                       cudaStream_t s)
 {
     int dev = 0;
@@ -916,12 +1054,9 @@ cudaError_t launch_tc(void (*kernel)(TcArgs), bool *attr_set, const TcArgs &a, i
         if (dev >= 0 && dev < 64)
             attr_set[dev] = true;
     }
-    int grid = sm_count();
-    if (units_hint > 0 && units_hint < grid)
-        grid = units_hint;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(kTcThreads);
+    cfg.blockDim = dim3(threads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     return cudaLaunchKernelEx(&cfg, kernel, a);
@@ -931,7 +1066,7 @@ cudaError_t launch_tc(void (*kernel)(TcArgs), bool *attr_set, const TcArgs &a, i
 
 bool tc_encode_a(TcArgs &a, const void *A, int64_t A_elems, int32_t d_in)
 {
-    // the A pool as a [A_elems / d_in, d_in] matrix, boxes of 64 columns x 8 rows
+    // the A pool as a [A_elems / d_in, d_in] matrix, boxes of 64 columns x 64, 32 and 8 rows
     a.a_tma = 0;
     const int64_t rows = A_elems / d_in;
     if (rows < 1 || rows > 0x7fffffffLL)
@@ -941,14 +1076,43 @@ bool tc_encode_a(TcArgs &a, const void *A, int64_t A_elems, int32_t d_in)
         return false;
     const cuuint64_t dims[2] = {(cuuint64_t)d_in, (cuuint64_t)rows};
     const cuuint64_t strides[1] = {(cuuint64_t)d_in * 2};
-    const cuuint32_t box[2] = {64, 8};
     const cuuint32_t estr[2] = {1, 1};
-    if (fn(&a.map_a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(A), dims, strides, box, estr,
-           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-        return false;
+    for (int i = 0; i < 3; ++i) {
+        const cuuint32_t box[2] = {64, (cuuint32_t)abox_rows(i)};
+        if (fn(&a.map_a[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(A), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return false;
+    }
     a.a_tma = 1;
     return true;
+}
+
+bool tc_encode_b(TcArgs &a, const void *B, int64_t B_elems)
+{
+    // the B pool as [B_elems / r, r] for r = 16, 32, 64, 128: boxes of 128 rows
+    // (outputs) x min(r, 64) columns, swizzled to the row width
+    a.b_tma = 0;
+    EncodeTiledFn fn = encode_fn();
+    if (!fn)
+        return false;
+    for (int m = 0; m < 4; ++m) {
+        const int r = 16 << m;
+        const int64_t rows = B_elems / r;
+        if (rows < 1 || rows > 0x7fffffffLL)
+            continue;
+        const cuuint64_t dims[2] = {(cuuint64_t)r, (cuuint64_t)rows};
+        const cuuint64_t strides[1] = {(cuuint64_t)r * 2};
+        const cuuint32_t box[2] = {(cuuint32_t)(r < 64 ? r : 64), 128};
+        const cuuint32_t estr[2] = {1, 1};
+        const CUtensorMapSwizzle sw = r == 16 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                    : (r == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B);
+        if (fn(&a.map_b[m], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(B), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS)
+            a.b_tma |= 1 << m;
+    }
+    return a.b_tma != 0;
 }
 
 bool tc_encode_x(TcArgs &a, const void *X, int32_t N, int32_t d_in, int64_t ldx)
@@ -961,17 +1125,70 @@ bool tc_encode_y(TcArgs &a, const void *Y, int32_t N, int32_t d_out, int64_t ldy
     return encode_rows(&a.map_y, Y, N, d_out, ldy);
 }
 
-cudaError_t launch_tc_shrink(const TcArgs &a, int max_tiles, cudaStream_t s)
+cudaError_t launch_tc_shrink(const TcArgs &args, int max_tiles, int kk, cudaStream_t s)
 {
+    // a stage: the x atom and round16(kk) A rows of 128 bytes; two CTAs per SM
     static bool attr_set[64] = {};
-    return launch_tc(k_tc_shrink, attr_set, a, ShrinkSmem::kBytes + 1024, max_tiles, s);
+    TcArgs a = args;
+    const int a_rows = (kk + 15) & ~15;
+    a.s_stage = kAtom + a_rows * 128;
+    a.s_stages = kk > 64 ? 3 : 4;
+    const int smem = a.s_stages * a.s_stage + 1024;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+        // the largest layout: 4 stages at rank 64 or 3 at rank 128 (same size)
+        if ((e = cudaFuncSetAttribute(k_tc_shrink, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      4 * (kAtom + 64 * 128) + 1024)) != cudaSuccess)
+            return e;
+        attr_set[dev] = true;
+    }
+    int grid = 2 * sm_count();
+    if (max_tiles > 0 && max_tiles < grid)
+        grid = max_tiles;
+    bool done = true;
+    return launch_tc(k_tc_shrink, &done, a, kTcThreads, smem, grid, s);
 }
 
-cudaError_t launch_tc_expand(const TcArgs &a, cudaStream_t s)
+cudaError_t launch_tc_expand(const TcArgs &args, int kk, cudaStream_t s)
 {
+    // shared memory: V and two B stages of one atom per 64 stacked ranks, then as
+    // many 32 KB y stages as fit (at least two)
     static bool attr_set[64] = {};
-    return launch_tc(k_tc_expand, attr_set, a, ExpandSmem::kBytes + 1024, 0, s);
+    int dev = 0, optin = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    if ((e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess)
+        return e;
+    cudaFuncAttributes fa;
+    if ((e = cudaFuncGetAttributes(&fa, k_tc_expand)) != cudaSuccess)
+        return e;
+    TcArgs a = args;
+    a.e_natoms = kk > 64 ? 2 : 1;
+    const int fixed = (1 + kExpandBStages) * a.e_natoms * kAtom + kStaging + 1024;
+    const int room = optin - (int)fa.sharedSizeBytes - fixed;
+    a.e_ystages = room / kY < kMaxYStages ? room / kY : kMaxYStages;
+    if (a.e_ystages < 2)
+        return cudaErrorInvalidConfiguration;
+    const int smem = fixed + a.e_ystages * kY;
+    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+        if ((e = cudaFuncSetAttribute(k_tc_expand, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      optin - (int)fa.sharedSizeBytes)) != cudaSuccess)
+            return e;
+        attr_set[dev] = true;
+    }
+    bool done = true;
+    return launch_tc(k_tc_expand, &done, a, kExpandThreads, smem, sm_count(), s);
 }
 
 }  // namespace lora
 
+#ifdef LORA_TC_TRACE
+extern "C" LORA_API int lora_debug_tc_trace(unsigned long long *host, int n)
+{
+    return (int)cudaMemcpyFromSymbol(host, lora::g_tc_trace, sizeof(unsigned long long) * (size_t)n);
+}
+#endif
