@@ -92,6 +92,16 @@ def rank_seed(workload_index: int, rank: int, set_index: int) -> int:
     return workload_index + 1000 * rank + 100000 * set_index
 
 
+def job_time_and_throughput(ms_local: float, steps: int, tokens_per_step_per_rank: int, world: int,
+                            dist, device=None):
+    """Whole-job numbers of a weak-scaling run: the step time is the slowest rank's
+    (max over ranks of its device-timed total / steps); the throughput counts the
+    tokens every rank processed in that time."""
+    ms = max_over_ranks(ms_local, dist, device)
+    ms_per_step = ms / steps
+    return ms_per_step, world * tokens_per_step_per_rank / (ms_per_step * 1e-3)
+
+
 # ----------------------------------------------------------------------------
 # clocks
 # ----------------------------------------------------------------------------
@@ -323,8 +333,7 @@ def run_ours(args):
         dist.barrier()
     clocks.stop()
     ms_local = e0.elapsed_time(e1)
-    ms = max_over_ranks(ms_local, dist, dev)
-    ms_per_step = ms / K
+    ms_per_step, job_tokens_s = job_time_and_throughput(ms_local, K, tokens_per_step, world, dist, dev)
 
     # end to end through the public call, host buffers, copies inside the timed region
     e2e = run_e2e(args, sets[0], ws_map, stream, dist, dev, world)
@@ -339,7 +348,7 @@ def run_ours(args):
             "scope": "whole step, algorithmic bytes per step / step time",
             "algorithmic_bytes_per_step": cost.bytes}
     out = {
-        "metric": METRIC, "value": round(world * tokens_per_step / t_step, 1), "unit": "tokens/s",
+        "metric": METRIC, "value": round(job_tokens_s, 1), "unit": "tokens/s",
         "n_gpus": world, "steps": K, "warmup": max(args.warmup, 3), "ms_per_step": round(ms_per_step, 6),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded; random-init adapters of the stated shapes)",
