@@ -94,17 +94,26 @@ __device__ __forceinline__ uint32_t n_clusters_x()
 __device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
 __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// 16-byte asynchronous copy global -> shared (both 16-byte aligned), and the wait for all of them
+__device__ __forceinline__ void cp_async16(void *dst, const void *src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)), "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 #ifdef LORA_PHASE_TIMING
 // Development aid: per-CTA %globaltimer stamps at phase boundaries of the first item.
-__device__ unsigned long long g_phase[65536 * 12];
+__device__ unsigned long long g_phase[65536 * 16];
 #define PHASE(i)                                                                     \
     do {                                                                             \
         if (threadIdx.x == 0 && first && blockIdx.x < 65536) {                       \
             unsigned long long t_;                                                   \
             asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                   \
-            g_phase[blockIdx.x * 12 + (i)] = t_;                                     \
+            g_phase[blockIdx.x * 16 + (i)] = t_;                                     \
         }                                                                            \
     } while (0)
 #else
@@ -169,47 +178,71 @@ __device__ __forceinline__ void shrink_tiles(const __nv_bfloat16 *Aa, int d_in, 
 // (8 outputs each, from output o0): Y += s (V_hi + V_lo) B^T with NKB
 // 32-rank blocks; a batch's B fragments and y values are all requested
 // before its MMAs, and the V fragments are read from shared memory once.
-template <int NKB>
+// ST: B and y come from the staged copies in shared memory (bst: [Wo][r] from
+// output o0; yst: [kFT][Wo]), else from global memory.
+template <int NKB, bool ST>
 __device__ __forceinline__ void expand_tiles(const __nv_bfloat16 *Ba, int r, int o0, int n_ot, int warp, int nw,
-                                             const __nv_bfloat16 *vhi, const __nv_bfloat16 *vlo, int g, int qd,
-                                             __nv_bfloat16 *y0row, __nv_bfloat16 *y1row, bool row0, bool row1,
-                                             float sc)
+                                             const __nv_bfloat16 *vhi, const __nv_bfloat16 *vlo, int vs, int g,
+                                             int qd, __nv_bfloat16 *y0row, __nv_bfloat16 *y1row, bool row0,
+                                             bool row1, float sc, const __nv_bfloat16 *bst,
+                                             const __nv_bfloat16 *yst, int Wo)
 {
-    constexpr int TPB = NKB == 1 ? 8 : NKB == 2 ? 4 : 2;   // tiles per batch
-    constexpr bool HOIST = NKB <= 2;                       // keep V fragments in registers
+    constexpr int TPB = ST ? 16 : (NKB == 1 ? 8 : NKB == 2 ? 4 : 2);   // tiles per batch
+    constexpr bool HOIST = NKB <= 2;                                  // keep V fragments in registers
     uint4 h0[HOIST ? NKB : 1], h1[HOIST ? NKB : 1], l0[HOIST ? NKB : 1], l1[HOIST ? NKB : 1];
     if (HOIST) {
 #pragma unroll
         for (int kb = 0; kb < (HOIST ? NKB : 1); ++kb) {
             const int kc = kb * 32 + qd * 8;
-            h0[kb] = *reinterpret_cast<const uint4 *>(vhi + g * kVS + kc);
-            h1[kb] = *reinterpret_cast<const uint4 *>(vhi + (g + 8) * kVS + kc);
-            l0[kb] = *reinterpret_cast<const uint4 *>(vlo + g * kVS + kc);
-            l1[kb] = *reinterpret_cast<const uint4 *>(vlo + (g + 8) * kVS + kc);
+            h0[kb] = *reinterpret_cast<const uint4 *>(vhi + g * vs + kc);
+            h1[kb] = *reinterpret_cast<const uint4 *>(vhi + (g + 8) * vs + kc);
+            l0[kb] = *reinterpret_cast<const uint4 *>(vlo + g * vs + kc);
+            l1[kb] = *reinterpret_cast<const uint4 *>(vlo + (g + 8) * vs + kc);
         }
     }
     for (int ot0 = warp; ot0 < n_ot; ot0 += TPB * nw) {
-        uint4 bw[TPB][NKB];
-        __nv_bfloat162 ya[TPB], yb[TPB];
+        uint4 bw[ST ? 1 : TPB][NKB];
+        __nv_bfloat162 ya[ST ? 1 : TPB], yb[ST ? 1 : TPB];
+        if (!ST) {
 #pragma unroll
-        for (int t = 0; t < TPB; ++t) {
-            const int ot = ot0 + t * nw;
-            const bool ok = ot < n_ot;
-            const int ob = o0 + ot * 8;
-            const __nv_bfloat16 *brow = Ba + (int64_t)(ob + g) * r;
+            for (int t = 0; t < TPB; ++t) {
+                const int ot = ot0 + t * nw;
+                const bool ok = ot < n_ot;
+                const int ob = o0 + ot * 8;
+                const __nv_bfloat16 *brow = Ba + (int64_t)(ob + g) * r;
 #pragma unroll
-            for (int kb = 0; kb < NKB; ++kb) {
-                const int kc = kb * 32 + qd * 8;   // r and kc are multiples of 8
-                bw[t][kb] = (ok && kc < r) ? ld_stream(brow + kc) : make_uint4(0, 0, 0, 0);
+                for (int kb = 0; kb < NKB; ++kb) {
+                    const int kc = kb * 32 + qd * 8;   // r and kc are multiples of 8
+                    bw[ST ? 0 : t][kb] = (ok && kc < r) ? ld_stream(brow + kc) : make_uint4(0, 0, 0, 0);
+                }
+                const __nv_bfloat162 z = __floats2bfloat162_rn(0.f, 0.f);
+                ya[ST ? 0 : t] = (ok && row0) ? *reinterpret_cast<const __nv_bfloat162 *>(y0row + ob + 2 * qd) : z;
+                yb[ST ? 0 : t] = (ok && row1) ? *reinterpret_cast<const __nv_bfloat162 *>(y1row + ob + 2 * qd) : z;
             }
-            const __nv_bfloat162 z = __floats2bfloat162_rn(0.f, 0.f);
-            ya[t] = (ok && row0) ? *reinterpret_cast<const __nv_bfloat162 *>(y0row + ob + 2 * qd) : z;
-            yb[t] = (ok && row1) ? *reinterpret_cast<const __nv_bfloat162 *>(y1row + ob + 2 * qd) : z;
         }
 #pragma unroll
         for (int t = 0; t < TPB; ++t) {
             const int ot = ot0 + t * nw;
             if (ot < n_ot) {
+                const int ol = ot * 8;          // output offset within this CTA's chunk
+                uint4 bfr[NKB];
+                __nv_bfloat162 yva, yvb;
+                if (ST) {
+#pragma unroll
+                    for (int kb = 0; kb < NKB; ++kb) {
+                        const int kc = kb * 32 + qd * 8;
+                        bfr[kb] = kc < r ? *reinterpret_cast<const uint4 *>(bst + (ol + g) * r + kc)
+                                         : make_uint4(0, 0, 0, 0);
+                    }
+                    yva = *reinterpret_cast<const __nv_bfloat162 *>(yst + g * Wo + ol + 2 * qd);
+                    yvb = *reinterpret_cast<const __nv_bfloat162 *>(yst + (g + 8) * Wo + ol + 2 * qd);
+                } else {
+#pragma unroll
+                    for (int kb = 0; kb < NKB; ++kb)
+                        bfr[kb] = bw[ST ? 0 : t][kb];
+                    yva = ya[ST ? 0 : t];
+                    yvb = yb[ST ? 0 : t];
+                }
                 float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int kb = 0; kb < NKB; ++kb) {
@@ -221,26 +254,28 @@ __device__ __forceinline__ void expand_tiles(const __nv_bfloat16 *Ba, int r, int
                         c1 = l1[HOIST ? kb : 0];
                     } else {
                         const int kc = kb * 32 + qd * 8;
-                        a0 = *reinterpret_cast<const uint4 *>(vhi + g * kVS + kc);
-                        a1 = *reinterpret_cast<const uint4 *>(vhi + (g + 8) * kVS + kc);
-                        c0 = *reinterpret_cast<const uint4 *>(vlo + g * kVS + kc);
-                        c1 = *reinterpret_cast<const uint4 *>(vlo + (g + 8) * kVS + kc);
+                        a0 = *reinterpret_cast<const uint4 *>(vhi + g * vs + kc);
+                        a1 = *reinterpret_cast<const uint4 *>(vhi + (g + 8) * vs + kc);
+                        c0 = *reinterpret_cast<const uint4 *>(vlo + g * vs + kc);
+                        c1 = *reinterpret_cast<const uint4 *>(vlo + (g + 8) * vs + kc);
                     }
-                    mma16816(d, a0.x, a1.x, a0.y, a1.y, bw[t][kb].x, bw[t][kb].y);
-                    mma16816(d, c0.x, c1.x, c0.y, c1.y, bw[t][kb].x, bw[t][kb].y);
-                    mma16816(d, a0.z, a1.z, a0.w, a1.w, bw[t][kb].z, bw[t][kb].w);
-                    mma16816(d, c0.z, c1.z, c0.w, c1.w, bw[t][kb].z, bw[t][kb].w);
+                    mma16816(d, a0.x, a1.x, a0.y, a1.y, bfr[kb].x, bfr[kb].y);
+                    mma16816(d, c0.x, c1.x, c0.y, c1.y, bfr[kb].x, bfr[kb].y);
+                    mma16816(d, a0.z, a1.z, a0.w, a1.w, bfr[kb].z, bfr[kb].w);
+                    mma16816(d, c0.z, c1.z, c0.w, c1.w, bfr[kb].z, bfr[kb].w);
                 }
                 // D fragment: tokens g, g+8; outputs ob + 2qd, ob + 2qd + 1
-                const int o = o0 + ot * 8 + 2 * qd;
+                const int o = o0 + ol + 2 * qd;
+                __nv_bfloat16 *d0 = y0row + o;
+                __nv_bfloat16 *d1 = y1row + o;
                 if (row0) {
-                    const float2 y = __bfloat1622float2(ya[t]);
-                    *reinterpret_cast<__nv_bfloat162 *>(y0row + o) =
+                    const float2 y = __bfloat1622float2(yva);
+                    *reinterpret_cast<__nv_bfloat162 *>(d0) =
                         __floats2bfloat162_rn(fmaf(sc, d[0], y.x), fmaf(sc, d[1], y.y));
                 }
                 if (row1) {
-                    const float2 y = __bfloat1622float2(yb[t]);
-                    *reinterpret_cast<__nv_bfloat162 *>(y1row + o) =
+                    const float2 y = __bfloat1622float2(yvb);
+                    *reinterpret_cast<__nv_bfloat162 *>(d1) =
                         __floats2bfloat162_rn(fmaf(sc, d[2], y.x), fmaf(sc, d[3], y.y));
                 }
             }
@@ -251,13 +286,18 @@ __device__ __forceinline__ void expand_tiles(const __nv_bfloat16 *Ba, int r, int
 __global__ void __launch_bounds__(kFThreads, 5) k_bgmv_fused(FusedBgmvArgs p)
 {
     extern __shared__ __align__(16) unsigned char sm_raw[];
-    const FusedSmem L = fused_smem_layout(p.N, p.pool.n_adapters, p.Wk);
+    const FusedSmem L = fused_smem_layout(p.N, p.pool.n_adapters, p.pool.max_rank, p.Wo);
+    const int vs = L.vs;
+    const int mr = p.pool.max_rank < kMaxRank ? p.pool.max_rank : kMaxRank;
     int32_t *ids_s = reinterpret_cast<int32_t *>(sm_raw + L.ids);
     int32_t *ipre = reinterpret_cast<int32_t *>(sm_raw + L.cnt);    // [n_ad + 1]
-    float *vpart = reinterpret_cast<float *>(sm_raw + L.vpart);     // [kMaxRank][kFT], read by the cluster
-    // V split into bf16 hi and lo parts, token-major: [kFT][kVS] each
+    float *vpart = reinterpret_cast<float *>(sm_raw + L.vpart);     // [max_rank][kFT], read by the cluster
+    // V split into bf16 hi and lo parts, token-major: [kFT][vs] each
     __nv_bfloat16 *vhi = reinterpret_cast<__nv_bfloat16 *>(sm_raw + L.vsum);
-    __nv_bfloat16 *vlo = vhi + kFT * kVS;
+    __nv_bfloat16 *vlo = vhi + kFT * vs;
+    // staged (when L.staged): this CTA's B chunk [Wo][r] and the item's y rows [kFT][Wo]
+    __nv_bfloat16 *bst = reinterpret_cast<__nv_bfloat16 *>(sm_raw + L.bst);
+    __nv_bfloat16 *yst = reinterpret_cast<__nv_bfloat16 *>(sm_raw + L.yst);
     __shared__ int32_t tok[kFT];
     __shared__ int32_t s_ad, s_g, s_cnt, s_bad, s_r;
     __shared__ int64_t s_aoff, s_boff;
@@ -355,31 +395,19 @@ __global__ void __launch_bounds__(kFThreads, 5) k_bgmv_fused(FusedBgmvArgs p)
             }
             s_ad = lo;
             s_g = item - ipre[lo];
+        }
+        __syncthreads();
+        PHASE(9);
+        const int a = s_ad;
+        // warp 1 fetches the adapter's metadata while warp 0 finds the item's tokens
+        if (tid == 32) {
             int32_t r = 0;
             int64_t ao = 0, bo = 0;
-            s_r = adapter_ok(p.pool, lo, &r, &ao, &bo) ? r : 0;
+            const bool ok = adapter_ok(p.pool, a, &r, &ao, &bo);
+            s_r = ok ? r : 0;
             s_aoff = ao;
             s_boff = bo;
         }
-        __syncthreads();
-        const int a = s_ad;
-        const int r = s_r;
-        if (r == 0) {
-            // the same decision in every CTA of the cluster
-            if (!waited) {
-                pdl_trigger();
-                pdl_wait();
-                waited = true;
-            }
-            if (crank == 0 && tid == 0)
-                atomicOr(p.err, (uint32_t)LORA_ERR_BAD_ADAPTER);
-            __syncthreads();
-            continue;
-        }
-        const __nv_bfloat16 *Aa = p.pool.A + s_aoff;
-        const __nv_bfloat16 *Ba = p.pool.B + s_boff;
-        if (tid == 32 && o1 > o0)   // this CTA's B chunk towards L2 (immutable input)
-            prefetch_l2(Ba + (int64_t)o0 * r, (uint32_t)((o1 - o0) * r * 2));
         if (warp == 0) {
             const int lo = s_g * kFT;
             int seen = 0;
@@ -397,14 +425,39 @@ __global__ void __launch_bounds__(kFThreads, 5) k_bgmv_fused(FusedBgmvArgs p)
             if (lane == 0)
                 s_cnt = min(kFT, seen - lo);
         }
-        for (int e = tid; e < kMaxRank * kFT; e += kFThreads)
+        for (int e = tid; e < mr * kFT; e += kFThreads)
             vpart[e] = 0.f;
         __syncthreads();
+        PHASE(10);
+        const int r = s_r;
         const int cnt = s_cnt;
+        if (r == 0) {
+            // the same decision in every CTA of the cluster
+            if (!waited) {
+                pdl_trigger();
+                pdl_wait();
+                waited = true;
+            }
+            if (crank == 0 && tid == 0)
+                atomicOr(p.err, (uint32_t)LORA_ERR_BAD_ADAPTER);
+            __syncthreads();
+            continue;
+        }
+        const __nv_bfloat16 *Aa = p.pool.A + s_aoff;
+        const __nv_bfloat16 *Ba = p.pool.B + s_boff;
+        if (L.staged) {
+            // this CTA's B chunk into shared memory (immutable input): lands during the shrink
+            const int nch = (o1 - o0) * r / 8;
+            const __nv_bfloat16 *src = Ba + (int64_t)o0 * r;
+            for (int c = tid; c < nch; c += kFThreads)
+                cp_async16(bst + c * 8, src + c * 8);
+        } else if (tid == 32 && o1 > o0) {   // this CTA's B chunk towards L2 (immutable input)
+            prefetch_l2(Ba + (int64_t)o0 * r, (uint32_t)((o1 - o0) * r * 2));
+        }
         // the tokens' y rows towards L2: a prefetch only fills L2, which is the
         // point of coherence, so it cannot expose data older than a write that
         // the previous kernel completes later
-        if (tid >= 32 && tid < 32 + cnt && o1 > o0)
+        if (!L.staged && tid >= 32 && tid < 32 + cnt && o1 > o0)
             prefetch_l2(p.Y + (int64_t)tok[tid - 32] * p.ldy + o0, (uint32_t)((o1 - o0) * 2));
         PHASE(3);
 
@@ -427,6 +480,16 @@ __global__ void __launch_bounds__(kFThreads, 5) k_bgmv_fused(FusedBgmvArgs p)
             pdl_wait();   // from here on x, y and the workspace may be touched
             waited = true;
         }
+        PHASE(11);
+        if (L.staged) {
+            // the item's y rows into shared memory: land during the shrink and the exchange
+            const int cpr = (o1 - o0) / 8;
+            for (int c = tid; c < cnt * cpr; c += kFThreads) {
+                const int t = c / cpr, j = c - t * cpr;
+                cp_async16(yst + t * p.Wo + j * 8, p.Y + (int64_t)tok[t] * p.ldy + o0 + j * 8);
+            }
+        }
+        cp_async_commit();
         {
             const bool row0 = g < cnt, row1 = g + 8 < cnt;
             const __nv_bfloat16 *x0 = p.X + (int64_t)(row0 ? tok[g] : 0) * p.ldx;
@@ -477,6 +540,7 @@ __global__ void __launch_bounds__(kFThreads, 5) k_bgmv_fused(FusedBgmvArgs p)
         // then split V into bf16 hi + lo, token-major, zero beyond cnt and r
         cluster_arrive();
         cluster_wait();
+        PHASE(13);
         {
             namespace cg = cooperative_groups;
             cg::cluster_group cl = cg::this_cluster();
@@ -501,13 +565,14 @@ __global__ void __launch_bounds__(kFThreads, 5) k_bgmv_fused(FusedBgmvArgs p)
                     if (idx < kFT * rp) {
                         const int t = idx & (kFT - 1), j = idx >> 4;
                         const __nv_bfloat16 h = __float2bfloat16_rn(s[u]);
-                        vhi[t * kVS + j] = h;
-                        vlo[t * kVS + j] = __float2bfloat16_rn(s[u] - __bfloat162float(h));
+                        vhi[t * vs + j] = h;
+                        vlo[t * vs + j] = __float2bfloat16_rn(s[u] - __bfloat162float(h));
                     }
                 }
             }
         }
         cluster_arrive();   // our reads of the other CTAs' partials are done
+        cp_async_wait_all();
         __syncthreads();
         PHASE(6);
 
@@ -517,13 +582,27 @@ __global__ void __launch_bounds__(kFThreads, 5) k_bgmv_fused(FusedBgmvArgs p)
             const bool row0 = g < cnt, row1 = g + 8 < cnt;
             __nv_bfloat16 *y0row = p.Y + (int64_t)(row0 ? tok[g] : 0) * p.ldy;
             __nv_bfloat16 *y1row = p.Y + (int64_t)(row1 ? tok[g + 8] : 0) * p.ldy;
-            switch ((r + 31) >> 5) {
-            case 1: expand_tiles<1>(Ba, r, o0, n_ot, warp, kFWarps, vhi, vlo, g, qd, y0row, y1row, row0, row1, p.scale); break;
-            case 2: expand_tiles<2>(Ba, r, o0, n_ot, warp, kFWarps, vhi, vlo, g, qd, y0row, y1row, row0, row1, p.scale); break;
-            case 3: expand_tiles<3>(Ba, r, o0, n_ot, warp, kFWarps, vhi, vlo, g, qd, y0row, y1row, row0, row1, p.scale); break;
-            default: expand_tiles<4>(Ba, r, o0, n_ot, warp, kFWarps, vhi, vlo, g, qd, y0row, y1row, row0, row1, p.scale); break;
+#define LORA_EXPAND(NKB, ST)                                                                             \
+    expand_tiles<NKB, ST>(Ba, r, o0, n_ot, warp, kFWarps, vhi, vlo, vs, g, qd, y0row, y1row, row0, row1, p.scale, \
+                          bst, yst, p.Wo)
+            if (L.staged) {
+                switch ((r + 31) >> 5) {
+                case 1: LORA_EXPAND(1, true); break;
+                case 2: LORA_EXPAND(2, true); break;
+                case 3: LORA_EXPAND(3, true); break;
+                default: LORA_EXPAND(4, true); break;
+                }
+            } else {
+                switch ((r + 31) >> 5) {
+                case 1: LORA_EXPAND(1, false); break;
+                case 2: LORA_EXPAND(2, false); break;
+                case 3: LORA_EXPAND(3, false); break;
+                default: LORA_EXPAND(4, false); break;
+                }
             }
+#undef LORA_EXPAND
         }
+        PHASE(12);
         __syncthreads();
         PHASE(7);
         cluster_wait();     // no CTA reuses its partials while another may still read them
@@ -540,16 +619,17 @@ __global__ void __launch_bounds__(kFThreads, 5) k_bgmv_fused(FusedBgmvArgs p)
 
 }  // namespace
 
-size_t fused_smem_bytes(int32_t N, int32_t n_adapters, int32_t Wk)
+size_t fused_smem_bytes(int32_t N, int32_t n_adapters, int32_t max_rank, int32_t Wo)
 {
-    return fused_smem_layout(N, n_adapters, Wk).total;
+    return fused_smem_layout(N, n_adapters, max_rank, Wo).total;
 }
 
 bool fused_bgmv_supported(int32_t N, int32_t n_adapters, int32_t d_in)
 {
+    // the layout at the largest rank, without staging (staging is dropped when it does not fit)
     const int32_t Wk = fused_chunk(d_in);
     return N <= kFMaxTokens && n_adapters <= kFMaxAdapters && Wk <= kFMaxChunk &&
-           fused_smem_bytes(N, n_adapters, Wk) <= kFMaxSmem;
+           fused_smem_bytes(N, n_adapters, kMaxRank, 0) <= kFMaxSmem;
 }
 
 namespace {
@@ -599,7 +679,7 @@ int max_active_clusters(int dev, size_t smem, cudaStream_t s)
 
 cudaError_t launch_bgmv_fused(const FusedBgmvArgs &a, cudaStream_t s, bool pdl)
 {
-    const size_t smem = fused_smem_bytes(a.N, a.pool.n_adapters, a.Wk);
+    const size_t smem = fused_smem_bytes(a.N, a.pool.n_adapters, a.pool.max_rank, a.Wo);
     static bool attr_set[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);

@@ -123,24 +123,39 @@ constexpr int kFMaxChunk = 1 << 20; // d_in chunk per CTA (nothing of it is stag
 constexpr size_t kFMaxSmem = 200 * 1024;
 
 struct FusedSmem {
-    size_t ids, cnt, vpart, vsum, total;
+    size_t ids, cnt, vpart, vsum, bst, yst, total;
+    int vs;          // bf16 row stride of the staged rank-r vectors
+    bool staged;     // this CTA's B chunk and the item's y rows are copied to shared memory
 };
 
 __host__ __device__ inline size_t fused_align16(size_t x) { return (x + 15) & ~(size_t)15; }
 
-__host__ __device__ inline FusedSmem fused_smem_layout(int32_t N, int32_t n_adapters, int32_t Wk)
+// Shared memory of the fused decode kernel.  The rank-dependent parts are sized
+// by the pool's max_rank; when a CTA's B chunk (Wo x max_rank) and the y rows of
+// an item (kFT x Wo) fit 16 KB each, both are staged with cp.async while the
+// shrink and the cluster exchange run.
+__host__ __device__ inline FusedSmem fused_smem_layout(int32_t N, int32_t n_adapters, int32_t max_rank, int32_t Wo)
 {
-    (void)Wk;
     FusedSmem L;
+    const int mr = max_rank > kMaxRank ? kMaxRank : max_rank;
+    L.vs = mr <= 32 ? 40 : kVS;                       // 80-byte rows: 16-byte reads conflict-free
     size_t off = 0;
     L.ids = off;
     off = fused_align16(off + 4 * (size_t)N);
     L.cnt = off;
     off = fused_align16(off + 4 * ((size_t)n_adapters + 1));
     L.vpart = off;
-    off = fused_align16(off + 4 * (size_t)kMaxRank * kFT);
+    off = fused_align16(off + 4 * (size_t)mr * kFT);
     L.vsum = off;
-    off = fused_align16(off + 2 * 2 * (size_t)kFT * kVS);   // bf16 hi and lo
+    off = fused_align16(off + 2 * 2 * (size_t)kFT * L.vs);   // bf16 hi and lo
+    L.staged = Wo > 0 && (int64_t)Wo * mr <= 8192 && (int64_t)kFT * Wo <= 8192 &&
+               off + 2 * 16384 + 32 <= kFMaxSmem;
+    L.bst = off;
+    if (L.staged)
+        off = fused_align16(off + 2 * (size_t)Wo * mr);
+    L.yst = off;
+    if (L.staged)
+        off = fused_align16(off + 2 * (size_t)kFT * Wo);
     L.total = off;
     return L;
 }
@@ -165,7 +180,7 @@ struct FusedBgmvArgs {
     uint32_t *err;
 };
 
-size_t fused_smem_bytes(int32_t N, int32_t n_adapters, int32_t Wk);
+size_t fused_smem_bytes(int32_t N, int32_t n_adapters, int32_t max_rank, int32_t Wo);
 bool fused_bgmv_supported(int32_t N, int32_t n_adapters, int32_t d_in);
 cudaError_t launch_bgmv_fused(const FusedBgmvArgs &a, cudaStream_t s, bool pdl);
 bool pdl_enabled();
