@@ -77,6 +77,10 @@ __global__ void __launch_bounds__(kPlanThreads) k_plan(PlanArgs p)
     extern __shared__ int32_t hist[];   // [n_adapters] (route mode only)
     __shared__ long long sm_scan[33];
     __shared__ int32_t sm_flag;
+    // programmatic dependent launch: the previous kernel on the stream (which may
+    // produce this call's inputs or still read the workspace) completes first
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int tid = threadIdx.x;
     const int32_t N = p.N;
     const int32_t *item_off = p.item_off;
@@ -228,11 +232,16 @@ cudaError_t launch_plan(const PlanArgs &a, cudaStream_t s)
         if (dev >= 0 && dev < 64)
             attr_set[dev] = true;
     }
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(1);
     cfg.blockDim = dim3(kPlanThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl_enabled() ? 1 : 0;
     return cudaLaunchKernelEx(&cfg, k_plan, a);
 }
 

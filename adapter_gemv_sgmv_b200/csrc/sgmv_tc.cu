@@ -137,6 +137,46 @@ __device__ __forceinline__ void ld_shared_v4(uint32_t addr, uint32_t (&w)[4])
                  : "memory");
 }
 
+// The same with an L2 eviction-priority hint (a createpolicy value).
+__device__ __forceinline__ void tma_load_2d_hint(void *dst, const CUtensorMap *map, uint64_t *bar, int x, int y,
+                                                 uint64_t policy)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4}], [%2], %5;"
+        ::"r"(smem_u32(dst)), "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y), "l"(policy)
+        : "memory");
+}
+
+// L2 policies: streamed data (x, y) leaves L2 first, adapter weights (re-read by
+// every tile of a segment) last.
+__device__ __forceinline__ uint64_t policy_evict_first()
+{
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+__device__ __forceinline__ uint64_t policy_evict_last()
+{
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+__device__ __forceinline__ void st_global_v4_hint(void *ptr, uint32_t a, uint32_t b, uint32_t c, uint32_t d,
+                                                  uint64_t policy)
+{
+    asm volatile("st.global.L1::no_allocate.L2::cache_hint.v4.b32 [%0], {%1,%2,%3,%4}, %5;" ::"l"(ptr), "r"(a),
+                 "r"(b), "r"(c), "r"(d), "l"(policy)
+                 : "memory");
+}
+
+// Programmatic dependent launch: wait until the previous kernel on the stream has
+// completed (its writes visible), then let the next one start its prologue.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // 16-byte async copy global -> shared; when !pred the destination is zero-filled
 // and nothing is read (the source must still be a valid address).
 // (No memory clobber: the copy lands asynchronously anyway, and the address
@@ -406,9 +446,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) k_tc_shrink(const __grid_consta
     __shared__ int abort_flag;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int n_units = p.hdr->n_groups;
     const int G = gridDim.x;
-    const int u0 = (int)((int64_t)blockIdx.x * n_units / G), u1 = (int)((int64_t)(blockIdx.x + 1) * n_units / G);
     const int d_in = p.pool.d_in;
     const int n_kb = (d_in + kBK - 1) / kBK;
     const int n_st = p.s_stages;
@@ -431,6 +469,10 @@ __global__ void __launch_bounds__(kTcThreads, 2) k_tc_shrink(const __grid_consta
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_base;
+    pdl_wait();                                  // the plan kernel's tiles are complete
+    pdl_trigger();
+    const int n_units = p.hdr->n_groups;
+    const int u0 = (int)((int64_t)blockIdx.x * n_units / G), u1 = (int)((int64_t)(blockIdx.x + 1) * n_units / G);
 
     if (warp == 0) {
         // ------------------------------------------------ producer
@@ -475,6 +517,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) k_tc_shrink(const __grid_consta
                 __syncwarp();
             }
             const uint32_t tx = (uint32_t)kAtom + (use_tma ? (uint32_t)st.ktot * 128u : 0u);
+            const uint64_t pol_x = policy_evict_first(), pol_a = policy_evict_last();
             for (int kb = 0; kb < n_kb; ++kb, ++it) {
                 const int s = it % n_st;
                 const uint32_t ph = (it / n_st) & 1;
@@ -486,12 +529,12 @@ __global__ void __launch_bounds__(kTcThreads, 2) k_tc_shrink(const __grid_consta
                 unsigned char *as = xs + kAtom;
                 if (lane == 0) {
                     mbar_arrive_expect_tx(&full_bar[s], tx);
-                    tma_load_2d(xs, &p.map_x, &full_bar[s], kb * kBK, gr.p0);
+                    tma_load_2d_hint(xs, &p.map_x, &full_bar[s], kb * kBK, gr.p0, pol_x);
                 }
                 __syncwarp();
                 if (use_tma) {
                     if (lane < nbox)
-                        tma_load_2d(as + box_j * 128, &p.map_a[box_m], &full_bar[s], kb * kBK, box_row);
+                        tma_load_2d_hint(as + box_j * 128, &p.map_a[box_m], &full_bar[s], kb * kBK, box_row, pol_a);
                 } else {
                     // stacked row j, 16-byte chunk c; rows past the stack feed only
                     // accumulator columns that are never stored
@@ -637,9 +680,7 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_tc_expand(const __grid_co
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int d_out = p.pool.d_out;
     const int n_ns = (d_out + kBN - 1) / kBN;           // output slices
-    const int64_t n_units = (int64_t)p.hdr->n_groups * n_ns;
     const int G = gridDim.x;
-    const int64_t u0 = (int64_t)blockIdx.x * n_units / G, u1 = (int64_t)(blockIdx.x + 1) * n_units / G;
     const int n_ys = p.e_ystages;
     const int szB = p.e_natoms * kAtom;                 // one B stage (and V)
     unsigned char *const smV = sm;
@@ -671,6 +712,10 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_tc_expand(const __grid_co
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_base;
+    pdl_wait();                                  // tiles and V of the previous kernels are complete
+    pdl_trigger();
+    const int64_t n_units = (int64_t)p.hdr->n_groups * n_ns;
+    const int64_t u0 = (int64_t)blockIdx.x * n_units / G, u1 = (int64_t)(blockIdx.x + 1) * n_units / G;
 
     if (warp == 0) {
         // ------------------------------------------------ producer: y tiles and B slices
@@ -680,6 +725,7 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_tc_expand(const __grid_co
         int nch = 0, o_l = 0, c_l = 0, dq = 0, dr = 0;
         int p0 = 0;
         int bx_m = 0, bx_y = 0, bx_dst = 0, bx_two = 0;   // this lane's B box (TMA path, lane < n)
+        const uint64_t pol_y = policy_evict_first(), pol_b = policy_evict_last();
         for (int64_t u = u0; u < u1; ++u, ++it) {
             const int tile = (int)(u / n_ns), ns = (int)(u - (int64_t)tile * n_ns);
             if (tile != prev_tile) {
@@ -728,8 +774,8 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_tc_expand(const __grid_co
             unsigned char *ys = smY + sy * kY;
             if (lane == 0) {
                 mbar_arrive_expect_tx(&y_full[sy], kY);
-                tma_load_2d(ys, &p.map_y, &y_full[sy], o0, p0);
-                tma_load_2d(ys + kAtom, &p.map_y, &y_full[sy], o0 + 64, p0);
+                tma_load_2d_hint(ys, &p.map_y, &y_full[sy], o0, p0, pol_y);
+                tma_load_2d_hint(ys + kAtom, &p.map_y, &y_full[sy], o0 + 64, p0, pol_y);
             }
             const int sb = it % kExpandBStages;
             if (!warp_wait(&b_empty[sb], ((it / kExpandBStages) & 1) ^ 1, &abort_flag, p.err))
@@ -744,9 +790,9 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_tc_expand(const __grid_co
                     mbar_arrive_expect_tx(&b_full[sb], (uint32_t)st.ktot * 256u);
                 __syncwarp();
                 if (lane < st.n) {
-                    tma_load_2d(bs + bx_dst, &p.map_b[bx_m], &b_full[sb], 0, bx_y + o0);
+                    tma_load_2d_hint(bs + bx_dst, &p.map_b[bx_m], &b_full[sb], 0, bx_y + o0, pol_b);
                     if (bx_two)
-                        tma_load_2d(bs + bx_dst + kAtom, &p.map_b[bx_m], &b_full[sb], 64, bx_y + o0);
+                        tma_load_2d_hint(bs + bx_dst + kAtom, &p.map_b[bx_m], &b_full[sb], 64, bx_y + o0, pol_b);
                 }
             } else {
                 if (lane == 0)
@@ -854,6 +900,7 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_tc_expand(const __grid_co
         int it = 0, vt = 0;
         int64_t prev_tile = -1;
         Group gr = {0, 0, 0, 0};
+        const uint64_t pol_st = policy_evict_first();
         for (int64_t u = u0; u < u1; ++u, ++it) {
             const int tile = (int)(u / n_ns), ns = (int)(u - (int64_t)tile * n_ns);
             if (tile != prev_tile) {
@@ -977,8 +1024,8 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_tc_expand(const __grid_co
                         if (rl < n_rows) {
                             uint32_t w[4];
                             ld_shared_v4(stg + rl * 64 + ((cc ^ ((rl >> 1) & 3)) << 4), w);
-                            *reinterpret_cast<uint4 *>(p.Y + (int64_t)(gr.p0 + q * 32 + rl) * p.ldy + o) =
-                                make_uint4(w[0], w[1], w[2], w[3]);
+                            st_global_v4_hint(p.Y + (int64_t)(gr.p0 + q * 32 + rl) * p.ldy + o, w[0], w[1], w[2],
+                                              w[3], pol_st);
                         }
                     }
                 }
@@ -1054,11 +1101,16 @@ cudaError_t launch_tc(void (*kernel)(TcArgs), bool *attr_set, const TcArgs &a, i
         if (dev >= 0 && dev < 64)
             attr_set[dev] = true;
     }
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(threads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl_enabled() ? 1 : 0;
     return cudaLaunchKernelEx(&cfg, kernel, a);
 }
 
