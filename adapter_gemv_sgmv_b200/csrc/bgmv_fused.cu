@@ -283,6 +283,69 @@ __device__ __forceinline__ void expand_tiles(const __nv_bfloat16 *Ba, int r, int
     }
 }
 
+// Expand for ranks <= 16: one k16 step per tile.  Inside the 16 ranks the k order
+// is permuted identically for both operands so that thread quad qd holds ranks
+// 4qd .. 4qd+3 (8-byte fragments of V and B), and the two MMAs per tile are the
+// V_hi and V_lo halves.
+template <bool ST>
+__device__ __forceinline__ void expand_tiles16(const __nv_bfloat16 *Ba, int r, int o0, int n_ot, int warp, int nw,
+                                               const __nv_bfloat16 *vhi, const __nv_bfloat16 *vlo, int vs, int g,
+                                               int qd, __nv_bfloat16 *y0row, __nv_bfloat16 *y1row, bool row0,
+                                               bool row1, float sc, const __nv_bfloat16 *bst,
+                                               const __nv_bfloat16 *yst, int Wo)
+{
+    // global operands: a batch's B fragments and y values are requested before its MMAs;
+    // staged operands (shared memory) are read tile by tile
+    constexpr int TPB = ST ? 1 : 8;
+    const int kc = qd * 4;
+    const bool kin = kc < r;
+    const uint2 h0 = *reinterpret_cast<const uint2 *>(vhi + g * vs + kc);
+    const uint2 h1 = *reinterpret_cast<const uint2 *>(vhi + (g + 8) * vs + kc);
+    const uint2 l0 = *reinterpret_cast<const uint2 *>(vlo + g * vs + kc);
+    const uint2 l1 = *reinterpret_cast<const uint2 *>(vlo + (g + 8) * vs + kc);
+    const __nv_bfloat162 z = __floats2bfloat162_rn(0.f, 0.f);
+    for (int ot0 = warp; ot0 < n_ot; ot0 += TPB * nw) {
+        uint2 bw[TPB];
+        __nv_bfloat162 ya[TPB], yb[TPB];
+#pragma unroll
+        for (int t = 0; t < TPB; ++t) {
+            const int ot = ot0 + t * nw;
+            const bool ok = ot < n_ot;
+            const int ol = ot * 8;
+            if (ST) {
+                bw[t] = (ok && kin) ? *reinterpret_cast<const uint2 *>(bst + (ol + g) * r + kc) : make_uint2(0, 0);
+                ya[t] = ok ? *reinterpret_cast<const __nv_bfloat162 *>(yst + g * Wo + ol + 2 * qd) : z;
+                yb[t] = ok ? *reinterpret_cast<const __nv_bfloat162 *>(yst + (g + 8) * Wo + ol + 2 * qd) : z;
+            } else {
+                bw[t] = (ok && kin) ? *reinterpret_cast<const uint2 *>(Ba + (int64_t)(o0 + ol + g) * r + kc)
+                                    : make_uint2(0, 0);
+                ya[t] = (ok && row0) ? *reinterpret_cast<const __nv_bfloat162 *>(y0row + o0 + ol + 2 * qd) : z;
+                yb[t] = (ok && row1) ? *reinterpret_cast<const __nv_bfloat162 *>(y1row + o0 + ol + 2 * qd) : z;
+            }
+        }
+#pragma unroll
+        for (int t = 0; t < TPB; ++t) {
+            const int ot = ot0 + t * nw;
+            if (ot < n_ot) {
+                float d[4] = {0.f, 0.f, 0.f, 0.f};
+                mma16816(d, h0.x, h1.x, h0.y, h1.y, bw[t].x, bw[t].y);
+                mma16816(d, l0.x, l1.x, l0.y, l1.y, bw[t].x, bw[t].y);
+                const int o = o0 + ot * 8 + 2 * qd;
+                if (row0) {
+                    const float2 y = __bfloat1622float2(ya[t]);
+                    *reinterpret_cast<__nv_bfloat162 *>(y0row + o) =
+                        __floats2bfloat162_rn(fmaf(sc, d[0], y.x), fmaf(sc, d[1], y.y));
+                }
+                if (row1) {
+                    const float2 y = __bfloat1622float2(yb[t]);
+                    *reinterpret_cast<__nv_bfloat162 *>(y1row + o) =
+                        __floats2bfloat162_rn(fmaf(sc, d[2], y.x), fmaf(sc, d[3], y.y));
+                }
+            }
+        }
+    }
+}
+
 __global__ void __launch_bounds__(kFThreads, 5) k_bgmv_fused(FusedBgmvArgs p)
 {
     extern __shared__ __align__(16) unsigned char sm_raw[];
@@ -585,7 +648,14 @@ __global__ void __launch_bounds__(kFThreads, 5) k_bgmv_fused(FusedBgmvArgs p)
 #define LORA_EXPAND(NKB, ST)                                                                             \
     expand_tiles<NKB, ST>(Ba, r, o0, n_ot, warp, kFWarps, vhi, vlo, vs, g, qd, y0row, y1row, row0, row1, p.scale, \
                           bst, yst, p.Wo)
-            if (L.staged) {
+            if (r <= 16) {
+                if (L.staged)
+                    expand_tiles16<true>(Ba, r, o0, n_ot, warp, kFWarps, vhi, vlo, vs, g, qd, y0row, y1row, row0,
+                                         row1, p.scale, bst, yst, p.Wo);
+                else
+                    expand_tiles16<false>(Ba, r, o0, n_ot, warp, kFWarps, vhi, vlo, vs, g, qd, y0row, y1row, row0,
+                                          row1, p.scale, bst, yst, p.Wo);
+            } else if (L.staged) {
                 switch ((r + 31) >> 5) {
                 case 1: LORA_EXPAND(1, true); break;
                 case 2: LORA_EXPAND(2, true); break;
