@@ -351,6 +351,7 @@ __global__ void __launch_bounds__(kFThreads, 5) k_bgmv_fused(FusedBgmvArgs p)
     extern __shared__ __align__(16) unsigned char sm_raw[];
     const FusedSmem L = fused_smem_layout(p.N, p.pool.n_adapters, p.pool.max_rank, p.Wo);
     const int vs = L.vs;
+    int16_t *item_ad = reinterpret_cast<int16_t *>(sm_raw + L.items);   // adapter of items < L.n_tab
     const int mr = p.pool.max_rank < kMaxRank ? p.pool.max_rank : kMaxRank;
     int32_t *ids_s = reinterpret_cast<int32_t *>(sm_raw + L.ids);
     int32_t *ipre = reinterpret_cast<int32_t *>(sm_raw + L.cnt);    // [n_ad + 1]
@@ -432,6 +433,8 @@ __global__ void __launch_bounds__(kFThreads, 5) k_bgmv_fused(FusedBgmvArgs p)
         for (int a = b; a < e; ++a) {
             const int gr = (ipre[a] + kFT - 1) / kFT;
             ipre[a] = run;
+            for (int j = 0; j < gr && run + j < L.n_tab; ++j)
+                item_ad[run + j] = (int16_t)a;
             run += gr;
         }
         if (tid == 0)
@@ -448,13 +451,18 @@ __global__ void __launch_bounds__(kFThreads, 5) k_bgmv_fused(FusedBgmvArgs p)
     for (int item = (int)cluster_id_x(); item < n_items; item += n_cl) {
         // ---- the item's adapter, metadata and tokens (immutable inputs only)
         if (tid == 0) {
-            int lo = 0, hi = n_ad;   // last adapter with ipre[a] <= item
-            while (hi - lo > 1) {
-                const int mid = (lo + hi) >> 1;
-                if (ipre[mid] <= item)
-                    lo = mid;
-                else
-                    hi = mid;
+            int lo = 0;
+            if (item < L.n_tab) {
+                lo = item_ad[item];      // written by the grouping
+            } else {
+                int hi = n_ad;           // last adapter with ipre[a] <= item
+                while (hi - lo > 1) {
+                    const int mid = (lo + hi) >> 1;
+                    if (ipre[mid] <= item)
+                        lo = mid;
+                    else
+                        hi = mid;
+                }
             }
             s_ad = lo;
             s_g = item - ipre[lo];

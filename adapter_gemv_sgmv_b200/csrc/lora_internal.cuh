@@ -122,8 +122,11 @@ constexpr int kFMaxAdapters = 8192; // per-adapter group offsets in shared memor
 constexpr int kFMaxChunk = 1 << 20; // d_in chunk per CTA (nothing of it is staged)
 constexpr size_t kFMaxSmem = 200 * 1024;
 
+constexpr int kFItemTable = 1024;   // most items whose adapter the grouping writes into a table
+
 struct FusedSmem {
-    size_t ids, cnt, vpart, vsum, bst, yst, total;
+    size_t ids, cnt, items, vpart, vsum, bst, yst, total;
+    int n_tab;       // entries of the item -> adapter table (int16)
     int vs;          // bf16 row stride of the staged rank-r vectors
     bool staged;     // this CTA's B chunk and the item's y rows are copied to shared memory
 };
@@ -144,6 +147,11 @@ __host__ __device__ inline FusedSmem fused_smem_layout(int32_t N, int32_t n_adap
     off = fused_align16(off + 4 * (size_t)N);
     L.cnt = off;
     off = fused_align16(off + 4 * ((size_t)n_adapters + 1));
+    // items: at most min(N, n_adapters) adapters plus one more 16-token group per 16 tokens
+    const int64_t max_items = (int64_t)(N < n_adapters ? N : n_adapters) + N / kFT + 1;
+    L.n_tab = (int)(max_items < kFItemTable ? max_items : kFItemTable);
+    L.items = off;
+    off = fused_align16(off + 2 * (size_t)L.n_tab);
     L.vpart = off;
     off = fused_align16(off + 4 * (size_t)mr * kFT);
     L.vsum = off;
