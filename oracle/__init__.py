@@ -117,8 +117,9 @@ class Oracle:
         lib.oracle_apply_multi.argtypes = [P, i64, P, P, P, P, P, i32, i32, i32, P, P, P, P, i32, i32,
                                            P, i32, P]
         lib.oracle_route.argtypes = [P, i32, i32, P, P, P, P, P]
+        lib.oracle_merge.argtypes = [P, i64, P, P, P, P, P, i32, i32, i32, i32, f64, P, i32, P]
         for f in (lib.oracle_bgmv_delta, lib.oracle_sgmv_shrink, lib.oracle_sgmv_expand,
-                  lib.oracle_sgmv_delta, lib.oracle_apply_multi, lib.oracle_route):
+                  lib.oracle_sgmv_delta, lib.oracle_apply_multi, lib.oracle_route, lib.oracle_merge):
             f.restype = ctypes.c_int
         self.lib = lib
         self.path = path
@@ -204,6 +205,18 @@ class Oracle:
         _check(rc, "apply_multi")
         return D
 
+    def merge(self, W: np.ndarray, pool: HostPool, adapter: int, scale: float,
+              rows: Optional[np.ndarray] = None) -> np.ndarray:
+        """Wm[k] = W[o] + scale * (B[a] A[a])[o] for o = rows[k] (all rows by default), unrounded."""
+        W = _c(W, np.uint16)
+        rows, n_rows = _rows(rows, pool.d_out)
+        Wm = np.zeros((n_rows, pool.d_in), dtype=np.float64)
+        rc = self.lib.oracle_merge(_p(W), W.shape[1], _p(pool.A), _p(pool.A_off), _p(pool.B), _p(pool.B_off),
+                                   _p(pool.rank), pool.n_adapters, pool.d_in, pool.d_out, int(adapter),
+                                   float(scale), _p(rows), n_rows, _p(Wm))
+        _check(rc, "merge")
+        return Wm
+
     def route(self, ids: np.ndarray, n_adapters: int):
         """Stable counting sort of ids by adapter: (perm, seg_off, seg_ad); id -1 left out."""
         ids = _c(ids, np.int32)
@@ -252,6 +265,10 @@ def apply_multi_delta(*a, **k):
 
 def route(*a, **k):
     return default().route(*a, **k)
+
+
+def merge(*a, **k):
+    return default().merge(*a, **k)
 
 
 def widen_bf16(bits: np.ndarray) -> np.ndarray:

@@ -329,3 +329,47 @@ int oracle_route(const int32_t *ids, int32_t N, int32_t n_adapters,
     *n_seg_out = n_seg;
     return ORC_OK;
 }
+
+/*
+ * Merge (same page, section "LoRA: merged or alongside": a merged LoRA is
+ * W' = W + B A folded into the weight; switching adapters merges one and
+ * unmerges the other, i.e. adds and subtracts s * B A).  For adapter a and the
+ * base weight W [d_out, d_in] (bf16 bit patterns, row stride ldw):
+ *     Wm[k][i] = W[o][i] + s * sum_j B[a][o][j] * A[a][j][i],   o = rows[k]
+ * in double, without rounding (all rows in order when rows == NULL, n_rows =
+ * d_out).  Unmerging is the same call with -s.
+ */
+int oracle_merge(const uint16_t *W, int64_t ldw,
+                 const uint16_t *A, const int64_t *A_off,
+                 const uint16_t *B, const int64_t *B_off, const int32_t *rank,
+                 int32_t n_adapters, int32_t d_in, int32_t d_out, int32_t a, double scale,
+                 const int32_t *rows, int32_t n_rows, double *Wm)
+{
+    if (a < 0 || a >= n_adapters)
+        return ORC_BAD_ID;
+    int32_t r = rank[a];
+    if (r <= 0 || r > 128)
+        return ORC_BAD_RANK;
+    if (rows == NULL)
+        n_rows = d_out;
+    const uint16_t *Aa = A + A_off[a];
+    const uint16_t *Ba = B + B_off[a];
+    int status = ORC_OK;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int32_t k = 0; k < n_rows; ++k) {
+        int32_t o = rows ? rows[k] : k;
+        double *w_row = Wm + (int64_t)k * d_in;
+        if (o < 0 || o >= d_out) {
+#pragma omp atomic write
+            status = ORC_BAD_SEGMENT;
+            continue;
+        }
+        for (int32_t i = 0; i < d_in; ++i) {
+            double acc = 0.0;
+            for (int32_t j = 0; j < r; ++j)
+                acc += widen_bf16(Ba[(int64_t)o * r + j]) * widen_bf16(Aa[(int64_t)j * d_in + i]);
+            w_row[i] = widen_bf16(W[(int64_t)o * ldw + i]) + scale * acc;
+        }
+    }
+    return status;
+}

@@ -16,6 +16,7 @@ IP-Adapter", section "LoRA: merged or alongside", unless stated):
   the stable grouping (route) and integer-coded routing.
 * table row "Stacking several LoRAs": a few more alongside computations
   -> additivity and rank stacking.
+* merging folds s B A into W (and switching unmerges it) -> the merge pins.
 """
 from __future__ import annotations
 
@@ -83,6 +84,45 @@ def pin_mixed_ranks_per_token(orc):
     s = 2.0
     _close(orc.bgmv_delta(X, p, ids, s), numpy_delta_rows(X, p, ids, s))
     assert np.all(orc.bgmv_delta(X, p, ids, s)[ids == -1] == 0.0)
+
+
+def pin_merge_is_the_dense_rank_r_update(orc):
+    """Merging adapter a into W is W + s B_a A_a (numpy float64 matmul), on every row
+    or on a subset of rows; d_in != d_out != rank so a transposed operand fails."""
+    rng = np.random.default_rng(21)
+    d_in, d_out = 40, 24
+    p = rand_host_pool(rng, [8, 16, 24], d_in, d_out)
+    W = rand_x(rng, d_out, d_in)
+    for a, s in ((1, 0.75), (2, -1.25)):
+        want = widen(W) + s * (B_of(p, a) @ A_of(p, a))
+        _close(orc.merge(W, p, a, s), want)
+        rows = np.array([5, 0, 23], np.int32)
+        _close(orc.merge(W, p, a, s, rows=rows), want[rows])
+
+
+def pin_merge_agrees_with_the_unmerged_delta(orc):
+    """The merged-weight identity through the oracle's two paths: x Wm^T - x W^T
+    (merge) equals the unmerged delta s B_a A_a x (bgmv) for every token."""
+    rng = np.random.default_rng(22)
+    N, d_in, d_out = 9, 32, 48
+    p = rand_host_pool(rng, [16, 8], d_in, d_out)
+    W = rand_x(rng, d_out, d_in)
+    X = rand_x(rng, N, d_in)
+    for a, s in ((0, 1.5), (1, 0.5)):
+        Wm = orc.merge(W, p, a, s)
+        via_merge = widen(X) @ Wm.T - widen(X) @ widen(W).T
+        delta = orc.bgmv_delta(X, p, np.full(N, a, np.int32), s)
+        _close(via_merge, delta, rel=1e-10)
+
+
+def pin_merge_zero_B_and_unmerge(orc):
+    """B = 0 leaves W exactly as it was; merging with s and with -s averages to W."""
+    rng = np.random.default_rng(23)
+    p0 = rand_host_pool(rng, [8], 16, 24, zero_B=True)
+    W = rand_x(rng, 24, 16)
+    assert np.array_equal(orc.merge(W, p0, 0, 2.0), widen(W))
+    p = rand_host_pool(rng, [8], 16, 24)
+    _close(0.5 * (orc.merge(W, p, 0, 0.7) + orc.merge(W, p, 0, -0.7)), widen(W))
 
 
 def pin_zero_B(orc):

@@ -21,6 +21,12 @@ MUTANTS = {
                           "        for (int32_t j = 0; j + 1 < r; ++j)\n            acc += widen_bf16(Ba"),
     "unstable_route": ("for (int32_t n = 0; n < N; ++n)\n            if (ids[n] == a)",
                        "for (int32_t n = N - 1; n >= 0; --n)\n            if (ids[n] == a)"),
+    "merge_transposed_B": ("acc += widen_bf16(Ba[(int64_t)o * r + j]) * widen_bf16(Aa[(int64_t)j * d_in + i]);",
+                           "acc += widen_bf16(Ba[(int64_t)j * d_out + o]) * widen_bf16(Aa[(int64_t)j * d_in + i]);"),
+    "merge_dropped_base": ("w_row[i] = widen_bf16(W[(int64_t)o * ldw + i]) + scale * acc;",
+                           "w_row[i] = scale * acc;"),
+    "merge_sign": ("w_row[i] = widen_bf16(W[(int64_t)o * ldw + i]) + scale * acc;",
+                   "w_row[i] = widen_bf16(W[(int64_t)o * ldw + i]) - scale * acc;"),
     "dropped_last_adapter": ("for (int32_t p = ad_off[q]; p < ad_off[q + 1]; ++p)",
                              "for (int32_t p = ad_off[q]; p + 1 < ad_off[q + 1]; ++p)"),
 }
