@@ -20,13 +20,13 @@ __all__ = [
     "lora_kernel_launches",
     "lora_get_error", "lora_route", "lora_bgmv", "lora_sgmv_shrink", "lora_sgmv_expand",
     "lora_apply_multi", "lora_apply_multi_static", "make_pool_struct", "Workspace", "OP_BGMV", "OP_SGMV_SHRINK", "OP_SGMV_EXPAND",
-    "OP_APPLY_MULTI", "OP_ROUTE", "STATUS",
+    "OP_APPLY_MULTI", "OP_ROUTE", "OP_MERGE", "STATUS", "lora_merge",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 _LIBNAME = "liblora_sgmv.so"
 
-OP_BGMV, OP_SGMV_SHRINK, OP_SGMV_EXPAND, OP_APPLY_MULTI, OP_ROUTE = range(5)
+OP_BGMV, OP_SGMV_SHRINK, OP_SGMV_EXPAND, OP_APPLY_MULTI, OP_ROUTE, OP_MERGE = range(6)
 STATUS = {0: "LORA_OK", 1: "LORA_ERR_INVALID_ARG", 2: "LORA_ERR_UNSUPPORTED", 4: "LORA_ERR_BAD_ADAPTER",
           8: "LORA_ERR_BAD_SEGMENT", 16: "LORA_ERR_CUDA", 32: "LORA_ERR_WORKSPACE", 64: "LORA_ERR_TIMEOUT"}
 MAX_ADS_PER_REQ = 8
@@ -90,6 +90,8 @@ def load():
         lib.lora_apply_multi.argtypes = [P, i64, P, i64, PP, P, P, P, P, i32, i32, i32, P, sz, P]
         lib.lora_apply_multi_static.restype = ctypes.c_int
         lib.lora_apply_multi_static.argtypes = [P, i64, P, i64, PP, P, P, P, P, i32, i32, i32, P, P]
+        lib.lora_merge.restype = ctypes.c_int
+        lib.lora_merge.argtypes = [P, i64, PP, i32, f32, P, sz, P]
         _lib = lib
     return _lib
 
@@ -308,3 +310,21 @@ def lora_apply_multi_static(X, Y, pool, req_off, ad_off, ad_id, ad_scale, max_ad
     _rc(lib.lora_apply_multi_static(_ptr(X), ldx, _ptr(Y), ldy, ctypes.byref(ps), _ptr(req_off), _ptr(ad_off),
                                     _ptr(ad_id), _ptr(ad_scale), n_req, N, int(max_ads_per_req), _ptr(err_out),
                                     _stream_ptr(stream)), "lora_apply_multi_static")
+
+
+def lora_merge(W, pool, adapter: int, scale: float, ws: Workspace | None = None, stream=None,
+               max_rank: int | None = None):
+    """W[o] += scale * (B[a] A[a])[o] in place for the base weight W [d_out, d_in] (bf16);
+    unmerge with -scale.  Returns the workspace (its error word: lora_get_error)."""
+    lib = load()
+    _check_dev(W)
+    ps = make_pool_struct(pool, max_rank)
+    ldw = _mat(W, ps.d_in, "W")
+    if int(W.shape[0]) != ps.d_out:
+        raise LoraError("W must have pool.d_out rows", 1)
+    need = lora_workspace_size(OP_MERGE, ps.d_out, ps.n_adapters, ps.d_in, ps.d_out, ps.max_rank)
+    ws = ws or _workspace(need, W.device)
+    _rc(lib.lora_merge(_ptr(W), ldw, ctypes.byref(ps), int(adapter), float(scale), ws.ptr(), ws.nbytes,
+                       _stream_ptr(stream)), "lora_merge")
+    return ws
+

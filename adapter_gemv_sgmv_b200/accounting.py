@@ -121,11 +121,20 @@ def multi_cost(req_off: np.ndarray, ad_off: np.ndarray, ad_id: np.ndarray, ranks
 def call_cost(call) -> Cost:
     """Cost of one workload call (duck-typed on the call's host metadata)."""
     p = call.pool
+    if hasattr(call, "W"):
+        return merge_cost(p.d_in, p.d_out, int(p.ranks_h[call.adapter]))
     if hasattr(call, "ids_h"):
         return bgmv_cost(call.ids_h, p.ranks_h, p.d_in, p.d_out)
     if hasattr(call, "seg_off_h"):
         return sgmv_cost(call.seg_off_h, call.seg_ad_h, p.ranks_h, p.d_in, p.d_out)
     return multi_cost(call.req_off_h, call.ad_off_h, call.ad_id_h, p.ranks_h, p.d_in, p.d_out)
+
+
+def merge_cost(d_in: int, d_out: int, r: int) -> Cost:
+    """Merging one adapter into W [d_out, d_in]: W read and written once (bf16), the
+    adapter read once; 2 d_out d_in r FLOPs (the rank-r product B A)."""
+    return Cost(flops=2 * d_out * d_in * r, nbytes=2 * 2 * d_out * d_in + 2 * r * (d_in + d_out), tokens=d_out,
+                adapter_bytes=2 * r * (d_in + d_out), act_bytes=2 * 2 * d_out * d_in)
 
 
 def workload_cost(wl) -> Cost:

@@ -175,7 +175,9 @@ const char *lora_version(void) { return "lora_sgmv_b200 0.1 (sm_100a)"; }
 size_t lora_workspace_size(int op, int32_t N, int32_t n_adapters, int32_t d_in, int32_t d_out,
                            int32_t max_rank, int32_t n_items, int32_t max_ads_per_req)
 {
-    (void)d_out;
+    if (op == LORA_OP_MERGE)
+        return n_adapters >= 1 && n_adapters <= LORA_MAX_ADAPTERS && N == d_out
+                   ? merge_workspace_size(d_in, d_out, max_rank) : 0;
     if (op < LORA_OP_BGMV || op > LORA_OP_ROUTE)
         return 0;
     Layout L;
@@ -198,6 +200,8 @@ int lora_kernel_launches(int op, int32_t N, int32_t n_adapters, int32_t d_in, in
         return n_items > 0 ? 3 : 0;
     case LORA_OP_ROUTE:
         return 1;
+    case LORA_OP_MERGE:
+        return 3;
     default:
         return 0;
     }

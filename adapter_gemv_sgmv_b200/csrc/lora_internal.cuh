@@ -237,6 +237,9 @@ cudaError_t launch_tc_shrink(const TcArgs &a, int max_tiles, int kk, cudaStream_
 cudaError_t launch_tc_expand(const TcArgs &a, int kk, cudaStream_t s);
 bool tc_enabled();
 
+// Workspace bytes of lora_merge (0 for unsupported sizes).
+size_t merge_workspace_size(int32_t d_in, int32_t d_out, int32_t max_rank);
+
 // Launchers (return the CUDA error of the launch).
 cudaError_t launch_plan(const PlanArgs &a, cudaStream_t s);
 cudaError_t launch_shrink(const ShrinkArgs &a, int grid_groups, int n_chunks, int max_ads, cudaStream_t s);

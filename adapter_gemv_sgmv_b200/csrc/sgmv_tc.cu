@@ -648,7 +648,9 @@ done:
 // ============================================================ expand kernel
 //
 // Unit = (tile, 128-output slice).  D[128 x 128] = V_tile B_stack[slice]^T over
-// the stacked rank (V staged once per tile as bf16 with the scales folded in);
+// the stacked rank (V staged once per tile as bf16, with each adapter's scale
+// folded in when a request stacks several; a single adapter's scale multiplies
+// the fp32 accumulator instead);
 // the epilogue adds D to the y tile (TMA-loaded; threads only read it, so a
 // stage goes back to the producer as soon as it is read) and each epilogue
 // warp stores its rows through a small staging area with coalesced 16-byte
@@ -914,7 +916,10 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_tc_expand(const __grid_co
                     if (k < st.ktot) {
                         const int e = stack_entry(st, k);
                         c = st.slot[e] * p.slot_stride + (k - st.kb[e]);
-                        sc = st.s[e];
+                        // several adapters: each one's scale goes into its V columns; one
+                        // adapter: V is staged as it is and D is scaled in fp32 (for the merge,
+                        // whose V is exactly bf16, this keeps a single rounding of W)
+                        sc = p.mode == kModeMulti ? st.s[e] : 1.f;
                     }
                     vsrc[e8][lane] = c;
                     vsc[e8][lane] = sc;
@@ -923,7 +928,7 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_tc_expand(const __grid_co
                 // wait until the MMAs of the previous tile stopped reading V
                 if (vt > 0 && !warp_wait(&v_empty, (vt - 1) & 1, &abort_flag, p.err))
                     goto done;
-                // V[vr][stacked k] = bf16(s_e * V_e[vr][k - kb_e]), zero outside the tile's rows and
+                // V[vr][stacked k] = bf16(s_e * V_e[vr][k - kb_e]) (s_e = 1 for one adapter), zero outside the tile's rows and
                 // the stack; thread et stages row et % 128, stacked ranks 64 (et / 128) .. + 63
                 const int vr = et & 127, vh = et >> 7;
                 const bool valid = vr < gr.cnt;
@@ -989,14 +994,15 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_tc_expand(const __grid_co
             if (warp == 2)
                 TC_STAMP(2, it, 4);
             const bool none = st.kpad == 0;     // no valid adapter: no MMA ran, y is stored unchanged
+            const float dsc = p.mode == kModeMulti ? 1.f : p.scale;
             uint32_t ow[8][4];
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const float2 yf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&yw[c][e]));
-                    const float d0 = none ? 0.f : __uint_as_float(d[c * 8 + 2 * e]);
-                    const float d1 = none ? 0.f : __uint_as_float(d[c * 8 + 2 * e + 1]);
+                    const float d0 = none ? 0.f : dsc * __uint_as_float(d[c * 8 + 2 * e]);
+                    const float d1 = none ? 0.f : dsc * __uint_as_float(d[c * 8 + 2 * e + 1]);
                     const __nv_bfloat162 r2 = __floats2bfloat162_rn(yf.x + d0, yf.y + d1);
                     ow[c][e] = *reinterpret_cast<const uint32_t *>(&r2);
                 }

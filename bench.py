@@ -50,7 +50,14 @@ WORKLOAD_DESC = {
                         "ranks U{8,16,32,64,128}, Zipf(1.0) ids, q/k/v/o/gate/up/down",
     "diffusion_multi": "diffusion multi-adapter: 16 images x 4096 tokens, 1280->1280 x Q,K,V,O, rank 32, "
                        "200 adapters, 1-3 co-occurring adapters per image, scales U[0.5,1]",
+    "merge_mlp_up": "merge: fold one rank-64 adapter of a 64-adapter pool into the Llama-3-8B MLP up-proj "
+                    "weight W [14336, 4096] in place (W += s B A)",
 }
+
+
+def unit_of(workload: str) -> str:
+    """The merge streams weight rows; every other workload, token rows."""
+    return "weight rows/s" if workload == "merge_mlp_up" else "tokens/s"
 
 
 # ----------------------------------------------------------------------------
@@ -203,6 +210,8 @@ def launches_per_call(call) -> int:
     """Kernels one step of this call launches, as the library reports them."""
     import adapter_gemv_sgmv_b200 as L
     p = call.pool
+    if hasattr(call, "W"):
+        return L.lora_kernel_launches(L.OP_MERGE, p.d_out, p.n_adapters, p.d_in)
     if hasattr(call, "ids_h"):
         return L.lora_kernel_launches(L.OP_BGMV, call.n_tokens, p.n_adapters, p.d_in)
     if hasattr(call, "seg_off_h"):
@@ -220,7 +229,10 @@ def make_step(wl, ws_map, stream):
     fns = []
     for c in wl.calls:
         ws = ws_map[id(c)]
-        if hasattr(c, "ids_h"):
+        if hasattr(c, "W"):
+            # one merge of the adapter into the weight (W drifts by s B A per step; timing only)
+            fns.append(lambda c=c, ws=ws: L.lora_merge(c.W, c.pool, c.adapter, c.scale, ws=ws, stream=stream))
+        elif hasattr(c, "ids_h"):
             fns.append(lambda c=c, ws=ws: L.lora_bgmv(c.X, c.Y, c.pool, c.ids, c.scale, ws=ws, stream=stream))
         elif hasattr(c, "seg_off_h"):
             V = torch.empty(c.X.shape[0], c.pool.max_rank, dtype=torch.float32, device=c.X.device)
@@ -244,7 +256,9 @@ def make_step(wl, ws_map, stream):
 def workspace_for(call):
     import adapter_gemv_sgmv_b200 as L
     p = call.pool
-    if hasattr(call, "ids_h"):
+    if hasattr(call, "W"):
+        n = L.lora_workspace_size(L.OP_MERGE, p.d_out, p.n_adapters, p.d_in, p.d_out, p.max_rank)
+    elif hasattr(call, "ids_h"):
         n = L.lora_workspace_size(L.OP_BGMV, call.n_tokens, p.n_adapters, p.d_in, p.d_out, p.max_rank)
     elif hasattr(call, "seg_off_h"):
         n = max(L.lora_workspace_size(op, call.n_tokens, p.n_adapters, p.d_in, p.d_out, p.max_rank,
@@ -252,7 +266,7 @@ def workspace_for(call):
     else:
         n = L.lora_workspace_size(L.OP_APPLY_MULTI, call.n_tokens, p.n_adapters, p.d_in, p.d_out, p.max_rank,
                                   len(call.req_off_h) - 1, 3)
-    return L.Workspace(n, device=call.X.device)
+    return L.Workspace(n, device=(call.W if hasattr(call, "W") else call.X).device)
 
 
 # ----------------------------------------------------------------------------
@@ -287,7 +301,8 @@ def run_ours(args):
     set_bytes = 0
     for wl in sets:
         for c in wl.calls:
-            set_bytes += c.pool.A.numel() * 2 + c.pool.B.numel() * 2 + c.X.numel() * 2 + c.Y.numel() * 2
+            io = c.W.numel() * 2 if hasattr(c, "W") else c.X.numel() * 2 + c.Y.numel() * 2
+            set_bytes += c.pool.A.numel() * 2 + c.pool.B.numel() * 2 + io
     launches_step = sum(launches_per_call(c) for c in sets[0].calls)
 
     # eager warm-up (also sets per-device function attributes before capture)
@@ -348,7 +363,7 @@ def run_ours(args):
             "scope": "whole step, algorithmic bytes per step / step time",
             "algorithmic_bytes_per_step": cost.bytes}
     out = {
-        "metric": METRIC, "value": round(job_tokens_s, 1), "unit": "tokens/s",
+        "metric": METRIC, "value": round(job_tokens_s, 1), "unit": unit_of(args.workload),
         "n_gpus": world, "steps": K, "warmup": max(args.warmup, 3), "ms_per_step": round(ms_per_step, 6),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded; random-init adapters of the stated shapes)",
@@ -380,14 +395,15 @@ def run_e2e(args, wl, ws_map, stream, dist, dev, world):
     hosts = []
     h2d = d2h = 0
     for c in calls:
-        ins = {"X": c.X, "Y": c.Y}
+        ins = {"W": c.W} if hasattr(c, "W") else {"X": c.X, "Y": c.Y}
         for k in ("ids", "seg_off", "seg_ad", "req_off", "ad_off", "ad_id", "ad_scale"):
             if hasattr(c, k):
                 ins[k] = getattr(c, k)
         pin = {k: torch.empty(v.shape, dtype=v.dtype, device="cpu", pin_memory=True) for k, v in ins.items()}
         for k, v in ins.items():
             pin[k].copy_(v)
-        out_pin = torch.empty(c.Y.shape, dtype=c.Y.dtype, device="cpu", pin_memory=True)
+        res = c.W if hasattr(c, "W") else c.Y
+        out_pin = torch.empty(res.shape, dtype=res.dtype, device="cpu", pin_memory=True)
         hosts.append((c, pin, out_pin))
     shared_x = set()
     for c, pin, out_pin in hosts:
@@ -413,7 +429,7 @@ def run_e2e(args, wl, ws_map, stream, dist, dev, world):
                     dst.copy_(v, non_blocking=True)
             step()
             for c, pin, out_pin in hosts:
-                out_pin.copy_(c.Y, non_blocking=True)
+                out_pin.copy_(c.W if hasattr(c, "W") else c.Y, non_blocking=True)
     for _ in range(3):
         one()
     stream.synchronize()
@@ -427,7 +443,7 @@ def run_e2e(args, wl, ws_map, stream, dist, dev, world):
     e1.record(stream)
     torch.cuda.synchronize()
     ms = max_over_ranks(e0.elapsed_time(e1), dist, dev) / n
-    return {"value": round(world * wl.n_tokens / (ms * 1e-3), 1), "unit": "tokens/s",
+    return {"value": round(world * wl.n_tokens / (ms * 1e-3), 1), "unit": unit_of(args.workload),
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": n,
             "ms_per_step": round(ms, 6),
             "path": "pinned host -> device copies, public Python call (eager launches), device -> host"}
@@ -442,7 +458,10 @@ def _host_calls(wl):
     from workloads import to_host
     out = []
     for c in wl.calls:
-        if hasattr(c, "ids_h"):
+        if hasattr(c, "W"):
+            hp, remap = compact_from_device_pool(c.pool, [c.adapter])
+            out.append(("merge", to_host(c.W), hp, int(remap[c.adapter]), c))
+        elif hasattr(c, "ids_h"):
             used = np.unique(c.ids_h[c.ids_h >= 0])
             hp, remap = compact_from_device_pool(c.pool, used)
             ids = np.where(c.ids_h >= 0, remap[np.maximum(c.ids_h, 0)], -1).astype(np.int32)
@@ -463,7 +482,9 @@ def _oracle_pass(oracle, hc, rows_per_call):
     """Run the oracle on the given rows of every call; returns tokens processed."""
     done = 0
     for (kind, X, hp, meta, c), rows in zip(hc, rows_per_call):
-        if kind == "bgmv":
+        if kind == "merge":
+            oracle.merge(X, hp, meta, c.scale, rows=rows)
+        elif kind == "bgmv":
             oracle.bgmv_delta(X, hp, meta, c.scale, rows=rows)
         elif kind == "sgmv":
             oracle.sgmv_delta(X, hp, meta[0], meta[1], c.scale, rows=rows)
@@ -498,7 +519,8 @@ def cpu_baseline(args, wl, budget_s=12.0):
         if time.perf_counter() - t0 > 1.5 * budget_s:
             break
     dt = time.perf_counter() - t0
-    return {"value": round(tokens / dt, 2), "unit": "tokens/s", "cores": oracle.threads(), "kind": "oracle",
+    return {"value": round(tokens / dt, 2), "unit": unit_of(args.workload), "cores": oracle.threads(),
+            "kind": "oracle",
             "sample": f"{tokens} tokens ({n_tok} sampled rows x {passes} passes) of one "
                       f"{args.workload} batch, all projections, fp64 C loops, OpenMP over rows",
             "seconds": round(dt, 2)}
@@ -535,14 +557,17 @@ def run_reference(args):
     sample = (f"each step: {n_tok} sampled token rows of one {args.workload} batch (all projections), "
               f"fp64 C loops, OpenMP over rows")
     print(json.dumps({
-        "impl": "reference", "metric": METRIC, "value": round(v, 3), "unit": "tokens/s", "n_gpus": args.gpus,
+        "impl": "reference", "metric": METRIC, "value": round(v, 3), "unit": unit_of(args.workload),
+        "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / max(args.steps, 1) * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded)",
         "config": {"workload": WORKLOAD_DESC[args.workload], "tokens_per_step": n_tok},
-        "cpu_baseline": {"value": round(v, 3), "unit": "tokens/s", "cores": oracle.threads(), "kind": "oracle",
+        "cpu_baseline": {"value": round(v, 3), "unit": unit_of(args.workload), "cores": oracle.threads(),
+                         "kind": "oracle",
                          "sample": sample},
-        "e2e": {"value": round(v, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "e2e": {"value": round(v, 3), "unit": unit_of(args.workload), "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
     }), flush=True)
 
 

@@ -107,12 +107,14 @@ typedef enum {
     LORA_OP_SGMV_SHRINK = 1,
     LORA_OP_SGMV_EXPAND = 2,
     LORA_OP_APPLY_MULTI = 3,
-    LORA_OP_ROUTE = 4
+    LORA_OP_ROUTE = 4,
+    LORA_OP_MERGE = 5
 } lora_op;
 
 /* Bytes of workspace `op` needs for N token rows.  n_items = n_seg for the
  * SGMV ops, n_req for lora_apply_multi, ignored otherwise; max_ads_per_req is
- * used by lora_apply_multi only.  Pure host function, no CUDA call.  Returns
+ * used by lora_apply_multi only.  For LORA_OP_MERGE, N = d_out (the rows of
+ * the weight being merged into).  Pure host function, no CUDA call.  Returns
  * 0 for arguments the corresponding entry point would reject. */
 LORA_API size_t lora_workspace_size(int op, int32_t N, int32_t n_adapters, int32_t d_in, int32_t d_out,
                            int32_t max_rank, int32_t n_items, int32_t max_ads_per_req);
@@ -240,6 +242,30 @@ LORA_API lora_status lora_apply_multi_static(const void *X, int64_t ldx, void *Y
                                              int32_t max_ads_per_req, uint32_t *err_out, void *stream);
 
 /* Library version string (host). */
+/*
+ * lora_merge -- fold an adapter into a base weight, or take it out again.
+ *
+ * "Serving several LoRAs, ControlNet and IP-Adapter", section "LoRA: merged or
+ * alongside": a merged LoRA is W' = W + B A in the weight itself (no per-token
+ * cost), and switching adapters means unmerging one and merging another.  For
+ * the base weight W [pool->d_out, pool->d_in] (bf16, row-major, leading
+ * dimension ldw, a multiple of 8; 16-byte aligned; updated in place) and
+ * adapter `adapter` of the pool:
+ *     W[o][i] <- bf16( W[o][i] + scale * sum_j B[a][o][j] * A[a][j][i] )
+ * accumulated in fp32 with one bf16 rounding per element.  Unmerging is the
+ * same call with -scale; as W is rounded each time, merge then unmerge
+ * restores W to within bf16 rounding, not bit for bit.
+ *
+ * ws: at least lora_workspace_size(LORA_OP_MERGE, pool->d_out, ...) bytes
+ * (the error word sits at its start, as for the other ops).  Errors: the
+ * host checks of the other entry points, and `adapter` outside
+ * [0, n_adapters) -> LORA_ERR_INVALID_ARG; an adapter whose device metadata is
+ * invalid leaves W unchanged and sets LORA_ERR_BAD_ADAPTER in the error word.
+ * Launches three kernels (adapter preparation, tiling, the expand).
+ */
+LORA_API lora_status lora_merge(void *W, int64_t ldw, const lora_pool *pool, int32_t adapter, float scale,
+                                void *ws, size_t ws_bytes, void *stream);
+
 LORA_API const char *lora_version(void);
 
 #ifdef __cplusplus

@@ -36,7 +36,8 @@ def declared():
 def test_header_declares_the_entry_points():
     names = set(declared())
     assert {"lora_bgmv", "lora_sgmv_shrink", "lora_sgmv_expand", "lora_apply_multi", "lora_route",
-            "lora_workspace_size", "lora_workspace_init", "lora_get_error", "lora_version"} <= names
+            "lora_workspace_size", "lora_workspace_init", "lora_get_error", "lora_version",
+            "lora_merge"} <= names
 
 
 def test_every_declared_symbol_is_exported(lib):
@@ -57,6 +58,11 @@ def test_workspace_size(lib):
     assert L.lora_workspace_size(L.OP_BGMV, 4, 128, 4096, 4096, 256) == 0
     assert L.lora_workspace_size(L.OP_APPLY_MULTI, 4, 8, 64, 64, 16, 1, 9) == 0
     assert L.lora_workspace_size(99, 4, 8, 64, 64, 16) == 0
+    # merge: N is d_out; the workspace holds A^T (bf16) and B (fp32) of one adapter
+    m = L.lora_workspace_size(L.OP_MERGE, 14336, 64, 4096, 14336, 64)
+    assert m >= 4096 * 64 * 2 + 14336 * 64 * 4 and m % 256 == 0
+    assert L.lora_workspace_size(L.OP_MERGE, 100, 64, 4096, 14336, 64) == 0
+    assert L.lora_kernel_launches(L.OP_MERGE, 14336, 64, 4096) == 3
 
 
 FAKE = 0x10000          # a 256-byte-aligned address that is never dereferenced
@@ -124,6 +130,13 @@ def test_other_entry_points_validate(lib):
     assert lib.lora_route(FAKE, 4, 0, FAKE, FAKE, FAKE, FAKE, None, 0, None) == UNSUPPORTED
     assert lib.lora_route(None, 4, 8, FAKE, FAKE, FAKE, FAKE, None, 0, None) == INVALID
     assert lib.lora_route(FAKE, 4, 8, FAKE, FAKE, FAKE, FAKE, None, 0, None) == WORKSPACE
+    # merge: adapter out of range, W below one row / misaligned, no workspace
+    assert lib.lora_merge(FAKE, 64, p, 4, 1.0, None, 0, None) == INVALID
+    assert lib.lora_merge(FAKE, 64, p, -1, 1.0, None, 0, None) == INVALID
+    assert lib.lora_merge(FAKE, 32, p, 1, 1.0, None, 0, None) == INVALID
+    assert lib.lora_merge(FAKE + 2, 64, p, 1, 1.0, None, 0, None) == UNSUPPORTED
+    assert lib.lora_merge(FAKE, 64, p, 1, 1.0, None, 0, None) == WORKSPACE
+    assert lib.lora_merge(FAKE, 64, None, 1, 1.0, None, 0, None) == INVALID
     # workspace helpers reject a null / misaligned workspace before touching CUDA
     assert lib.lora_workspace_init(None, None) == WORKSPACE
     assert lib.lora_get_error(FAKE + 8, None) == WORKSPACE

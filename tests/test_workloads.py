@@ -53,3 +53,14 @@ def test_pool_layout_packed_without_padding():
     assert p.A.numel() == (8 + 128 + 16) * 32
     B1 = p.adapter_B(1).float()
     assert abs(B1.std().item() - 128 ** -0.5) < 0.02
+
+
+def test_merge_workload_shapes():
+    wl = make_workload("merge_mlp_up", d_in=64, d_out=32, rank=16, n_adapters=4)
+    c = wl.calls[0]
+    assert tuple(c.W.shape) == (32, 64) and c.W.dtype == torch.bfloat16
+    assert 0 <= c.adapter < 4 and wl.n_tokens == 32
+    from adapter_gemv_sgmv_b200 import accounting
+    cost = accounting.workload_cost(wl)
+    assert cost.bytes == 2 * 2 * 32 * 64 + 2 * 16 * (64 + 32) and cost.flops == 2 * 32 * 64 * 16
+

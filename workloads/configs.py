@@ -234,6 +234,23 @@ class MultiCall:
 
 
 @dataclass
+class MergeCall:
+    """Fold adapter `adapter` of `pool` into the base weight W [d_out, d_in] in place:
+    W += scale * B[a] A[a] (unmerge: -scale)."""
+
+    name: str
+    W: torch.Tensor          # bf16 [d_out, d_in]
+    pool: Pool
+    adapter: int
+    scale: float
+
+    @property
+    def n_tokens(self) -> int:
+        # rows of W (the unit the merge streams)
+        return int(self.W.shape[0])
+
+
+@dataclass
 class Workload:
     name: str
     calls: list
@@ -307,6 +324,7 @@ WORKLOAD_NAMES = [
     "prefill_sgmv",       # 32 prompts U[128,1024], 4096->14336, r64, 64 adapters, Zipf(1.1)
     "mixed_rank_layer",   # 512 decode tokens, 1000 adapters r in {8..128}, 7 Llama-3-8B projections
     "diffusion_multi",    # 16 images x 4096 tokens, 1280->1280 x QKVO, r32, 200 adapters, 1-3 per image
+    "merge_mlp_up",       # fold one rank-64 adapter into W [14336, 4096] (Llama-3-8B MLP up-proj) in place
 ]
 
 LLAMA3_8B_PROJ = [  # name, d_in, d_out, which input it reads
@@ -407,4 +425,15 @@ def make_workload(which, device="cpu", seed: Optional[int] = None, y0: str = "ze
             calls.append(multi_call(pname, X, pool, req_off, ad_off, np.asarray(ad_id, np.int32),
                                     np.asarray(ad_scale, np.float32), device, y0, seed * 100 + p_i))
         return Workload("diffusion_multi", calls, {"tokens": N, "op": "multi", "images": n_img})
+    if idx == 5:
+        d_in = overrides.get("d_in", 4096)
+        d_out = overrides.get("d_out", 14336)
+        r = overrides.get("rank", 64)
+        n_ad = overrides.get("n_adapters", 64)
+        pool = make_pool([r] * n_ad, d_in, d_out, seed, device)
+        # base weight ~ N(0, 1/d_in): the same scale as B A, so the update is not lost in rounding
+        W = _randn_rows_bf16(d_out, d_in, 1.0 / math.sqrt(d_in), gen, device)
+        a = int(rng.integers(0, n_ad))
+        call = MergeCall("up", W, pool, a, overrides.get("scale", 1.0))
+        return Workload("merge_mlp_up", [call], {"tokens": d_out, "op": "merge"})
     raise ValueError(f"unknown workload {which!r}")
