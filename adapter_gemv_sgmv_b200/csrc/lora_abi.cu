@@ -200,8 +200,8 @@ int lora_kernel_launches(int op, int32_t N, int32_t n_adapters, int32_t d_in, in
         return n_items > 0 ? 3 : 0;
     case LORA_OP_ROUTE:
         return 1;
-    case LORA_OP_MERGE:
-        return 3;
+    case LORA_OP_MERGE:   // preparation + expand (tensor cores), or + plan + expand
+        return tc_enabled() && N >= kTcGroup ? 2 : 3;
     default:
         return 0;
     }

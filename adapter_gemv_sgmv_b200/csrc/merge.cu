@@ -36,6 +36,9 @@ struct PrepArgs {
     int32_t nbA;                  // blocks transposing A_a; the rest widen B_a
     MergeMeta *meta;
     uint32_t *err;                // the workspace's error word
+    WsHeader *hdr;                // direct tensor-core path: the tiles of W's rows (else nullptr)
+    Group *groups;
+    int32_t n_tiles;
     __nv_bfloat16 *At;            // [d_in][r]
     float *Bf;                    // [d_out][ld]
 };
@@ -64,6 +67,23 @@ __global__ void __launch_bounds__(kPrepThreads) k_merge_prep(PrepArgs p)
     __shared__ int32_t s_r;
     __shared__ int64_t s_ao, s_bo;
     const int tid = threadIdx.x;
+    // programmatic dependent launch: the previous kernel (which may still use W or the
+    // workspace) completes first; the next one may start its prologue
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    if (blockIdx.x == 0 && p.hdr) {
+        // W's rows as one segment, cut into tiles of kTcGroup rows
+        for (int t = tid; t < p.n_tiles; t += kPrepThreads) {
+            Group g;
+            g.p0 = t * kTcGroup;
+            g.cnt = min(kTcGroup, p.pool.d_out - t * kTcGroup);
+            g.item = 0;
+            g.pad = 0;
+            p.groups[t] = g;
+        }
+        if (tid == 0)
+            p.hdr->n_groups = p.n_tiles;
+    }
     if (tid == 0) {
         int32_t r = 0;
         int64_t ao = 0, bo = 0;
@@ -104,13 +124,21 @@ __global__ void __launch_bounds__(kPrepThreads) k_merge_prep(PrepArgs p)
                 p.At[(int64_t)(i0 + ii) * r + j] = tile[j][ii];
         }
     } else {
-        // B_a rows o0 .. o0 + 63 widened to fp32
+        // B_a rows o0 .. o0 + 63 widened to fp32, 8 elements (16 bytes in, 32 out) at a time
         const int o0 = (blockIdx.x - p.nbA) * kPrepCols;
         const __nv_bfloat16 *Ba = p.pool.B + s_bo;
-        for (int e = tid; e < r * kPrepCols; e += kPrepThreads) {
-            const int oo = e / r, j = e - oo * r;
-            if (o0 + oo < d_out)
-                p.Bf[(int64_t)(o0 + oo) * p.ld + j] = __bfloat162float(Ba[(int64_t)(o0 + oo) * r + j]);
+        const int cpr = r / 8;
+        for (int e = tid; e < cpr * kPrepCols; e += kPrepThreads) {
+            const int oo = e / cpr, j = (e - oo * cpr) * 8;
+            if (o0 + oo < d_out) {
+                const uint4 v = *reinterpret_cast<const uint4 *>(Ba + (int64_t)(o0 + oo) * r + j);
+                const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&v);
+                const float2 f0 = __bfloat1622float2(h[0]), f1 = __bfloat1622float2(h[1]);
+                const float2 f2 = __bfloat1622float2(h[2]), f3 = __bfloat1622float2(h[3]);
+                float4 *dst = reinterpret_cast<float4 *>(p.Bf + (int64_t)(o0 + oo) * p.ld + j);
+                dst[0] = make_float4(f0.x, f0.y, f1.x, f1.y);
+                dst[1] = make_float4(f2.x, f2.y, f3.x, f3.y);
+            }
         }
     }
 }
@@ -192,12 +220,28 @@ extern "C" lora_status lora_merge(void *W, int64_t ldw, const lora_pool *pool, i
     pa.ld = pool->max_rank;
     pa.nbA = (pool->d_in + kPrepCols - 1) / kPrepCols;
     pa.meta = meta;
-    pa.err = &reinterpret_cast<WsHeader *>(w + L.expand_ws)->err;
+    WsHeader *hdr = reinterpret_cast<WsHeader *>(w + L.expand_ws);
+    pa.err = &hdr->err;
+    // the tensor-core expand is launched directly on W's tiles (written by the
+    // preparation kernel where lora_sgmv_expand's plan kernel would put them)
+    const bool direct = tc_enabled() && pool->d_out >= kTcGroup;
+    Group *groups = reinterpret_cast<Group *>(w + L.expand_ws + sizeof(WsHeader));
+    pa.n_tiles = (pool->d_out + kTcGroup - 1) / kTcGroup;
+    pa.hdr = direct ? hdr : nullptr;
+    pa.groups = groups;
     pa.At = At;
     pa.Bf = Bf;
     const int nbB = (pool->d_out + kPrepCols - 1) / kPrepCols;
-    k_merge_prep<<<pa.nbA + nbB, kPrepThreads, 0, s>>>(pa);
-    if (cudaGetLastError() != cudaSuccess)
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(pa.nbA + nbB);
+    cfg.blockDim = dim3(kPrepThreads);
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl_enabled() ? 1 : 0;
+    if (cudaLaunchKernelEx(&cfg, k_merge_prep, pa) != cudaSuccess)
         return LORA_ERR_CUDA;
 
     // the one-adapter pool: its "B" is A_a^T ([d_in, r], offset 0), 8 dummy inputs
@@ -214,6 +258,37 @@ extern "C" lora_status lora_merge(void *W, int64_t ldw, const lora_pool *pool, i
     tmp.d_in = 8;
     tmp.d_out = pool->d_in;
     tmp.max_rank = pool->max_rank;
+    if (direct) {
+        TcArgs ta = {};
+        tc_encode_b(ta, At, tmp.B_elems);
+        if (tc_encode_y(ta, W, pool->d_out, pool->d_in, ldw)) {
+            ta.mode = kModeSgmv;
+            ta.groups = groups;
+            ta.hdr = hdr;
+            ta.seg_ad = meta->seg_ad;
+            ta.max_ads = 1;
+            ta.scale = scale;
+            ta.pool.A = At;
+            ta.pool.B = At;
+            ta.pool.A_off = meta->A_off;
+            ta.pool.B_off = meta->B_off;
+            ta.pool.rank = meta->rank;
+            ta.pool.A_elems = tmp.A_elems;
+            ta.pool.B_elems = tmp.B_elems;
+            ta.pool.n_adapters = 1;
+            ta.pool.max_rank = tmp.max_rank;
+            ta.pool.d_in = tmp.d_in;
+            ta.pool.d_out = tmp.d_out;
+            ta.V = Bf;
+            ta.ldv = pool->max_rank;
+            ta.slot_stride = 0;
+            ta.Y = static_cast<__nv_bfloat16 *>(W);
+            ta.ldy = ldw;
+            ta.err = &hdr->err;
+            return launch_tc_expand(ta, pool->max_rank, s) == cudaSuccess ? LORA_OK : LORA_ERR_CUDA;
+        }
+        // no tensor map: the tiles are written, but the general path re-plans them
+    }
     return lora_sgmv_expand(Bf, pool->max_rank, W, ldw, &tmp, meta->seg_off, meta->seg_ad, 1, pool->d_out, scale,
                             w + L.expand_ws, L.meta, stream);
 }

@@ -261,7 +261,9 @@ LORA_API lora_status lora_apply_multi_static(const void *X, int64_t ldx, void *Y
  * host checks of the other entry points, and `adapter` outside
  * [0, n_adapters) -> LORA_ERR_INVALID_ARG; an adapter whose device metadata is
  * invalid leaves W unchanged and sets LORA_ERR_BAD_ADAPTER in the error word.
- * Launches three kernels (adapter preparation, tiling, the expand).
+ * Launches two kernels (adapter preparation, the tensor-core expand over W's
+ * tiles), or three on the CUDA-core path (d_out < 128: preparation, tiling,
+ * expand).
  */
 LORA_API lora_status lora_merge(void *W, int64_t ldw, const lora_pool *pool, int32_t adapter, float scale,
                                 void *ws, size_t ws_bytes, void *stream);

@@ -62,7 +62,8 @@ def test_workspace_size(lib):
     m = L.lora_workspace_size(L.OP_MERGE, 14336, 64, 4096, 14336, 64)
     assert m >= 4096 * 64 * 2 + 14336 * 64 * 4 and m % 256 == 0
     assert L.lora_workspace_size(L.OP_MERGE, 100, 64, 4096, 14336, 64) == 0
-    assert L.lora_kernel_launches(L.OP_MERGE, 14336, 64, 4096) == 3
+    assert L.lora_kernel_launches(L.OP_MERGE, 14336, 64, 4096) == 2
+    assert L.lora_kernel_launches(L.OP_MERGE, 64, 64, 4096) == 3
 
 
 FAKE = 0x10000          # a 256-byte-aligned address that is never dereferenced
