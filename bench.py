@@ -55,6 +55,12 @@ WORKLOAD_DESC = {
 }
 
 
+# DRAM traffic of the step's only kernel, from one ncu capture of the current kernel
+# (dram__bytes_read.sum + dram__bytes_write.sum of one launch); None where the step has
+# several kernels or no capture of the current kernel exists.
+NCU_TRAFFIC = {"decode_bgmv": 21_570_560}
+
+
 def unit_of(workload: str) -> str:
     """The merge streams weight rows; every other workload, token rows."""
     return "weight rows/s" if workload == "merge_mlp_up" else "tokens/s"
@@ -358,7 +364,7 @@ def run_ours(args):
     gbs = cost.bytes / t_step / 1e9
     tflops = cost.flops / t_step / 1e12
     roof = {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-            "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": None,
+            "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": NCU_TRAFFIC.get(args.workload),
             "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else "fallback",
             "scope": "whole step, algorithmic bytes per step / step time",
             "algorithmic_bytes_per_step": cost.bytes}
