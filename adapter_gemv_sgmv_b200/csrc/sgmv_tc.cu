@@ -39,7 +39,8 @@ namespace lora {
 namespace {
 
 constexpr int kTcThreads = 192;       // shrink: producer, MMA, 4 epilogue warps
-constexpr int kExpandThreads = 320;   // expand: producer, MMA, 8 epilogue warps
+constexpr int kExpandThreads = 576;   // expand: producer, MMA, 16 epilogue warps
+constexpr int kEpiWarps = 16;
 // heights of the A-pool TMA boxes (map_a[m])
 __host__ __device__ constexpr int abox_rows(int m) { return m == 0 ? 64 : (m == 1 ? 32 : 8); }
 // B-pool TMA views: map_b[m] sees the pool as [B_elems / r, r] for r = 16 << m, so
@@ -661,7 +662,7 @@ done:
 // the rest (up to kMaxYStages), so a rank-64 call keeps five 32 KB y tiles in flight.
 constexpr int kY = kBM * kBN * 2;                  // y: 128 rows x 128 outputs (two 64-column atoms)
 constexpr int kMaxYStages = 6;
-constexpr int kStaging = 8 * 2048;                 // per epilogue warp: 32 rows x 32 outputs of bf16
+constexpr int kStaging = kEpiWarps * 1024;         // per epilogue warp: 32 rows x 16 outputs of bf16
 
 __global__ void __launch_bounds__(kExpandThreads, 1) k_tc_expand(const __grid_constant__ TcArgs p)
 {
@@ -674,8 +675,8 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_tc_expand(const __grid_co
     __shared__ __align__(8) StackSm stk[kExpandThreads / 32];
     __shared__ long long cb_off[kKMax / 8];  // producer: B element offset of stacked 8-rank chunk c in output row 0
     __shared__ int cb_r[kKMax / 8];          // its row stride (the adapter's rank); 0 = padding chunk
-    __shared__ int vsrc[8][kKMax / 8];       // epilogue warp e: V column of stacked chunk c (-1: zero)
-    __shared__ float vsc[8][kKMax / 8];      // and its adapter's scale
+    __shared__ int vsrc[kEpiWarps][kKMax / 8];   // epilogue warp e: V column of stacked chunk c (-1: zero)
+    __shared__ float vsc[kEpiWarps][kKMax / 8];  // and its adapter's scale
     __shared__ uint32_t tmem_base;
     __shared__ int abort_flag;
 
@@ -697,13 +698,13 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_tc_expand(const __grid_co
         }
         for (int s = 0; s < kMaxYStages; ++s) {
             mbar_init(&y_full[s], 1);        // expect_tx
-            mbar_init(&y_empty[s], 8);       // epilogue warps: the tile is stored
+            mbar_init(&y_empty[s], kEpiWarps);   // epilogue warps: the tile is read
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&acc_full[b], 1);
-            mbar_init(&acc_empty[b], 8);     // epilogue warps
+            mbar_init(&acc_empty[b], kEpiWarps); // epilogue warps
         }
-        mbar_init(&v_full, 8);               // epilogue warps, after staging V
+        mbar_init(&v_full, kEpiWarps);       // epilogue warps, after staging V
         mbar_init(&v_empty, 1);              // MMA commit after a tile's last unit
         abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -891,13 +892,16 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_tc_expand(const __grid_co
         }
     } else {
         // ------------------------------------------------ epilogue: V staging, y += D, store
-        // Eight warps: warp w reads TMEM lane quarter w % 4 (rows 32 (w % 4) ..) and
-        // owns output half h (one 64-column y atom) of every unit.
-        const int e8 = warp - 2;                // 0..7
+        // Sixteen warps: warp w reads TMEM lane quarter w % 4 (rows 32 (w % 4) ..) and
+        // owns output quarter cq (32 columns: half cq / 2 of a 64-column y atom) of every
+        // unit -- 64 values per thread, so the sixteen warps keep twice as many
+        // independent update chains in flight as eight warps of 64 columns could.
+        const int e8 = warp - 2;                // 0..15
         const int q = warp & 3;
-        const int h = e8 >> 2;
+        const int cq = e8 >> 2;
+        const int h = cq >> 1;
         const int row = q * 32 + lane;
-        const int et = tid - 64;                // 0..255 over the epilogue warps
+        const int et = tid - 64;                // 0..511 over the epilogue warps
         StackSm &st = stk[warp];
         int it = 0, vt = 0;
         int64_t prev_tile = -1;
@@ -929,13 +933,13 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_tc_expand(const __grid_co
                 if (vt > 0 && !warp_wait(&v_empty, (vt - 1) & 1, &abort_flag, p.err))
                     goto done;
                 // V[vr][stacked k] = bf16(s_e * V_e[vr][k - kb_e]) (s_e = 1 for one adapter), zero outside the tile's rows and
-                // the stack; thread et stages row et % 128, stacked ranks 64 (et / 128) .. + 63
-                const int vr = et & 127, vh = et >> 7;
+                // the stack; thread et stages row et % 128, stacked ranks 32 (et / 128) .. + 31
+                const int vr = et & 127, vq = et >> 7;
                 const bool valid = vr < gr.cnt;
                 const float *vrow = p.V + (int64_t)(gr.p0 + (valid ? vr : 0)) * p.ldv;
-                const uint32_t vbase = smem_u32(smV) + vh * kAtom;
-                const int c_end = min(st.kpad / 8, vh * 8 + 8);
-                for (int c = vh * 8; c < c_end; ++c) {
+                const uint32_t vbase = smem_u32(smV);
+                const int c_end = min(st.kpad / 8, vq * 4 + 4);
+                for (int c = vq * 4; c < c_end; ++c) {
                     const int col = vsrc[e8][c];
                     uint32_t w[4] = {0u, 0u, 0u, 0u};
                     if (valid && col >= 0) {
@@ -951,7 +955,7 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_tc_expand(const __grid_co
                         w[2] = *reinterpret_cast<const uint32_t *>(&h2);
                         w[3] = *reinterpret_cast<const uint32_t *>(&h3);
                     }
-                    st_shared_v4(vbase + sw128_off(vr, c & 7), w[0], w[1], w[2], w[3]);
+                    st_shared_v4(vbase + (c >> 3) * kAtom + sw128_off(vr, c & 7), w[0], w[1], w[2], w[3]);
                 }
                 fence_async_smem();
                 __syncwarp();
@@ -974,19 +978,20 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_tc_expand(const __grid_co
             tc_fence_after();
             const int o0 = ns * kBN;
             const uint32_t atom = smem_u32(smY + sy * kY) + h * kAtom;
-            // this row's 64 y values (eight 16-byte chunks); the stage is then free again:
+            const int c0 = (cq & 1) * 4;            // this quarter's first 16-byte chunk in the atom
+            // this row's 32 y values (four 16-byte chunks); the stage is then free again:
             // threads only read the TMA-loaded tiles, never write them
-            uint32_t yw[8][4];
+            uint32_t yw[4][4];
 #pragma unroll
-            for (int c = 0; c < 8; ++c)
-                ld_shared_v4(atom + sw128_off(row, c), yw[c]);
+            for (int c = 0; c < 4; ++c)
+                ld_shared_v4(atom + sw128_off(row, c0 + c), yw[c]);
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(&y_empty[sy]);
             if (warp == 2)
                 TC_STAMP(2, it, 3);
-            uint32_t d[64];
-            tmem_ld64(tmem + b * 128 + ((uint32_t)(q * 32) << 16) + h * 64, d);
+            float d[32];
+            tmem_ld32(tmem + b * 128 + ((uint32_t)(q * 32) << 16) + cq * 32, d);
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
@@ -995,41 +1000,41 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_tc_expand(const __grid_co
                 TC_STAMP(2, it, 4);
             const bool none = st.kpad == 0;     // no valid adapter: no MMA ran, y is stored unchanged
             const float dsc = p.mode == kModeMulti ? 1.f : p.scale;
-            uint32_t ow[8][4];
+            uint32_t ow[4][4];
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
+            for (int c = 0; c < 4; ++c) {
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const float2 yf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&yw[c][e]));
-                    const float d0 = none ? 0.f : dsc * __uint_as_float(d[c * 8 + 2 * e]);
-                    const float d1 = none ? 0.f : dsc * __uint_as_float(d[c * 8 + 2 * e + 1]);
+                    const float d0 = none ? 0.f : dsc * d[c * 8 + 2 * e];
+                    const float d1 = none ? 0.f : dsc * d[c * 8 + 2 * e + 1];
                     const __nv_bfloat162 r2 = __floats2bfloat162_rn(yf.x + d0, yf.y + d1);
                     ow[c][e] = *reinterpret_cast<const uint32_t *>(&r2);
                 }
             }
             if (warp == 2)
                 TC_STAMP(2, it, 5);
-            // store through this warp's 2 KB staging area, 32 columns at a time: rows of 64
-            // bytes (4 chunks, XOR-swizzled by row / 2), read back 4 lanes per row so every
-            // store instruction writes 8 rows x 64 contiguous bytes
-            const uint32_t stg = smem_u32(smS) + e8 * 2048;
+            // store through this warp's 1 KB staging area, 16 columns at a time: rows of 32
+            // bytes (2 chunks, XOR-swizzled by row / 4), read back 2 lanes per row so every
+            // store instruction writes 16 rows x 32 contiguous bytes (whole sectors)
+            const uint32_t stg = smem_u32(smS) + e8 * 1024;
             const int n_rows = min(gr.cnt - q * 32, 32);
 #pragma unroll
             for (int pass = 0; pass < 2; ++pass) {
 #pragma unroll
-                for (int c = 0; c < 4; ++c)
-                    st_shared_v4(stg + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4), ow[4 * pass + c][0],
-                                 ow[4 * pass + c][1], ow[4 * pass + c][2], ow[4 * pass + c][3]);
+                for (int c = 0; c < 2; ++c)
+                    st_shared_v4(stg + lane * 32 + ((c ^ ((lane >> 2) & 1)) << 4), ow[2 * pass + c][0],
+                                 ow[2 * pass + c][1], ow[2 * pass + c][2], ow[2 * pass + c][3]);
                 __syncwarp();
-                const int cc = lane & 3;
-                const int o = o0 + h * 64 + pass * 32 + cc * 8;
+                const int cc = lane & 1;
+                const int o = o0 + cq * 32 + pass * 16 + cc * 8;
                 if (o < d_out) {
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const int rl = 8 * j + (lane >> 2);
+                    for (int j = 0; j < 2; ++j) {
+                        const int rl = 16 * j + (lane >> 1);
                         if (rl < n_rows) {
                             uint32_t w[4];
-                            ld_shared_v4(stg + rl * 64 + ((cc ^ ((rl >> 1) & 3)) << 4), w);
+                            ld_shared_v4(stg + rl * 32 + ((cc ^ ((rl >> 2) & 1)) << 4), w);
                             st_global_v4_hint(p.Y + (int64_t)(gr.p0 + q * 32 + rl) * p.ldy + o, w[0], w[1], w[2],
                                               w[3], pol_st);
                         }
