@@ -20,7 +20,7 @@ __all__ = [
     "lora_kernel_launches",
     "lora_get_error", "lora_route", "lora_bgmv", "lora_sgmv_shrink", "lora_sgmv_expand",
     "lora_apply_multi", "lora_apply_multi_static", "make_pool_struct", "Workspace", "OP_BGMV", "OP_SGMV_SHRINK", "OP_SGMV_EXPAND",
-    "OP_APPLY_MULTI", "OP_ROUTE", "OP_MERGE", "STATUS", "lora_merge",
+    "OP_APPLY_MULTI", "OP_ROUTE", "OP_MERGE", "STATUS", "lora_merge", "PoolManager",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -92,6 +92,14 @@ def load():
         lib.lora_apply_multi_static.argtypes = [P, i64, P, i64, PP, P, P, P, P, i32, i32, i32, P, P]
         lib.lora_merge.restype = ctypes.c_int
         lib.lora_merge.argtypes = [P, i64, PP, i32, f32, P, sz, P]
+        lib.lora_pm_create.restype = ctypes.c_int
+        lib.lora_pm_create.argtypes = [PP, P, ctypes.POINTER(ctypes.c_void_p)]
+        lib.lora_pm_destroy.restype = None
+        lib.lora_pm_destroy.argtypes = [P]
+        lib.lora_pm_register.restype = ctypes.c_int
+        lib.lora_pm_register.argtypes = [P, i64, P, P, i32]
+        lib.lora_pm_acquire.restype = ctypes.c_int
+        lib.lora_pm_acquire.argtypes = [P, P, i32, P, P, P]
         _lib = lib
     return _lib
 
@@ -327,4 +335,62 @@ def lora_merge(W, pool, adapter: int, scale: float, ws: Workspace | None = None,
     _rc(lib.lora_merge(_ptr(W), ldw, ctypes.byref(ps), int(adapter), float(scale), ws.ptr(), ws.nbytes,
                        _stream_ptr(stream)), "lora_merge")
     return ws
+
+
+class PoolManager:
+    """A resident pool of n_slots adapter slots with on-demand loads (lora_pm_*).
+
+    Owns the pool's device tensors (A, B, A_off, B_off, rank) and is itself the pool
+    the ops take (slot indices are the adapter ids).  register() records an adapter's
+    host copy (CPU bf16 tensors A [r, d_in], B [d_out, r]; pinned memory makes the
+    loads asynchronous); acquire(keys) makes a batch's adapters resident and returns
+    their slots, loading missing ones on `stream` over least recently used slots."""
+
+    def __init__(self, n_slots: int, d_in: int, d_out: int, max_rank: int, device="cuda", stream=None):
+        torch = _torch()
+        self.d_in, self.d_out, self.max_rank = int(d_in), int(d_out), int(max_rank)
+        self.A = torch.zeros(n_slots * max_rank * d_in, dtype=torch.bfloat16, device=device)
+        self.B = torch.zeros(n_slots * d_out * max_rank, dtype=torch.bfloat16, device=device)
+        self.A_off = torch.zeros(n_slots, dtype=torch.int64, device=device)
+        self.B_off = torch.zeros(n_slots, dtype=torch.int64, device=device)
+        self.rank = torch.zeros(n_slots, dtype=torch.int32, device=device)
+        self._host = {}
+        self._h = ctypes.c_void_p()
+        ps = make_pool_struct(self)
+        _rc(load().lora_pm_create(ctypes.byref(ps), _stream_ptr(stream), ctypes.byref(self._h)), "lora_pm_create")
+
+    @property
+    def n_adapters(self) -> int:
+        return int(self.rank.numel())
+
+    def register(self, key: int, A_host, B_host):
+        torch = _torch()
+        r = int(A_host.shape[0])
+        if (A_host.dtype != torch.bfloat16 or B_host.dtype != torch.bfloat16 or A_host.device.type != "cpu" or
+                B_host.device.type != "cpu" or tuple(A_host.shape) != (r, self.d_in) or
+                tuple(B_host.shape) != (self.d_out, r) or not A_host.is_contiguous() or not B_host.is_contiguous()):
+            raise LoraError("register: A [r, d_in] and B [d_out, r] contiguous bf16 CPU tensors", 1)
+        self._host[int(key)] = (A_host, B_host)        # kept alive while a copy may be in flight
+        _rc(load().lora_pm_register(self._h, int(key), A_host.data_ptr(), B_host.data_ptr(), r), "lora_pm_register")
+
+    def acquire(self, keys, stream=None):
+        """slots (int32 numpy array, one per key) and the number of adapters loaded."""
+        import numpy as np
+        keys = np.ascontiguousarray(np.asarray(keys, dtype=np.int64))
+        slots = np.zeros(max(len(keys), 1), dtype=np.int32)
+        n_loaded = ctypes.c_int32(0)
+        _rc(load().lora_pm_acquire(self._h, keys.ctypes.data, len(keys), slots.ctypes.data,
+                                   ctypes.byref(n_loaded), _stream_ptr(stream)), "lora_pm_acquire")
+        return slots[:len(keys)], int(n_loaded.value)
+
+    def close(self):
+        if self._h:
+            load().lora_pm_destroy(self._h)
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 

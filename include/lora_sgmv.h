@@ -268,6 +268,44 @@ LORA_API lora_status lora_apply_multi_static(const void *X, int64_t ldx, void *Y
 LORA_API lora_status lora_merge(void *W, int64_t ldw, const lora_pool *pool, int32_t adapter, float scale,
                                 void *ws, size_t ws_bytes, void *stream);
 
+/*
+ * Resident adapter pool with on-demand loads -- the system layer around the ops.
+ *
+ * "Serving several LoRAs, ControlNet and IP-Adapter", section "Placement": the
+ * adapters in use stay resident on the GPU; the rest wait in host memory and are
+ * brought in when a batch needs them.  The caller owns the pool's device storage:
+ * a lora_pool `storage` of n_slots = storage->n_adapters fixed-size slots, with
+ * A_elems >= n_slots * max_rank * d_in, B_elems >= n_slots * d_out * max_rank and
+ * A_off, B_off (int64) and rank (int32) arrays of n_slots.  Slot s holds one
+ * adapter at A_off[s] = s * max_rank * d_in, B_off[s] = s * d_out * max_rank; an
+ * empty slot has rank 0 (the ops reject it).  `storage` itself, with its slots as
+ * adapter indices, is the pool the ops take.
+ *
+ * lora_pm_create: host state for `storage` (n_slots <= LORA_MAX_ADAPTERS); writes
+ *   the offsets and empties every slot, on `stream`.  Free with lora_pm_destroy
+ *   (host state only; the storage stays the caller's).
+ * lora_pm_register: the host copy of adapter `key` (>= 0): A [rank, d_in] and
+ *   B [d_out, rank] bf16, row-major, in host memory that stays valid while a copy
+ *   of it may be in flight (pinned memory makes the copies asynchronous).
+ *   Registering a key again replaces its copy and marks it for reloading.
+ * lora_pm_acquire: makes keys[0..n) resident and writes each one's slot to
+ *   slots[i] (NULL allowed: preloading).  A resident key keeps its slot; a
+ *   missing one takes a free slot, else the least recently used slot that no key
+ *   of this call occupies; its A and B are copied in and its rank set, all on
+ *   `stream`, so later work on that stream sees them (work on other streams must
+ *   synchronise with it; a slot being replaced must not be in use there).
+ *   *n_loaded (optional) = adapters copied.  Unregistered key ->
+ *   LORA_ERR_INVALID_ARG, more distinct keys than slots -> LORA_ERR_UNSUPPORTED,
+ *   both before anything changes.  Calls on one manager are serialised.
+ */
+typedef struct lora_pool_mgr lora_pool_mgr;
+LORA_API lora_status lora_pm_create(const lora_pool *storage, void *stream, lora_pool_mgr **out);
+LORA_API void lora_pm_destroy(lora_pool_mgr *m);
+LORA_API lora_status lora_pm_register(lora_pool_mgr *m, int64_t key, const void *A_host, const void *B_host,
+                                      int32_t rank);
+LORA_API lora_status lora_pm_acquire(lora_pool_mgr *m, const int64_t *keys, int32_t n, int32_t *slots,
+                                     int32_t *n_loaded, void *stream);
+
 LORA_API const char *lora_version(void);
 
 #ifdef __cplusplus
