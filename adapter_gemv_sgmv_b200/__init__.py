@@ -18,7 +18,7 @@ import threading
 __all__ = [
     "LoraError", "load", "library_path", "lora_version", "lora_workspace_size", "lora_workspace_init",
     "lora_kernel_launches",
-    "lora_get_error", "lora_route", "lora_bgmv", "lora_sgmv_shrink", "lora_sgmv_expand",
+    "lora_get_error", "lora_route", "lora_bgmv", "lora_sgmv_shrink", "lora_sgmv_shrink_proj", "lora_sgmv_expand",
     "lora_apply_multi", "lora_apply_multi_static", "make_pool_struct", "Workspace", "OP_BGMV", "OP_SGMV_SHRINK", "OP_SGMV_EXPAND",
     "OP_APPLY_MULTI", "OP_ROUTE", "OP_MERGE", "STATUS", "lora_merge", "PoolManager",
 ]
@@ -84,6 +84,8 @@ def load():
         lib.lora_bgmv.argtypes = [P, i64, P, i64, PP, P, i32, f32, P, sz, P]
         lib.lora_sgmv_shrink.restype = ctypes.c_int
         lib.lora_sgmv_shrink.argtypes = [P, i64, P, i64, PP, P, P, i32, i32, P, sz, P]
+        lib.lora_sgmv_shrink_proj.restype = ctypes.c_int
+        lib.lora_sgmv_shrink_proj.argtypes = [P, i64, P, i64, PP, i32, P, P, i32, i32, P, sz, P]
         lib.lora_sgmv_expand.restype = ctypes.c_int
         lib.lora_sgmv_expand.argtypes = [P, i64, P, i64, PP, P, P, i32, i32, f32, P, sz, P]
         lib.lora_apply_multi.restype = ctypes.c_int
@@ -259,6 +261,40 @@ def lora_sgmv_shrink(X, V, pool, seg_off, seg_ad, ws: Workspace | None = None, s
                              _ptr(seg_ad), n_seg, N, ws.ptr(), ws.nbytes, _stream_ptr(stream)),
         "lora_sgmv_shrink")
     return ws
+
+
+def lora_sgmv_shrink_proj(X, V, pools, seg_off, seg_ad, ws: Workspace | None = None, stream=None,
+                          max_ranks=None):
+    """Shrinks of projections sharing the input X (Q, K, V; gate, up) in one pass over X.
+
+    Projection p's rank vector lands in V columns [c_p, c_p + rank_p[a]), where
+    c_p is the sum of the earlier pools' max_rank; returns (ws, [c_p]).  Every
+    pool has the same d_in and n_adapters; V is fp32 [N, >= sum of max_rank]."""
+    lib = load()
+    torch = _torch()
+    pools = list(pools)
+    _check_dev(X, V, seg_off, seg_ad)
+    if max_ranks is None:
+        max_ranks = [None] * len(pools)
+    structs = [make_pool_struct(p, m) for p, m in zip(pools, max_ranks)]
+    arr = (LoraPoolStruct * max(len(structs), 1))(*structs)
+    ldx = _mat(X, structs[0].d_in if structs else X.shape[1], "X")
+    if V.dtype != torch.float32 or V.dim() != 2 or V.stride(1) != 1:
+        raise LoraError("V must be a 2-D fp32 tensor with unit-stride columns", 1)
+    N = int(X.shape[0])
+    n_seg = int(seg_ad.numel())
+    cols, c = [], 0
+    for ps in structs:
+        cols.append(c)
+        c += ps.max_rank
+    ps0 = structs[0] if structs else None
+    need = lora_workspace_size(OP_SGMV_SHRINK, N, ps0.n_adapters, ps0.d_in, ps0.d_out, ps0.max_rank,
+                               n_seg) if ps0 else 256
+    ws = ws or _workspace(need, X.device)
+    _rc(lib.lora_sgmv_shrink_proj(_ptr(X), ldx, _ptr(V), V.stride(0), arr, len(structs), _ptr(seg_off),
+                                  _ptr(seg_ad), n_seg, N, ws.ptr(), ws.nbytes, _stream_ptr(stream)),
+        "lora_sgmv_shrink_proj")
+    return ws, cols
 
 
 def lora_sgmv_expand(V, Y, pool, seg_off, seg_ad, scale: float, ws: Workspace | None = None,

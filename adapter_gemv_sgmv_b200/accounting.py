@@ -138,7 +138,18 @@ def merge_cost(d_in: int, d_out: int, r: int) -> Cost:
 
 
 def workload_cost(wl) -> Cost:
+    """Sum of the calls' costs.  Where the path reads an input shared by several
+    calls once (projections fused on a shared X), that X counts once."""
     c = Cost()
+    seen = set()
     for call in wl.calls:
-        c = c + call_cost(call)
+        cc = call_cost(call)
+        X = getattr(call, "X", None)
+        if wl.desc.get("x_read_once") and X is not None:
+            key = X.data_ptr()
+            if key in seen:
+                dup = BF16_BYTES * cc.tokens * int(call.pool.d_in)
+                cc = Cost(cc.flops, cc.bytes - dup, 0, cc.adapter_bytes, cc.act_bytes - dup)
+            seen.add(key)
+        c = c + cc
     return c

@@ -432,6 +432,109 @@ lora_status lora_sgmv_shrink(const void *X, int64_t ldx, float *V, int64_t ldv,
     return LORA_OK;
 }
 
+lora_status lora_sgmv_shrink_proj(const void *X, int64_t ldx, float *V, int64_t ldv,
+                                  const lora_pool *pools, int32_t n_proj, const int32_t *seg_off,
+                                  const int32_t *seg_ad, int32_t n_seg, int32_t N,
+                                  void *ws, size_t ws_bytes, void *stream)
+{
+    if (!pools || n_proj < 1)
+        return LORA_ERR_INVALID_ARG;
+    if (n_proj > LORA_MAX_PROJ)
+        return LORA_ERR_UNSUPPORTED;
+    int32_t vcol[LORA_MAX_PROJ];
+    int64_t vcols = 0;
+    for (int p = 0; p < n_proj; ++p) {
+        LORA_TRY(check_pool(&pools[p]));
+        if (pools[p].d_in != pools[0].d_in || pools[p].n_adapters != pools[0].n_adapters)
+            return LORA_ERR_INVALID_ARG;
+        vcol[p] = (int32_t)vcols;
+        vcols += pools[p].max_rank;
+    }
+    const int32_t d_in = pools[0].d_in;
+    if (N < 0 || n_seg < 0 || !seg_off || (n_seg > 0 && !seg_ad))
+        return LORA_ERR_INVALID_ARG;
+    LORA_TRY(check_mat(X, ldx, d_in, N));
+    if ((N > 0 && !V) || ldv < vcols)
+        return LORA_ERR_INVALID_ARG;
+    Layout L;
+    if (!layout(LORA_OP_SGMV_SHRINK, N, pools[0].n_adapters, d_in, pools[0].max_rank, n_seg, 1, &L))
+        return LORA_ERR_INVALID_ARG;
+    LORA_TRY(check_ws(ws, ws_bytes, L));
+    if (N == 0 || n_seg == 0)
+        return LORA_OK;
+    cudaStream_t s = (cudaStream_t)stream;
+    WsHeader *hdr = at<WsHeader>(ws, L.hdr);
+    Group *groups = at<Group>(ws, L.groups);
+
+    PlanArgs pa = {};
+    pa.mode = kModeSgmv;
+    pa.N = N;
+    pa.item_off = seg_off;
+    pa.n_items = n_seg;
+    pa.groups = groups;
+    pa.max_groups = L.max_groups;
+    pa.hdr = hdr;
+    if (long_items(N, n_seg) && aligned_v(V, ldv)) {
+        TcArgs ta = {};
+        if (tc_encode_x(ta, X, N, d_in, ldx)) {
+            pa.group = kTcGroup;
+            LORA_CUDA(launch_plan(pa, s));
+            ta.mode = kModeProj;
+            ta.groups = groups;
+            ta.hdr = hdr;
+            ta.seg_ad = seg_ad;
+            ta.max_ads = 1;
+            ta.scale = 1.0f;
+            ta.V = V;
+            ta.ldv = ldv;
+            ta.slot_stride = 0;
+            ta.err = &hdr->err;
+            // one launch per run of consecutive projections whose max_ranks fit
+            // one stacked accumulator: every launch reads X once
+            for (int p0 = 0; p0 < n_proj;) {
+                int p1 = p0, kk = 0;
+                while (p1 < n_proj && kk + pools[p1].max_rank <= kKMaxShrink)
+                    kk += pools[p1++].max_rank;
+                TcArgs tp = ta;
+                tp.a_tma = 0;
+                tp.n_proj = p1 - p0;
+                for (int q = p0; q < p1; ++q) {
+                    tp.proj[q - p0] = pool_dev(&pools[q]);
+                    tp.proj_vcol[q - p0] = vcol[q];
+                    tc_encode_a(tp, pools[q].A, pools[q].A_elems, d_in, q - p0);
+                }
+                tp.pool = tp.proj[0];
+                LORA_CUDA(launch_tc_shrink(tp, N / kTcGroup + n_seg + 1, kk, s));
+                p0 = p1;
+            }
+            return LORA_OK;
+        }
+    }
+
+    // short segments: the CUDA-core shrink, once per projection
+    pa.group = kGroup;
+    LORA_CUDA(launch_plan(pa, s));
+    for (int p = 0; p < n_proj; ++p) {
+        ShrinkArgs sa = {};
+        sa.X = static_cast<const __nv_bfloat16 *>(X);
+        sa.ldx = ldx;
+        sa.perm = nullptr;
+        sa.groups = groups;
+        sa.hdr = hdr;
+        sa.mode = kModeSgmv;
+        sa.seg_ad = seg_ad;
+        sa.pool = pool_dev(&pools[p]);
+        sa.kc = d_in;
+        sa.V = V + vcol[p];
+        sa.ldv = ldv;
+        sa.chunk_stride = 0;
+        sa.slot_stride = 0;
+        sa.err = &hdr->err;
+        LORA_CUDA(launch_shrink(sa, L.max_groups, 1, 1, s));
+    }
+    return LORA_OK;
+}
+
 lora_status lora_sgmv_expand(const float *V, int64_t ldv, void *Y, int64_t ldy,
                              const lora_pool *pool, const int32_t *seg_off, const int32_t *seg_ad,
                              int32_t n_seg, int32_t N, float scale,

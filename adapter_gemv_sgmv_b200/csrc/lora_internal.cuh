@@ -33,7 +33,7 @@ struct Group {
     int32_t p0, cnt, item, pad;
 };
 
-enum Mode : int32_t { kModeRoute = 0, kModeSgmv = 1, kModeMulti = 2 };
+enum Mode : int32_t { kModeRoute = 0, kModeSgmv = 1, kModeMulti = 2, kModeProj = 3 };
 
 // ---------------------------------------------------------------- plan kernel
 struct PlanArgs {
@@ -195,19 +195,22 @@ bool pdl_enabled();
 
 // ------------------------------------------------------------ tcgen05 kernels
 constexpr int kTcGroup = 128;       // rows per tensor-core tile
-constexpr int kKMax = 128;          // stacked rank a tile may carry
+constexpr int kKMax = 128;          // stacked rank a tile may carry (expand; shrink of one pool)
+constexpr int kKMaxShrink = 256;    // stacked rank of a shrink tile (projections sharing X)
+constexpr int kMaxProj = LORA_MAX_PROJ;
 
 struct TcArgs {
     CUtensorMap map_x;       // X [N, d_in], boxes 64 x 128, 128-byte swizzle (shrink)
     CUtensorMap map_y;       // Y [N, d_out], same boxes (expand)
-    CUtensorMap map_a[3];    // A pool as [A_elems / d_in, d_in], boxes of 64 columns x 64 / 32 / 8 rows
-    int32_t a_tma;           // map_a valid (shrink)
+    CUtensorMap map_a[3 * kMaxProj];   // A pool p as [A_elems / d_in, d_in], boxes of 64 columns x 64 / 32 / 8 rows: map_a[3p + m]
+    int32_t a_tma;           // bit p: map_a[3p .. 3p + 2] valid (shrink)
     CUtensorMap map_b[4];    // B pool as [B_elems / r, r], r = 16 << m, boxes of min(r, 64) x 128 rows
     int32_t b_tma;           // bit m: map_b[m] valid (expand)
     int32_t e_natoms;        // expand: 16 KB atoms per V / B stage (1 or 2; set by the launcher)
     int32_t e_ystages;       // expand: y stages (set by the launcher)
     int32_t s_stages;        // shrink: pipeline stages (set by the launcher)
     int32_t s_stage;         // shrink: bytes per stage (set by the launcher)
+    int32_t s_acc;           // shrink: TMEM columns per accumulator, 128 or 256 (set by the launcher)
     int32_t mode;            // kModeSgmv or kModeMulti
     const Group *groups;     // tiles of <= kTcGroup rows, one item each
     const WsHeader *hdr;
@@ -217,7 +220,10 @@ struct TcArgs {
     const float *ad_scale;
     int32_t max_ads;
     float scale;
-    PoolDev pool;
+    PoolDev pool;            // kModeProj: proj[0]
+    int32_t n_proj;          // kModeProj: a segment's stack is its adapter in proj[0 .. n_proj)
+    PoolDev proj[kMaxProj];
+    int32_t proj_vcol[kMaxProj];   // V column of projection p's rank 0
     float *V;                // fp32 intermediate, row stride ldv, stacked adapters slot_stride apart
     int64_t ldv;
     int32_t slot_stride;
@@ -229,9 +235,10 @@ struct TcArgs {
 bool tc_encode_x(TcArgs &a, const void *X, int32_t N, int32_t d_in, int64_t ldx);
 bool tc_encode_y(TcArgs &a, const void *Y, int32_t N, int32_t d_out, int64_t ldy);
 // optional: without it the shrink gathers A rows with cp.async
-bool tc_encode_a(TcArgs &a, const void *A, int64_t A_elems, int32_t d_in);
+bool tc_encode_a(TcArgs &a, const void *A, int64_t A_elems, int32_t d_in, int pool_index = 0);
 // optional: without it the expand gathers B rows with cp.async
 bool tc_encode_b(TcArgs &a, const void *B, int64_t B_elems);
+// kk: the largest stacked rank of any item (<= kKMaxShrink)
 cudaError_t launch_tc_shrink(const TcArgs &a, int max_tiles, int kk, cudaStream_t s);
 // kk: the largest stacked rank of any item (max_rank, or max_ads * max_rank)
 cudaError_t launch_tc_expand(const TcArgs &a, int kk, cudaStream_t s);

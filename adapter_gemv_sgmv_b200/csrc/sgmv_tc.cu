@@ -290,9 +290,10 @@ __device__ __forceinline__ bool adapter_ok(const PoolDev &P, int32_t a, int32_t 
 }
 
 // The adapter stack of one tile: entry i covers ranks [kb[i], kb[i] + r[i]) of
-// the stacked axis, reads V columns slot[i] * slot_stride + j and is scaled
-// by s[i].  The roles work on different tiles at any moment, so every warp
-// keeps its own copy in shared memory.
+// the stacked axis, maps to V columns vc0[i] + j, is scaled by s[i] and reads
+// its A rows from pool pool[i] (0 except for projections sharing an input).
+// The roles work on different tiles at any moment, so every warp keeps its own
+// copy in shared memory.
 struct StackSm {
     int n;                                  // entries
     int ktot;                               // stacked rank
@@ -301,7 +302,8 @@ struct StackSm {
     int b_tma;                              // every entry's B slice can come by TMA (see b_map)
     int r[LORA_MAX_ADS_PER_REQ];
     int kb[LORA_MAX_ADS_PER_REQ];
-    int slot[LORA_MAX_ADS_PER_REQ];
+    int vc0[LORA_MAX_ADS_PER_REQ];
+    signed char pool[LORA_MAX_ADS_PER_REQ];
     float s[LORA_MAX_ADS_PER_REQ];
     long long aoff[LORA_MAX_ADS_PER_REQ];
     long long boff[LORA_MAX_ADS_PER_REQ];
@@ -318,11 +320,12 @@ __device__ __forceinline__ int stack_entry(const StackSm &st, int k)
 }
 
 // One warp builds the stack of item `item`; lane e looks at the item's adapter
-// e.  Adapters failing validation are left out (and reported when `report`);
-// the shrink and the expand leave out the same ones.  The host sends only
-// calls whose stacks fit in kKMax ranks; an entry that would not fit is left
-// out and reported as a bad segment.
-__device__ void warp_build_stack(const TcArgs &p, int item, StackSm &st, bool report)
+// e (for projections sharing an input: the segment's adapter in pool e).
+// Adapters failing validation are left out (and reported when `report`); the
+// shrink and the expand leave out the same ones.  The host sends only calls
+// whose stacks fit in kmax ranks; an entry that would not fit is left out and
+// reported as a bad segment.
+__device__ void warp_build_stack(const TcArgs &p, int item, StackSm &st, bool report, int kmax = kKMax)
 {
     const int lane = threadIdx.x & 31;
     __syncwarp();                           // this warp's readers of the previous stack are done
@@ -330,14 +333,17 @@ __device__ void warp_build_stack(const TcArgs &p, int item, StackSm &st, bool re
     if (p.mode == kModeMulti) {
         lo = p.ad_off[item];
         n = min(p.ad_off[item + 1] - lo, p.max_ads);
+    } else if (p.mode == kModeProj) {
+        n = p.n_proj;
     }
+    const int pl = p.mode == kModeProj && lane < n ? lane : 0;   // this lane's pool
     int32_t r = 0;
     int64_t ao = 0, bo = 0;
     float sc = 0.f;
     bool ok = false;
     if (lane < n) {
         const int32_t a = p.mode == kModeMulti ? p.ad_id[lo + lane] : p.seg_ad[item];
-        ok = adapter_ok(p.pool, a, &r, &ao, &bo);
+        ok = adapter_ok(p.mode == kModeProj ? p.proj[pl] : p.pool, a, &r, &ao, &bo);
         if (!ok && report)
             atomicOr(p.err, (uint32_t)LORA_ERR_BAD_ADAPTER);
         sc = p.mode == kModeMulti ? p.ad_scale[lo + lane] : p.scale;
@@ -351,19 +357,20 @@ __device__ void warp_build_stack(const TcArgs &p, int item, StackSm &st, bool re
         if (lane >= d)
             incl += t;
     }
-    const bool fits = ok && incl <= kKMax;
+    const bool fits = ok && incl <= kmax;
     if (ok && !fits && report)
         atomicOr(p.err, (uint32_t)LORA_ERR_BAD_SEGMENT);
     const unsigned m = __ballot_sync(0xffffffffu, fits);
     const int ktot = (int)__reduce_max_sync(0xffffffffu, fits ? (unsigned)incl : 0u);
-    const bool a_tma = __all_sync(0xffffffffu, !fits || (ao % p.pool.d_in) == 0);
+    const bool a_tma = __all_sync(0xffffffffu, !fits || ((ao % p.pool.d_in) == 0 && ((p.a_tma >> pl) & 1)));
     const int bm = b_map(r);
     const bool b_tma = __all_sync(0xffffffffu, !fits || (bm >= 0 && ((p.b_tma >> bm) & 1) && (bo % r) == 0));
     if (fits) {
         const int i = __popc(m & ((1u << lane) - 1u));
         st.r[i] = r;
         st.kb[i] = incl - r;
-        st.slot[i] = lane;
+        st.vc0[i] = p.mode == kModeProj ? p.proj_vcol[pl] : lane * p.slot_stride;
+        st.pool[i] = (signed char)pl;
         st.s[i] = sc;
         st.aoff[i] = ao;
         st.boff[i] = bo;
@@ -396,11 +403,13 @@ __device__ unsigned long long g_tc_trace[3 * 1024 * 8];
 //
 // Unit = one tile of <= 128 rows of one item.  D[128 x kpad] = X_tile A_stack^T
 // over d_in in 64-column k-blocks; the epilogue writes V rows (fp32).  The A
-// rows of a k-block come by TMA in 8-row boxes over the A pool seen as a
-// [A_elems / d_in, d_in] matrix (every adapter packed at a multiple of d_in),
-// else by cp.async, 16 bytes at a time.  A stage holds the x atom and as many A
-// rows as the call's largest stacked rank (rounded to 16): at rank 64, 24 KB, and
-// four stages fit twice per SM, so two tiles can stream through one SM at once.
+// rows of a k-block come by TMA in 64-, 32- and 8-row boxes over the A pool
+// seen as a [A_elems / d_in, d_in] matrix (every adapter packed at a multiple
+// of d_in), else by cp.async, 16 bytes at a time.  A stage holds the x atom and
+// as many A rows as the call's largest stacked rank (rounded to 16): at rank
+// 64, 24 KB, and four stages fit twice per SM, so two tiles can stream through
+// one SM at once.  Projections that share X stack their A rows (from their own
+// pools) up to 256 ranks: then one CTA per SM, 48 KB stages, and MMA N = 256.
 
 __global__ void __launch_bounds__(kTcThreads, 2) k_tc_shrink(const __grid_constant__ TcArgs p)
 {
@@ -410,9 +419,9 @@ __global__ void __launch_bounds__(kTcThreads, 2) k_tc_shrink(const __grid_consta
     __shared__ __align__(8) uint64_t full_bar[kMaxShrinkStages], empty_bar[kMaxShrinkStages];
     __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2];
     __shared__ __align__(8) StackSm stk[kTcThreads / 32];
-    __shared__ long long arow[kKMax];        // producer, cp.async path: element offset of stacked row j's A row
-    __shared__ int4 abox[kKMax / 8];         // producer, TMA path: (stacked row, pool row, map) of each A box
-    __shared__ int vcol[4][kKMax / 4];       // epilogue warp q: V column of stacked columns 4g..4g+3 (-1: none)
+    __shared__ const __nv_bfloat16 *arow[kKMaxShrink];   // producer, cp.async path: stacked row j's A row
+    __shared__ int4 abox[kKMaxShrink / 8];   // producer, TMA path: (stacked row, pool row, map) of each A box
+    __shared__ int vcol[4][kKMaxShrink / 4]; // epilogue warp q: V column of stacked columns 4g..4g+3 (-1: none)
     __shared__ uint32_t tmem_base;
     __shared__ int abort_flag;
 
@@ -421,6 +430,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) k_tc_shrink(const __grid_consta
     const int d_in = p.pool.d_in;
     const int n_kb = (d_in + kBK - 1) / kBK;
     const int n_st = p.s_stages;
+    const int acc = p.s_acc;                     // TMEM columns per accumulator (two of them)
 
     if (tid == 0) {
         for (int s = 0; s < kMaxShrinkStages; ++s) {
@@ -435,7 +445,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) k_tc_shrink(const __grid_consta
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 1)
-        tmem_alloc(&tmem_base, 256);
+        tmem_alloc(&tmem_base, 2 * acc);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -451,9 +461,9 @@ __global__ void __launch_bounds__(kTcThreads, 2) k_tc_shrink(const __grid_consta
         int it = 0;
         for (int u = u0; u < u1; ++u) {
             const Group gr = p.groups[u];
-            warp_build_stack(p, gr.item, st, false);
-            const bool use_tma = st.a_tma && p.a_tma;
-            // A boxes: each entry's rows cut into 64-, 32- and 8-row boxes (at most 16 boxes)
+            warp_build_stack(p, gr.item, st, false, kKMaxShrink);
+            const bool use_tma = st.a_tma;
+            // A boxes: each entry's rows cut into 64-, 32- and 8-row boxes (at most 32 boxes)
             int nbox = 0;
             int box_j = 0, box_row = 0, box_m = 0;   // this lane's box: stacked row, pool row, map
             if (use_tma) {
@@ -462,7 +472,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) k_tc_shrink(const __grid_consta
                         const int row0 = (int)(st.aoff[e] / d_in);
                         for (int j = 0; j < st.r[e];) {
                             const int m = st.r[e] - j >= 64 ? 0 : (st.r[e] - j >= 32 ? 1 : 2);
-                            abox[nbox] = make_int4(st.kb[e] + j, row0 + j, m, 0);
+                            abox[nbox] = make_int4(st.kb[e] + j, row0 + j, 3 * st.pool[e] + m, 0);
                             ++nbox;
                             j += abox_rows(m);
                         }
@@ -477,11 +487,12 @@ __global__ void __launch_bounds__(kTcThreads, 2) k_tc_shrink(const __grid_consta
                     box_m = bx.z;
                 }
             } else {
-                for (int j = lane; j < kKMax; j += 32) {
-                    long long o = -1;
+                for (int j = lane; j < kKMaxShrink; j += 32) {
+                    const __nv_bfloat16 *o = p.pool.A;
                     if (j < st.ktot) {
                         const int e = stack_entry(st, j);
-                        o = st.aoff[e] + (long long)(j - st.kb[e]) * d_in;
+                        const __nv_bfloat16 *A = p.mode == kModeProj ? p.proj[st.pool[e]].A : p.pool.A;
+                        o = A + st.aoff[e] + (long long)(j - st.kb[e]) * d_in;
                     }
                     arow[j] = o;
                 }
@@ -513,7 +524,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) k_tc_shrink(const __grid_consta
                     const bool in = col < d_in;
                     const uint32_t abase = smem_u32(as);
                     for (int j = lane >> 3; j < st.ktot; j += 4)
-                        cp_async16(abase + sw128_off(j, c), in ? p.pool.A + arow[j] + col : p.pool.A, in);
+                        cp_async16(abase + sw128_off(j, c), in ? arow[j] + col : p.pool.A, in);
                 }
                 cp_async_arrive(&full_bar[s]);
                 TC_STAMP(0, it, 2);
@@ -525,9 +536,9 @@ __global__ void __launch_bounds__(kTcThreads, 2) k_tc_shrink(const __grid_consta
         int it = 0, t = 0;
         for (int u = u0; u < u1; ++u, ++t) {
             const Group gr = p.groups[u];
-            warp_build_stack(p, gr.item, st, false);
+            warp_build_stack(p, gr.item, st, false, kKMaxShrink);
             const int kpad = st.kpad;
-            const bool a_tma = st.a_tma && p.a_tma;
+            const bool a_tma = st.a_tma;
             const int b = t & 1;
             if (!warp_wait(&acc_empty[b], ((t >> 1) & 1) ^ 1, &abort_flag, p.err))
                 goto done;
@@ -548,7 +559,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) k_tc_shrink(const __grid_consta
                     const uint32_t aa = xa + kAtom;
 #pragma unroll
                     for (int k = 0; k < kBK / 16; ++k)
-                        tc_mma(tmem + b * 128, sw128_desc(xa + k * 32), sw128_desc(aa + k * 32), idesc,
+                        tc_mma(tmem + b * acc, sw128_desc(xa + k * 32), sw128_desc(aa + k * 32), idesc,
                                (kb > 0 || k > 0) ? 1u : 0u);
                     TC_STAMP(1, it, 2);
                 }
@@ -571,15 +582,15 @@ __global__ void __launch_bounds__(kTcThreads, 2) k_tc_shrink(const __grid_consta
         int t = 0;
         for (int u = u0; u < u1; ++u, ++t) {
             const Group gr = p.groups[u];
-            warp_build_stack(p, gr.item, st, warp == 2);
-            {
-                const int k = lane * 4;
+            warp_build_stack(p, gr.item, st, warp == 2, kKMaxShrink);
+            for (int g = lane; g < kKMaxShrink / 4; g += 32) {
+                const int k = g * 4;
                 int c = -1;
                 if (k < st.ktot) {
                     const int e = stack_entry(st, k);
-                    c = st.slot[e] * p.slot_stride + (k - st.kb[e]);
+                    c = st.vc0[e] + (k - st.kb[e]);
                 }
-                vc[lane] = c;
+                vc[g] = c;
             }
             __syncwarp();
             const int b = t & 1;
@@ -590,7 +601,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) k_tc_shrink(const __grid_consta
             float *vrow = p.V + (int64_t)(gr.p0 + (valid ? row : 0)) * p.ldv;
             for (int c0 = 0; c0 < st.kpad; c0 += 32) {
                 float v[32];
-                tmem_ld32(tmem + b * 128 + ((uint32_t)(q * 32) << 16) + c0, v);
+                tmem_ld32(tmem + b * acc + ((uint32_t)(q * 32) << 16) + c0, v);
                 if (valid) {
 #pragma unroll
                     for (int g = 0; g < 8; ++g) {
@@ -611,7 +622,7 @@ done:
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, 256);
+        tmem_dealloc(tmem, 2 * acc);
     }
 }
 
@@ -889,7 +900,7 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_tc_expand(const __grid_co
                     float sc = 0.f;
                     if (k < st.ktot) {
                         const int e = stack_entry(st, k);
-                        c = st.slot[e] * p.slot_stride + (k - st.kb[e]);
+                        c = st.vc0[e] + (k - st.kb[e]);
                         // several adapters: each one's scale goes into its V columns; one
                         // adapter: V is staged as it is and D is scaled in fp32 (for the merge,
                         // whose V is exactly bf16, this keeps a single rounding of W)
@@ -1097,10 +1108,12 @@ cudaError_t launch_tc(void (*kernel)(TcArgs), bool *attr_set, const TcArgs &a, i
 
 }  // namespace
 
-bool tc_encode_a(TcArgs &a, const void *A, int64_t A_elems, int32_t d_in)
+bool tc_encode_a(TcArgs &a, const void *A, int64_t A_elems, int32_t d_in, int pool_index)
 {
     // the A pool as a [A_elems / d_in, d_in] matrix, boxes of 64 columns x 64, 32 and 8 rows
-    a.a_tma = 0;
+    if (pool_index < 0 || pool_index >= kMaxProj)
+        return false;
+    a.a_tma &= ~(1 << pool_index);
     const int64_t rows = A_elems / d_in;
     if (rows < 1 || rows > 0x7fffffffLL)
         return false;
@@ -1112,12 +1125,12 @@ bool tc_encode_a(TcArgs &a, const void *A, int64_t A_elems, int32_t d_in)
     const cuuint32_t estr[2] = {1, 1};
     for (int i = 0; i < 3; ++i) {
         const cuuint32_t box[2] = {64, (cuuint32_t)abox_rows(i)};
-        if (fn(&a.map_a[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(A), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        if (fn(&a.map_a[3 * pool_index + i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(A), dims,
+               strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return false;
     }
-    a.a_tma = 1;
+    a.a_tma |= 1 << pool_index;
     return true;
 }
 
@@ -1160,25 +1173,32 @@ bool tc_encode_y(TcArgs &a, const void *Y, int32_t N, int32_t d_out, int64_t ldy
 
 cudaError_t launch_tc_shrink(const TcArgs &args, int max_tiles, int kk, cudaStream_t s)
 {
-    // a stage: the x atom and round16(kk) A rows of 128 bytes; two CTAs per SM
+    // a stage: the x atom and round16(kk) A rows of 128 bytes.  Up to 128
+    // stacked ranks: two CTAs per SM, each with two 128-column accumulators;
+    // above (projections sharing X): one CTA per SM (its four stages take
+    // more than half the SM's shared memory) with two 256-column accumulators
     static bool attr_set[64] = {};
+    if (kk < 1 || kk > kKMaxShrink)
+        return cudaErrorInvalidValue;
     TcArgs a = args;
     const int a_rows = (kk + 15) & ~15;
+    const bool wide = kk > kKMax;
     a.s_stage = kAtom + a_rows * 128;
-    a.s_stages = kk > 64 ? 3 : 4;
+    a.s_stages = wide ? 4 : (kk > 64 ? 3 : 4);
+    a.s_acc = wide ? 256 : 128;
     const int smem = a.s_stages * a.s_stage + 1024;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess)
         return e;
     if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-        // the largest layout: 4 stages at rank 64 or 3 at rank 128 (same size)
+        // the largest layout: 4 stages of 256 stacked ranks
         if ((e = cudaFuncSetAttribute(k_tc_shrink, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      4 * (kAtom + 64 * 128) + 1024)) != cudaSuccess)
+                                      4 * (kAtom + kKMaxShrink * 128) + 1024)) != cudaSuccess)
             return e;
         attr_set[dev] = true;
     }
-    int grid = 2 * sm_count();
+    int grid = (wide ? 1 : 2) * sm_count();
     if (max_tiles > 0 && max_tiles < grid)
         grid = max_tiles;
     bool done = true;

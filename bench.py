@@ -52,6 +52,9 @@ WORKLOAD_DESC = {
                        "200 adapters, 1-3 co-occurring adapters per image, scales U[0.5,1]",
     "merge_mlp_up": "merge: fold one rank-64 adapter of a 64-adapter pool into the Llama-3-8B MLP up-proj "
                     "weight W [14336, 4096] in place (W += s B A)",
+    "prefill_qkv": "prefill SGMV over shared-input projections: 32 prompts, lengths U[128,1024], Llama-3-8B "
+                   "q/k/v 4096->4096/1024/1024, rank 64, 64 adapters, Zipf(1.1) per request; one shrink "
+                   "reads X once for all three, then one expand per projection",
 }
 
 
@@ -228,11 +231,46 @@ def launches_per_call(call) -> int:
                                   len(call.req_off_h) - 1)
 
 
+def shrink_proj_passes(max_ranks, limit=256) -> int:
+    """Tensor-core launches of lora_sgmv_shrink_proj: runs of consecutive projections
+    whose max ranks sum to at most 256 (the header's rule)."""
+    n, k = 0, limit + 1
+    for r in max_ranks:
+        if k + r > limit:
+            n, k = n + 1, 0
+        k += r
+    return n
+
+
+def launches_per_step(wl) -> int:
+    import adapter_gemv_sgmv_b200 as L
+    if wl.desc.get("op") == "sgmv_proj":
+        c0 = wl.calls[0]
+        n = len(c0.seg_ad_h)
+        expands = sum(L.lora_kernel_launches(L.OP_SGMV_EXPAND, c.n_tokens, c.pool.n_adapters, c.pool.d_in, n)
+                      for c in wl.calls)
+        return 1 + shrink_proj_passes([c.pool.max_rank for c in wl.calls]) + expands
+    return sum(launches_per_call(c) for c in wl.calls)
+
+
 def make_step(wl, ws_map, stream):
     """Closure running one full pass of the path over workload `wl` on `stream`."""
     import torch
     import adapter_gemv_sgmv_b200 as L
     fns = []
+    if wl.desc.get("op") == "sgmv_proj":
+        # projections sharing X: one shrink over all of them, then each projection's expand
+        c0 = wl.calls[0]
+        pools = [c.pool for c in wl.calls]
+        V = torch.empty(c0.X.shape[0], sum(p.max_rank for p in pools), dtype=torch.float32, device=c0.X.device)
+        cols = np.cumsum([0] + [p.max_rank for p in pools])[:-1].tolist()
+
+        def proj_step():
+            L.lora_sgmv_shrink_proj(c0.X, V, pools, c0.seg_off, c0.seg_ad, ws=ws_map[id(c0)], stream=stream)
+            for c, col in zip(wl.calls, cols):
+                L.lora_sgmv_expand(V[:, col:], c.Y, c.pool, c.seg_off, c.seg_ad, c.scale, ws=ws_map[id(c)],
+                                   stream=stream)
+        return proj_step
     for c in wl.calls:
         ws = ws_map[id(c)]
         if hasattr(c, "W"):
@@ -306,10 +344,15 @@ def run_ours(args):
     tokens_per_step = sets[0].n_tokens
     set_bytes = 0
     for wl in sets:
+        seen_x = set()
         for c in wl.calls:
-            io = c.W.numel() * 2 if hasattr(c, "W") else c.X.numel() * 2 + c.Y.numel() * 2
+            if hasattr(c, "W"):
+                io = c.W.numel() * 2
+            else:
+                io = c.Y.numel() * 2 + (0 if c.X.data_ptr() in seen_x else c.X.numel() * 2)
+                seen_x.add(c.X.data_ptr())
             set_bytes += c.pool.A.numel() * 2 + c.pool.B.numel() * 2 + io
-    launches_step = sum(launches_per_call(c) for c in sets[0].calls)
+    launches_step = launches_per_step(sets[0])
 
     # eager warm-up (also sets per-device function attributes before capture)
     with torch.cuda.stream(stream):

@@ -70,6 +70,7 @@ extern "C" {
 #define LORA_MAX_RANK 128
 #define LORA_MAX_ADAPTERS 32768
 #define LORA_MAX_ADS_PER_REQ 8
+#define LORA_MAX_PROJ 4          /* projections sharing one input in lora_sgmv_shrink_proj */
 
 /* Status codes.  Host-side codes are returned directly; device-side codes are
  * bits of the workspace error word returned by lora_get_error (OR-ed). */
@@ -177,6 +178,33 @@ LORA_API lora_status lora_bgmv(const void *X, int64_t ldx, void *Y, int64_t ldy,
 LORA_API lora_status lora_sgmv_shrink(const void *X, int64_t ldx, float *V, int64_t ldv,
                              const lora_pool *pool, const int32_t *seg_off, const int32_t *seg_ad,
                              int32_t n_seg, int32_t N, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * lora_sgmv_shrink_proj -- the shrinks of several projections that read the
+ * same input (attention's Q, K and V; an MLP's gate and up), done as one
+ * shrink over their A rows stacked along the rank axis, so X is read once
+ * ("Serving several LoRAs, ControlNet and IP-Adapter", self-test answer 1:
+ * a LoRA attaches to the Q, K, V and O projections, sometimes the MLP):
+ *   V[n][c_p + j] = sum_i A_p[a][j][i] X[n][i],  j < rank_p[a],  a = seg_ad[k],
+ * for seg_off[k] <= n < seg_off[k+1] and every projection p < n_proj, where
+ * A_p is pools[p]'s A and c_p = pools[0].max_rank + ... + pools[p-1].max_rank.
+ * Projection p's expand is then lora_sgmv_expand(V + c_p, ldv, Y_p, ...,
+ * &pools[p], ...).
+ * pools: host array of n_proj (1 .. LORA_MAX_PROJ) pools with one d_in and
+ * one n_adapters (adapter a of every pool belongs to the same fine-tune);
+ * their d_out, ranks and storage may differ.  V: device fp32 [N, ldv],
+ * ldv >= sum of the pools' max_rank; entries past an adapter's rank and rows
+ * outside every segment are not written.  Segment arguments and workspace
+ * (LORA_OP_SGMV_SHRINK, sized with any of the pools' max_rank) as for
+ * lora_sgmv_shrink.  Long segments take one plan launch plus one tensor-core
+ * launch per group of consecutive projections whose max_ranks sum to at most
+ * 256; short ones take the plan plus one CUDA-core shrink per projection.
+ * A bad adapter id is reported once per projection pool it fails in.
+ */
+LORA_API lora_status lora_sgmv_shrink_proj(const void *X, int64_t ldx, float *V, int64_t ldv,
+                             const lora_pool *pools, int32_t n_proj, const int32_t *seg_off,
+                             const int32_t *seg_ad, int32_t n_seg, int32_t N,
+                             void *ws, size_t ws_bytes, void *stream);
 
 /*
  * lora_sgmv_expand -- the second half of the segmented product:

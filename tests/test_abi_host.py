@@ -37,7 +37,7 @@ def test_header_declares_the_entry_points():
     names = set(declared())
     assert {"lora_bgmv", "lora_sgmv_shrink", "lora_sgmv_expand", "lora_apply_multi", "lora_route",
             "lora_workspace_size", "lora_workspace_init", "lora_get_error", "lora_version",
-            "lora_merge"} <= names
+            "lora_merge", "lora_sgmv_shrink_proj"} <= names
 
 
 def test_every_declared_symbol_is_exported(lib):
@@ -141,3 +141,33 @@ def test_other_entry_points_validate(lib):
     # workspace helpers reject a null / misaligned workspace before touching CUDA
     assert lib.lora_workspace_init(None, None) == WORKSPACE
     assert lib.lora_get_error(FAKE + 8, None) == WORKSPACE
+
+
+def _pools(*ps):
+    return (L.LoraPoolStruct * len(ps))(*ps)
+
+
+def test_shrink_proj_validates(lib):
+    q, k, v = _pool(), _pool(d_out=16, max_rank=8), _pool(max_rank=32)
+    three = _pools(q, k, v)
+    sh = lib.lora_sgmv_shrink_proj
+    # no pools / too many projections
+    assert sh(FAKE, 64, FAKE, 56, None, 3, FAKE, FAKE, 2, 4, None, 0, None) == INVALID
+    assert sh(FAKE, 64, FAKE, 56, three, 0, FAKE, FAKE, 2, 4, None, 0, None) == INVALID
+    five = _pools(q, q, q, q, q)
+    assert sh(FAKE, 64, FAKE, 80, five, 5, FAKE, FAKE, 2, 4, None, 0, None) == UNSUPPORTED
+    # a bad pool anywhere in the list
+    assert sh(FAKE, 64, FAKE, 56, _pools(q, _pool(A=0), v), 3, FAKE, FAKE, 2, 4, None, 0, None) == INVALID
+    assert sh(FAKE, 64, FAKE, 56, _pools(q, k, _pool(max_rank=12)), 3, FAKE, FAKE, 2, 4, None, 0,
+              None) == UNSUPPORTED
+    # the pools must share d_in and n_adapters
+    assert sh(FAKE, 64, FAKE, 56, _pools(q, _pool(d_in=128), v), 3, FAKE, FAKE, 2, 4, None, 0, None) == INVALID
+    assert sh(FAKE, 64, FAKE, 56, _pools(q, _pool(n_adapters=5), v), 3, FAKE, FAKE, 2, 4, None, 0,
+              None) == INVALID
+    # V holds the ranks side by side: ldv >= 16 + 8 + 32
+    assert sh(FAKE, 64, FAKE, 48, three, 3, FAKE, FAKE, 2, 4, None, 0, None) == INVALID
+    assert sh(FAKE, 64, FAKE, 56, three, 3, None, FAKE, 2, 4, None, 0, None) == INVALID
+    assert sh(FAKE, 32, FAKE, 56, three, 3, FAKE, FAKE, 2, 4, None, 0, None) == INVALID
+    assert sh(FAKE, 64, FAKE, 56, three, 3, FAKE, FAKE, 2, 4, None, 0, None) == WORKSPACE
+    # two projections only: ldv 24 is enough
+    assert sh(FAKE, 64, FAKE, 24, three, 2, FAKE, FAKE, 2, 4, None, 0, None) == WORKSPACE

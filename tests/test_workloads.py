@@ -64,3 +64,18 @@ def test_merge_workload_shapes():
     cost = accounting.workload_cost(wl)
     assert cost.bytes == 2 * 2 * 32 * 64 + 2 * 16 * (64 + 32) and cost.flops == 2 * 32 * 64 * 16
 
+
+
+def test_qkv_workload_shares_x_and_counts_it_once():
+    wl = make_workload("prefill_qkv", n_req=3, len_range=(4, 9), d_in=64, d_outs=(64, 16, 16), rank=8,
+                       n_adapters=5)
+    q, k, v = wl.calls
+    assert q.X.data_ptr() == k.X.data_ptr() == v.X.data_ptr()
+    assert [c.pool.d_out for c in wl.calls] == [64, 16, 16]
+    assert np.array_equal(q.seg_off_h, v.seg_off_h) and np.array_equal(q.seg_ad_h, k.seg_ad_h)
+    assert q.seg_off_h[-1] == wl.n_tokens == q.X.shape[0]
+    from adapter_gemv_sgmv_b200 import accounting
+    N = wl.n_tokens
+    separate = sum(accounting.call_cost(c).bytes for c in wl.calls)
+    assert accounting.workload_cost(wl).bytes == separate - 2 * 2 * N * 64
+    assert accounting.workload_cost(wl).tokens == N

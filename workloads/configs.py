@@ -325,6 +325,7 @@ WORKLOAD_NAMES = [
     "mixed_rank_layer",   # 512 decode tokens, 1000 adapters r in {8..128}, 7 Llama-3-8B projections
     "diffusion_multi",    # 16 images x 4096 tokens, 1280->1280 x QKVO, r32, 200 adapters, 1-3 per image
     "merge_mlp_up",       # fold one rank-64 adapter into W [14336, 4096] (Llama-3-8B MLP up-proj) in place
+    "prefill_qkv",        # the prefill segments over Llama-3-8B q/k/v (4096 -> 4096/1024/1024), r64, X shared
 ]
 
 LLAMA3_8B_PROJ = [  # name, d_in, d_out, which input it reads
@@ -336,7 +337,7 @@ LLAMA3_8B_PROJ = [  # name, d_in, d_out, which input it reads
 
 def make_workload(which, device="cpu", seed: Optional[int] = None, y0: str = "zeros",
                   **overrides) -> Workload:
-    """Build one of the five named workloads (index or name).  seed defaults to the index.
+    """Build one of the named workloads (index or name).  seed defaults to the index.
 
     overrides shrink a workload for quick tests (e.g. n_req=4, d_out=512)."""
     idx = which if isinstance(which, int) else WORKLOAD_NAMES.index(which)
@@ -436,4 +437,27 @@ def make_workload(which, device="cpu", seed: Optional[int] = None, y0: str = "ze
         a = int(rng.integers(0, n_ad))
         call = MergeCall("up", W, pool, a, overrides.get("scale", 1.0))
         return Workload("merge_mlp_up", [call], {"tokens": d_out, "op": "merge"})
+    if idx == 6:
+        # the prefill recipe (prompt lengths, Zipf adapters, per-adapter segments) over the
+        # three attention projections that read the same input; an adapter fine-tunes all three
+        n_req = overrides.get("n_req", 32)
+        lo, hi = overrides.get("len_range", (128, 1024))
+        d_in = overrides.get("d_in", 4096)
+        d_outs = overrides.get("d_outs", (4096, 1024, 1024))
+        r = overrides.get("rank", 64)
+        n_ad = overrides.get("n_adapters", 64)
+        lens = rng.integers(lo, hi + 1, size=n_req).astype(np.int64)
+        req_ids = zipf_ids(rng, n_ad, overrides.get("zipf_s", 1.1), n_req)
+        order = np.argsort(req_ids, kind="stable")
+        tok_ids = np.repeat(req_ids[order], lens[order]).astype(np.int32)
+        seg_off, seg_ad = segments_from_sorted_ids(tok_ids, n_ad, keep_empty=False)
+        N = int(lens.sum())
+        X = _x(N, d_in, gen, device)
+        calls = []
+        for p_i, (pname, d_out) in enumerate(zip(("q", "k", "v"), d_outs)):
+            pool = make_pool([r] * n_ad, d_in, d_out, seed * 100 + p_i, device)
+            calls.append(sgmv_call(pname, X, pool, seg_off, seg_ad, overrides.get("scale", 1.0), device, y0,
+                                   seed * 100 + p_i))
+        return Workload("prefill_qkv", calls, {"tokens": N, "op": "sgmv_proj", "x_read_once": True,
+                                               "requests": n_req})
     raise ValueError(f"unknown workload {which!r}")
