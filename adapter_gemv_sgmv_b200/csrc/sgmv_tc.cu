@@ -50,7 +50,7 @@ constexpr int kBM = 128;            // rows per tile
 constexpr int kBN = 128;            // expand: outputs per unit
 constexpr int kBK = 64;             // shrink: d_in per k-block (one 128-byte swizzle atom)
 constexpr int kAtom = kBM * 128;    // bytes of a 128-row x 64-column bf16 swizzle atom
-constexpr int kMaxShrinkStages = 4;
+constexpr int kMaxShrinkStages = 6;
 constexpr int kExpandBStages = 2;
 constexpr unsigned long long kWaitNs = 2000000000ull;   // 2 s bound on any single wait
 
@@ -409,7 +409,8 @@ __device__ unsigned long long g_tc_trace[3 * 1024 * 8];
 // as many A rows as the call's largest stacked rank (rounded to 16): at rank
 // 64, 24 KB, and four stages fit twice per SM, so two tiles can stream through
 // one SM at once.  Projections that share X stack their A rows (from their own
-// pools) up to 256 ranks: then one CTA per SM, 48 KB stages, and MMA N = 256.
+// pools) up to 256 ranks: then one CTA per SM, as many 40-48 KB stages as fit,
+// and MMA N up to 256.
 
 __global__ void __launch_bounds__(kTcThreads, 2) k_tc_shrink(const __grid_constant__ TcArgs p)
 {
@@ -630,17 +631,19 @@ done:
 // ============================================================ expand kernel
 //
 // Unit = (tile, 128-output slice).  D[128 x 128] = V_tile B_stack[slice]^T over
-// the stacked rank (V staged once per tile as bf16, with each adapter's scale
-// folded in when a request stacks several; a single adapter's scale multiplies
-// the fp32 accumulator instead);
+// the stacked rank (V staged once per tile as a pair of bf16 matrices, high and
+// low parts, so the product sees V to about 2^-17 relative for one extra MMA per
+// 16 ranks; each adapter's scale folded in when a request stacks several, a
+// single adapter's scale multiplying the fp32 accumulator instead);
 // the epilogue adds D to the y tile (TMA-loaded; threads only read it, so a
 // stage goes back to the producer as soon as it is read) and each epilogue
 // warp stores its rows through a small staging area with coalesced 16-byte
 // stores.
 //
-// Shared memory is laid out at run time: V and every B stage take one 16 KB
-// atom per 64 stacked ranks the call can carry (1 or 2), and the y stages fill
-// the rest (up to kMaxYStages), so a rank-64 call keeps five 32 KB y tiles in flight.
+// Shared memory is laid out at run time: each half of V and every B stage take
+// one 16 KB atom per 64 stacked ranks the call can carry (1 or 2), and the y
+// stages fill the rest (up to kMaxYStages): four 32 KB y tiles in flight at rank
+// 64, two at 128.
 constexpr int kY = kBM * kBN * 2;                  // y: 128 rows x 128 outputs (two 64-column atoms)
 constexpr int kMaxYStages = 6;
 constexpr int kStaging = kEpiWarps * 1024;         // per epilogue warp: 32 rows x 16 outputs of bf16
@@ -666,9 +669,9 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_tc_expand(const __grid_co
     const int n_ns = (d_out + kBN - 1) / kBN;           // output slices
     const int G = gridDim.x;
     const int n_ys = p.e_ystages;
-    const int szB = p.e_natoms * kAtom;                 // one B stage (and V)
-    unsigned char *const smV = sm;
-    unsigned char *const smB = sm + szB;
+    const int szB = p.e_natoms * kAtom;                 // one B stage (and each half of V)
+    unsigned char *const smV = sm;                      // V high parts, then V low parts
+    unsigned char *const smB = sm + 2 * szB;
     unsigned char *const smS = smB + kExpandBStages * szB;   // epilogue warps' output staging
     unsigned char *const smY = smS + kStaging;
 
@@ -813,6 +816,7 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_tc_expand(const __grid_co
         bool b_tma = false;
         uint64_t ad[kKMax / 16], bd[kKMax / 16];
         const uint32_t va = smem_u32(smV);
+        const uint64_t lo_step = (uint64_t)((szB >> 4) & 0x3FFF);   // descriptor start field: V high -> V low
         for (int64_t u = u0; u < u1; ++u, ++it) {
             const int tile = (int)(u / n_ns);
             if (tile != prev_tile) {
@@ -859,8 +863,10 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_tc_expand(const __grid_co
                 const uint32_t idesc = idesc_bf16(kBM, kBN);
 #pragma unroll
                 for (int k16 = 0; k16 < kKMax / 16; ++k16)
-                    if (k16 < nsteps)
+                    if (k16 < nsteps) {
                         tc_mma(tmem + b * 128, ad[k16], bd[k16] + bbase, idesc, k16 > 0 ? 1u : 0u);
+                        tc_mma(tmem + b * 128, ad[k16] + lo_step, bd[k16] + bbase, idesc, 1u);
+                    }
                 TC_STAMP(1, it, 3);
                 tc_commit(&b_empty[sb]);
                 tc_commit(&acc_full[b]);
@@ -903,7 +909,8 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_tc_expand(const __grid_co
                         c = st.vc0[e] + (k - st.kb[e]);
                         // several adapters: each one's scale goes into its V columns; one
                         // adapter: V is staged as it is and D is scaled in fp32 (for the merge,
-                        // whose V is exactly bf16, this keeps a single rounding of W)
+                        // whose V is exactly bf16 -- low part zero -- this keeps a single
+                        // rounding of W)
                         sc = p.mode == kModeMulti ? st.s[e] : 1.f;
                     }
                     vsrc[e8][lane] = c;
@@ -913,8 +920,10 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_tc_expand(const __grid_co
                 // wait until the MMAs of the previous tile stopped reading V
                 if (vt > 0 && !warp_wait(&v_empty, (vt - 1) & 1, &abort_flag, p.err))
                     goto done;
-                // V[vr][stacked k] = bf16(s_e * V_e[vr][k - kb_e]) (s_e = 1 for one adapter), zero outside the tile's rows and
-                // the stack; thread et stages row et % 128, stacked ranks 32 (et / 128) .. + 31
+                // V[vr][stacked k] = s_e * V_e[vr][k - kb_e] (s_e = 1 for one adapter), zero outside the
+                // tile's rows and the stack, as two bf16 parts: hi = bf16(v) and lo = bf16(v - hi), so
+                // hi + lo carries v to about 2^-17 and the MMA sums both; thread et stages row
+                // et % 128, stacked ranks 32 (et / 128) .. + 31
                 const int vr = et & 127, vq = et >> 7;
                 const bool valid = vr < gr.cnt;
                 const float *vrow = p.V + (int64_t)(gr.p0 + (valid ? vr : 0)) * p.ldv;
@@ -922,21 +931,25 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_tc_expand(const __grid_co
                 const int c_end = min(st.kpad / 8, vq * 4 + 4);
                 for (int c = vq * 4; c < c_end; ++c) {
                     const int col = vsrc[e8][c];
-                    uint32_t w[4] = {0u, 0u, 0u, 0u};
+                    uint32_t w[4] = {0u, 0u, 0u, 0u}, wl[4] = {0u, 0u, 0u, 0u};
                     if (valid && col >= 0) {
                         const float sc = vsc[e8][c];
                         const float4 a = *reinterpret_cast<const float4 *>(vrow + col);
                         const float4 bq = *reinterpret_cast<const float4 *>(vrow + col + 4);
-                        const __nv_bfloat162 h0 = __floats2bfloat162_rn(sc * a.x, sc * a.y);
-                        const __nv_bfloat162 h1 = __floats2bfloat162_rn(sc * a.z, sc * a.w);
-                        const __nv_bfloat162 h2 = __floats2bfloat162_rn(sc * bq.x, sc * bq.y);
-                        const __nv_bfloat162 h3 = __floats2bfloat162_rn(sc * bq.z, sc * bq.w);
-                        w[0] = *reinterpret_cast<const uint32_t *>(&h0);
-                        w[1] = *reinterpret_cast<const uint32_t *>(&h1);
-                        w[2] = *reinterpret_cast<const uint32_t *>(&h2);
-                        w[3] = *reinterpret_cast<const uint32_t *>(&h3);
+                        const float v[8] = {sc * a.x, sc * a.y, sc * a.z, sc * a.w,
+                                            sc * bq.x, sc * bq.y, sc * bq.z, sc * bq.w};
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const __nv_bfloat162 hi = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
+                            const float2 hf = __bfloat1622float2(hi);
+                            const __nv_bfloat162 lo = __floats2bfloat162_rn(v[2 * j] - hf.x, v[2 * j + 1] - hf.y);
+                            w[j] = *reinterpret_cast<const uint32_t *>(&hi);
+                            wl[j] = *reinterpret_cast<const uint32_t *>(&lo);
+                        }
                     }
-                    st_shared_v4(vbase + (c >> 3) * kAtom + sw128_off(vr, c & 7), w[0], w[1], w[2], w[3]);
+                    const uint32_t dst = vbase + (c >> 3) * kAtom + sw128_off(vr, c & 7);
+                    st_shared_v4(dst, w[0], w[1], w[2], w[3]);
+                    st_shared_v4(dst + szB, wl[0], wl[1], wl[2], wl[3]);
                 }
                 fence_async_smem();
                 __syncwarp();
@@ -1180,21 +1193,30 @@ cudaError_t launch_tc_shrink(const TcArgs &args, int max_tiles, int kk, cudaStre
     static bool attr_set[64] = {};
     if (kk < 1 || kk > kKMaxShrink)
         return cudaErrorInvalidValue;
+    int dev = 0, optin = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    if ((e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess)
+        return e;
+    cudaFuncAttributes fa;
+    if ((e = cudaFuncGetAttributes(&fa, k_tc_shrink)) != cudaSuccess)
+        return e;
+    const int room = optin - (int)fa.sharedSizeBytes - 1024;
     TcArgs a = args;
     const int a_rows = (kk + 15) & ~15;
     const bool wide = kk > kKMax;
     a.s_stage = kAtom + a_rows * 128;
-    a.s_stages = wide ? 4 : (kk > 64 ? 3 : 4);
+    // wide: as many stages as one CTA's shared memory holds (5 at 192 ranks, 4 at 256)
+    a.s_stages = wide ? (room / a.s_stage < kMaxShrinkStages ? room / a.s_stage : kMaxShrinkStages)
+                      : (kk > 64 ? 3 : 4);
+    if (a.s_stages < 2)
+        return cudaErrorInvalidConfiguration;
     a.s_acc = wide ? 256 : 128;
     const int smem = a.s_stages * a.s_stage + 1024;
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess)
-        return e;
     if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-        // the largest layout: 4 stages of 256 stacked ranks
         if ((e = cudaFuncSetAttribute(k_tc_shrink, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      4 * (kAtom + kKMaxShrink * 128) + 1024)) != cudaSuccess)
+                                      optin - (int)fa.sharedSizeBytes)) != cudaSuccess)
             return e;
         attr_set[dev] = true;
     }
@@ -1207,8 +1229,8 @@ cudaError_t launch_tc_shrink(const TcArgs &args, int max_tiles, int kk, cudaStre
 
 cudaError_t launch_tc_expand(const TcArgs &args, int kk, cudaStream_t s)
 {
-    // shared memory: V and two B stages of one atom per 64 stacked ranks, then as
-    // many 32 KB y stages as fit (at least two)
+    // shared memory: V (high and low parts) and two B stages of one atom per 64
+    // stacked ranks, then as many 32 KB y stages as fit (at least two)
     static bool attr_set[64] = {};
     int dev = 0, optin = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -1221,7 +1243,7 @@ cudaError_t launch_tc_expand(const TcArgs &args, int kk, cudaStream_t s)
         return e;
     TcArgs a = args;
     a.e_natoms = kk > 64 ? 2 : 1;
-    const int fixed = (1 + kExpandBStages) * a.e_natoms * kAtom + kStaging + 1024;
+    const int fixed = (2 + kExpandBStages) * a.e_natoms * kAtom + kStaging + 1024;
     const int room = optin - (int)fa.sharedSizeBytes - fixed;
     a.e_ystages = room / kY < kMaxYStages ? room / kY : kMaxYStages;
     if (a.e_ystages < 2)

@@ -107,3 +107,48 @@ def test_tc_bad_adapter_in_a_segment_is_skipped_and_reported():
     good = np.array([0, 200, 200], np.int32)
     check_parity(got[:200], widen(Y0)[:200] + oracle.sgmv_delta(X, hp, good, np.array([1, 0], np.int32), 1.0)[:200],
                  "tc sgmv with a bad segment")
+
+
+@pytest.mark.parametrize("d_in", [192, 328])
+def test_tc_more_tiles_than_ctas_every_row(d_in):
+    """About 330 tiles of 128 rows, more than the CTAs of either shrink layout (two
+    per SM for one pool; one per SM for three projections stacked past 128 ranks):
+    every V entry and every output row of one projection against the oracle; the
+    output bound holds at |y| up to several rms, where the expand's V precision
+    shows (scale 1.5)."""
+    rng = np.random.default_rng(d_in)
+    ranks = [64, 16, 32, 64, 8, 40]
+    hps = [rand_host_pool(rng, ranks, d_in, d) for d in (136, 64, 200)]
+    lens = [7001, 5, 6900, 0, 8100, 12000, 7777]
+    ads = [2, 0, 4, 1, 3, 5, 2]
+    seg_off = np.concatenate([[3], 3 + np.cumsum(lens)]).astype(np.int32)
+    N = int(seg_off[-1]) + 9
+    X = rand_x(rng, N, d_in)
+    Xd = dev_bf16(X)
+    pools = [DevPool(hp) for hp in hps]
+    # one pool (two CTAs per SM, 296 CTAs)
+    V = torch.full((N, 64), float("nan"), dtype=torch.float32, device=DEV)
+    ws = L.lora_sgmv_shrink(Xd, V, pools[0], _i32(seg_off), _i32(ads))
+    assert L.lora_get_error(ws) == 0
+    Vref = oracle.sgmv_shrink(X, hps[0], seg_off, ads, ld=64)
+    Vh = to_host(V).astype(np.float64)
+    assert np.array_equal(np.isnan(Vh), np.isnan(Vref))
+    m = ~np.isnan(Vref)
+    check_close_f32(Vh[m], Vref[m], "many-tile shrink")
+    # three projections, 192 stacked ranks
+    W = torch.full((N, 192), float("nan"), dtype=torch.float32, device=DEV)
+    ws, cols = L.lora_sgmv_shrink_proj(Xd, W, pools, _i32(seg_off), _i32(ads))
+    assert L.lora_get_error(ws) == 0
+    Wh = to_host(W).astype(np.float64)
+    for p, c in enumerate(cols):
+        Vref = oracle.sgmv_shrink(X, hps[p], seg_off, ads, ld=64)
+        got = Wh[:, c:c + 64]
+        assert np.array_equal(np.isnan(got), np.isnan(Vref))
+        m = ~np.isnan(Vref)
+        check_close_f32(got[m], Vref[m], f"many-tile proj shrink p{p}")
+    # and the outputs of one projection from the fused V
+    Y0 = rand_x(rng, N, hps[2].d_out)
+    Y = dev_bf16(Y0)
+    ws = L.lora_sgmv_expand(torch.nan_to_num(W)[:, cols[2]:], Y, pools[2], _i32(seg_off), _i32(ads), 1.5)
+    assert L.lora_get_error(ws) == 0
+    check_parity(widen(to_host(Y)), widen(Y0) + oracle.sgmv_delta(X, hps[2], seg_off, ads, 1.5), "many-tile sgmv")
