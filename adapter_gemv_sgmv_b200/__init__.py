@@ -20,13 +20,14 @@ __all__ = [
     "lora_kernel_launches",
     "lora_get_error", "lora_route", "lora_bgmv", "lora_sgmv_shrink", "lora_sgmv_shrink_proj", "lora_sgmv_expand",
     "lora_apply_multi", "lora_apply_multi_static", "make_pool_struct", "Workspace", "OP_BGMV", "OP_SGMV_SHRINK", "OP_SGMV_EXPAND",
-    "OP_APPLY_MULTI", "OP_ROUTE", "OP_MERGE", "STATUS", "lora_merge", "PoolManager",
+    "OP_APPLY_MULTI", "OP_ROUTE", "OP_MERGE", "OP_LINEAR", "STATUS", "lora_merge", "lora_linear_sgmv",
+    "PoolManager",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 _LIBNAME = "liblora_sgmv.so"
 
-OP_BGMV, OP_SGMV_SHRINK, OP_SGMV_EXPAND, OP_APPLY_MULTI, OP_ROUTE, OP_MERGE = range(6)
+OP_BGMV, OP_SGMV_SHRINK, OP_SGMV_EXPAND, OP_APPLY_MULTI, OP_ROUTE, OP_MERGE, OP_LINEAR = range(7)
 STATUS = {0: "LORA_OK", 1: "LORA_ERR_INVALID_ARG", 2: "LORA_ERR_UNSUPPORTED", 4: "LORA_ERR_BAD_ADAPTER",
           8: "LORA_ERR_BAD_SEGMENT", 16: "LORA_ERR_CUDA", 32: "LORA_ERR_WORKSPACE", 64: "LORA_ERR_TIMEOUT"}
 MAX_ADS_PER_REQ = 8
@@ -85,6 +86,8 @@ def load():
         lib.lora_sgmv_shrink.restype = ctypes.c_int
         lib.lora_sgmv_shrink.argtypes = [P, i64, P, i64, PP, P, P, i32, i32, P, sz, P]
         lib.lora_sgmv_shrink_proj.restype = ctypes.c_int
+        lib.lora_linear_sgmv.restype = ctypes.c_int
+        lib.lora_linear_sgmv.argtypes = [P, i64, P, i64, P, i64, PP, P, P, i32, i32, f32, P, sz, P]
         lib.lora_sgmv_shrink_proj.argtypes = [P, i64, P, i64, PP, i32, P, P, i32, i32, P, sz, P]
         lib.lora_sgmv_expand.restype = ctypes.c_int
         lib.lora_sgmv_expand.argtypes = [P, i64, P, i64, PP, P, P, i32, i32, f32, P, sz, P]
@@ -295,6 +298,30 @@ def lora_sgmv_shrink_proj(X, V, pools, seg_off, seg_ad, ws: Workspace | None = N
                                   _ptr(seg_ad), n_seg, N, ws.ptr(), ws.nbytes, _stream_ptr(stream)),
         "lora_sgmv_shrink_proj")
     return ws, cols
+
+
+def lora_linear_sgmv(X, W, Y, pool, seg_off, seg_ad, scale: float, ws: Workspace | None = None, stream=None,
+                     max_rank: int | None = None):
+    """Y[n] = W X[n] + scale * B[a] A[a] X[n] for rows of segment k (a = seg_ad[k]; -1: W X[n] only).
+
+    W is the projection's bf16 weight [d_out, d_in]; Y is overwritten (rows outside every
+    segment are left as they are)."""
+    lib = load()
+    _check_dev(X, W, Y, seg_off, seg_ad)
+    ps = make_pool_struct(pool, max_rank)
+    ldx = _mat(X, ps.d_in, "X")
+    ldw = _mat(W, ps.d_in, "W")
+    ldy = _mat(Y, ps.d_out, "Y")
+    if W.shape[0] != ps.d_out:
+        raise LoraError(f"W must have d_out = {ps.d_out} rows", 1)
+    N = int(X.shape[0])
+    n_seg = int(seg_ad.numel())
+    need = lora_workspace_size(OP_LINEAR, N, ps.n_adapters, ps.d_in, ps.d_out, ps.max_rank, n_seg)
+    ws = ws or _workspace(need, X.device)
+    _rc(lib.lora_linear_sgmv(_ptr(X), ldx, _ptr(W), ldw, _ptr(Y), ldy, ctypes.byref(ps), _ptr(seg_off),
+                             _ptr(seg_ad), n_seg, N, float(scale), ws.ptr(), ws.nbytes, _stream_ptr(stream)),
+        "lora_linear_sgmv")
+    return ws
 
 
 def lora_sgmv_expand(V, Y, pool, seg_off, seg_ad, scale: float, ws: Workspace | None = None,

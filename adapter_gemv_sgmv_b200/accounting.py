@@ -118,9 +118,30 @@ def multi_cost(req_off: np.ndarray, ad_off: np.ndarray, ad_id: np.ndarray, ranks
     return _finish(n_tok, flops, distinct, ranks, d_in, d_out, meta)
 
 
+def linear_cost(seg_off: np.ndarray, seg_ad: np.ndarray, ranks: np.ndarray, d_in: int, d_out: int) -> Cost:
+    """The projection with its delta: the rows of every segment take x W^T (2 d_in d_out
+    FLOPs each) plus their adapter's delta; bytes: x read once, W read once, y written
+    once (not read), each touched adapter once, metadata."""
+    seg_off = np.asarray(seg_off, dtype=np.int64)
+    seg_ad = np.asarray(seg_ad)
+    ranks = np.asarray(ranks, dtype=np.int64)
+    lens = np.diff(seg_off)
+    n_tok = int(lens.sum())
+    flops = 2 * n_tok * int(d_in) * int(d_out)
+    flops += int(sum(lora_flops(int(l), ranks[a], d_in, d_out) for a, l in zip(seg_ad, lens) if a >= 0))
+    distinct = np.unique(seg_ad[(lens > 0) & (seg_ad >= 0)])
+    ad_bytes = int(sum(BF16_BYTES * adapter_elems(ranks[a], d_in, d_out) for a in distinct))
+    act = BF16_BYTES * n_tok * (int(d_in) + int(d_out))
+    w_bytes = BF16_BYTES * int(d_in) * int(d_out)
+    meta = 4 * (2 * len(seg_ad) + 1) + (8 + 8 + 4) * len(distinct)
+    return Cost(flops, act + w_bytes + ad_bytes + meta, n_tok, ad_bytes, act)
+
+
 def call_cost(call) -> Cost:
     """Cost of one workload call (duck-typed on the call's host metadata)."""
     p = call.pool
+    if hasattr(call, "W") and hasattr(call, "X"):
+        return linear_cost(call.seg_off_h, call.seg_ad_h, p.ranks_h, p.d_in, p.d_out)
     if hasattr(call, "W"):
         return merge_cost(p.d_in, p.d_out, int(p.ranks_h[call.adapter]))
     if hasattr(call, "ids_h"):

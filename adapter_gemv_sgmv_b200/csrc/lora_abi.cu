@@ -59,6 +59,7 @@ int32_t n_chunks_for(int op, int32_t d_in)
 struct Layout {
     size_t hdr, perm, seg_off, seg_ad, groups, V, total;
     int32_t max_groups, n_chunks;
+    int32_t kv;      // LORA_OP_LINEAR: column of the low parts of s V (max_rank rounded up to 64)
 };
 
 bool layout(int op, int32_t N, int32_t n_adapters, int32_t d_in, int32_t max_rank, int32_t n_items,
@@ -93,6 +94,10 @@ bool layout(int op, int32_t N, int32_t n_adapters, int32_t d_in, int32_t max_ran
         v = (size_t)L->n_chunks * N * max_rank * 4;
     else if (op == LORA_OP_APPLY_MULTI)
         v = (size_t)N * max_ads * max_rank * 4;
+    else if (op == LORA_OP_LINEAR) {
+        L->kv = (max_rank + 63) & ~63;
+        v = (size_t)N * 2 * L->kv * 2;      // s V, bf16 high and low parts
+    }
     off = align_up(off + v);
     L->total = off;
     return true;
@@ -178,7 +183,7 @@ size_t lora_workspace_size(int op, int32_t N, int32_t n_adapters, int32_t d_in, 
     if (op == LORA_OP_MERGE)
         return n_adapters >= 1 && n_adapters <= LORA_MAX_ADAPTERS && N == d_out
                    ? merge_workspace_size(d_in, d_out, max_rank) : 0;
-    if (op < LORA_OP_BGMV || op > LORA_OP_ROUTE)
+    if (op < LORA_OP_BGMV || op > LORA_OP_LINEAR || op == LORA_OP_MERGE)
         return 0;
     Layout L;
     if (!layout(op, N, n_adapters, d_in, max_rank, n_items, max_ads_per_req, &L))
@@ -202,6 +207,8 @@ int lora_kernel_launches(int op, int32_t N, int32_t n_adapters, int32_t d_in, in
         return 1;
     case LORA_OP_MERGE:   // preparation + expand (tensor cores), or + plan + expand
         return tc_enabled() && N >= kTcGroup ? 2 : 3;
+    case LORA_OP_LINEAR:  // plan + shrink + projection
+        return n_items > 0 ? 3 : 0;
     default:
         return 0;
     }
@@ -532,6 +539,83 @@ lora_status lora_sgmv_shrink_proj(const void *X, int64_t ldx, float *V, int64_t 
         sa.err = &hdr->err;
         LORA_CUDA(launch_shrink(sa, L.max_groups, 1, 1, s));
     }
+    return LORA_OK;
+}
+
+lora_status lora_linear_sgmv(const void *X, int64_t ldx, const void *W, int64_t ldw, void *Y, int64_t ldy,
+                             const lora_pool *pool, const int32_t *seg_off, const int32_t *seg_ad,
+                             int32_t n_seg, int32_t N, float scale, void *ws, size_t ws_bytes, void *stream)
+{
+    LORA_TRY(check_pool(pool));
+    if (N < 0 || n_seg < 0 || !seg_off || (n_seg > 0 && !seg_ad))
+        return LORA_ERR_INVALID_ARG;
+    LORA_TRY(check_mat(X, ldx, pool->d_in, N));
+    LORA_TRY(check_mat(Y, ldy, pool->d_out, N));
+    if (!W)
+        return LORA_ERR_INVALID_ARG;
+    LORA_TRY(check_mat(W, ldw, pool->d_in, pool->d_out));
+    Layout L;
+    if (!layout(LORA_OP_LINEAR, N, pool->n_adapters, pool->d_in, pool->max_rank, n_seg, 1, &L))
+        return LORA_ERR_INVALID_ARG;
+    LORA_TRY(check_ws(ws, ws_bytes, L));
+    if (N == 0 || n_seg == 0)
+        return LORA_OK;
+    if (!tc_enabled())
+        return LORA_ERR_UNSUPPORTED;
+    cudaStream_t s = (cudaStream_t)stream;
+    WsHeader *hdr = at<WsHeader>(ws, L.hdr);
+    Group *groups = at<Group>(ws, L.groups);
+    __nv_bfloat16 *Vb = at<__nv_bfloat16>(ws, L.V);
+    const int64_t ldvb = 2 * (int64_t)L.kv;
+
+    TcArgs ta = {};
+    tc_encode_a(ta, pool->A, pool->A_elems, pool->d_in);
+    LinArgs la = {};
+    la.kv = L.kv;
+    if (!tc_encode_x(ta, X, N, pool->d_in, ldx) ||
+        !lin_encode(la, X, ldx, N, W, ldw, Vb, ldvb, pool->B, pool->B_elems, pool->d_in, pool->d_out))
+        return LORA_ERR_UNSUPPORTED;
+
+    PlanArgs pa = {};
+    pa.mode = kModeSgmv;
+    pa.N = N;
+    pa.item_off = seg_off;
+    pa.n_items = n_seg;
+    pa.groups = groups;
+    pa.max_groups = L.max_groups;
+    pa.group = kTcGroup;
+    pa.hdr = hdr;
+    LORA_CUDA(launch_plan(pa, s));
+
+    // s V for every tile, as bf16 high and low parts
+    ta.mode = kModeSgmv;
+    ta.groups = groups;
+    ta.hdr = hdr;
+    ta.seg_ad = seg_ad;
+    ta.max_ads = 1;
+    ta.scale = scale;
+    ta.pool = pool_dev(pool);
+    ta.V = nullptr;
+    ta.ldv = 0;
+    ta.slot_stride = 0;
+    ta.Vb = Vb;
+    ta.ldvb = ldvb;
+    ta.vb_lo = L.kv;
+    ta.allow_none = 1;
+    ta.err = &hdr->err;
+    const int max_tiles = N / kTcGroup + n_seg + 1;
+    LORA_CUDA(launch_tc_shrink(ta, max_tiles, pool->max_rank, s));
+
+    la.groups = groups;
+    la.hdr = hdr;
+    la.seg_ad = seg_ad;
+    la.pool = pool_dev(pool);
+    la.Y = static_cast<__nv_bfloat16 *>(Y);
+    la.ldy = ldy;
+    la.err = &hdr->err;
+    const int64_t n_ns = (pool->d_out + 255) / 256;
+    const int64_t max_units = (int64_t)max_tiles * n_ns;
+    LORA_CUDA(launch_tc_linear(la, (int)(max_units < (1 << 30) ? max_units : (1 << 30)), s));
     return LORA_OK;
 }
 

@@ -70,6 +70,28 @@ struct PoolDev {
     int32_t n_adapters, max_rank, d_in, d_out;
 };
 
+// Adapter a of pool P passes the device checks: id in range, rank a multiple of 8
+// in [8, max_rank], A and B offsets non-negative multiples of 8 whose matrices end
+// inside the pool.
+__device__ __forceinline__ bool pool_adapter_ok(const PoolDev &P, int32_t a, int32_t *r_out, int64_t *aoff,
+                                                int64_t *boff)
+{
+    if (a < 0 || a >= P.n_adapters)
+        return false;
+    const int32_t r = P.rank[a];
+    const int64_t ao = P.A_off[a], bo = P.B_off[a];
+    if (r < 8 || r > P.max_rank || (r & 7))
+        return false;
+    if (ao < 0 || (ao & 7) || ao + (int64_t)r * P.d_in > P.A_elems)
+        return false;
+    if (bo < 0 || (bo & 7) || bo + (int64_t)r * P.d_out > P.B_elems)
+        return false;
+    *r_out = r;
+    *aoff = ao;
+    *boff = bo;
+    return true;
+}
+
 struct ShrinkArgs {
     const __nv_bfloat16 *X;
     int64_t ldx;
@@ -227,6 +249,10 @@ struct TcArgs {
     float *V;                // fp32 intermediate, row stride ldv, stacked adapters slot_stride apart
     int64_t ldv;
     int32_t slot_stride;
+    __nv_bfloat16 *Vb;       // shrink, if set (instead of V): scale * v as bf16 high part at Vb[n][c]
+    int64_t ldvb;            //   and low part at Vb[n][vb_lo + c]
+    int32_t vb_lo;
+    int32_t allow_none;      // an item adapter of -1 means no adapter (not reported)
     __nv_bfloat16 *Y;
     int64_t ldy;
     uint32_t *err;
@@ -243,6 +269,30 @@ cudaError_t launch_tc_shrink(const TcArgs &a, int max_tiles, int kk, cudaStream_
 // kk: the largest stacked rank of any item (max_rank, or max_ads * max_rank)
 cudaError_t launch_tc_expand(const TcArgs &a, int kk, cudaStream_t s);
 bool tc_enabled();
+
+// ------------------------------------------- projection + LoRA delta (tcgen05)
+struct LinArgs {
+    CUtensorMap map_x;       // X [N, d_in], boxes 64 x 128, 128-byte swizzle
+    CUtensorMap map_w;       // W [d_out, d_in], boxes 64 x 256
+    CUtensorMap map_v;       // s V as bf16 parts [N, 2 kv] (high, then low from column kv), boxes 64 x 128
+    CUtensorMap map_b[4];    // B pool as [B_elems / r, r], r = 16 << m, boxes of min(r, 64) x 128 rows
+    int32_t b_tma;           // bit m: map_b[m] valid
+    int32_t kv;              // column of the low parts (max_rank rounded up to 64)
+    const Group *groups;     // tiles of <= 128 rows, one segment each
+    const WsHeader *hdr;
+    const int32_t *seg_ad;   // -1: no adapter
+    PoolDev pool;
+    __nv_bfloat16 *Y;
+    int64_t ldy;
+    int32_t d_in, d_out;
+    uint32_t *err;
+};
+
+// Fills the tensor maps, d_in and d_out (kv must be set first); false if a map
+// cannot be encoded (alignment, sizes).
+bool lin_encode(LinArgs &a, const void *X, int64_t ldx, int32_t N, const void *W, int64_t ldw, const void *Vb,
+                int64_t ldvb, const void *B, int64_t B_elems, int32_t d_in, int32_t d_out);
+cudaError_t launch_tc_linear(const LinArgs &a, int max_units, cudaStream_t s);
 
 // Workspace bytes of lora_merge (0 for unsupported sizes).
 size_t merge_workspace_size(int32_t d_in, int32_t d_out, int32_t max_rank);

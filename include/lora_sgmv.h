@@ -109,7 +109,8 @@ typedef enum {
     LORA_OP_SGMV_EXPAND = 2,
     LORA_OP_APPLY_MULTI = 3,
     LORA_OP_ROUTE = 4,
-    LORA_OP_MERGE = 5
+    LORA_OP_MERGE = 5,
+    LORA_OP_LINEAR = 6
 } lora_op;
 
 /* Bytes of workspace `op` needs for N token rows.  n_items = n_seg for the
@@ -205,6 +206,32 @@ LORA_API lora_status lora_sgmv_shrink_proj(const void *X, int64_t ldx, float *V,
                              const lora_pool *pools, int32_t n_proj, const int32_t *seg_off,
                              const int32_t *seg_ad, int32_t n_seg, int32_t N,
                              void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * lora_linear_sgmv -- an adapted projection computed unmerged in one pass of
+ * the tensor cores ("Serving several LoRAs, ControlNet and IP-Adapter",
+ * section "LoRA: merged or alongside": served unmerged, the layer adds the
+ * low-rank x A^T B^T to x W^T):
+ *   Y[n][o] = sum_i W[o][i] X[n][i] + scale * sum_{j < rank[a]} B[a][o][j] V[n][j],
+ *   V[n][j] = sum_i A[a][j][i] X[n][i],
+ * for seg_off[k] <= n < seg_off[k+1], a = seg_ad[k]; seg_ad[k] = -1 means no
+ * adapter (Y = W X only).  Rows outside every segment are not written.  Y is
+ * OUTPUT ONLY (overwritten, not accumulated), rounded to bf16 once.
+ * W: device bf16 [d_out, d_in] row-major (a torch Linear weight), leading
+ * dimension ldw >= d_in, multiple of 8, 16-byte aligned; X [N, ldx] and
+ * Y [N, ldy] as elsewhere; pool->d_in / d_out give the projection's shape.
+ * Adapters in the LoRA part must have rank 16, 32, 64 or 128 with B_off[a]
+ * a multiple of the rank (what a packed pool of those ranks gives); a segment
+ * whose adapter fails this or the usual device checks gets Y = W X and sets
+ * LORA_ERR_BAD_ADAPTER.  Workspace: lora_workspace_size(LORA_OP_LINEAR, N,
+ * n_adapters, d_in, d_out, max_rank, n_seg, 0) (it holds s V).  Launches
+ * three kernels (plan, tcgen05 shrink, tcgen05 projection).  Needs the
+ * tensor-core path (B200): LORA_ERR_UNSUPPORTED where tensor maps cannot be
+ * built for the given pointers and strides.
+ */
+LORA_API lora_status lora_linear_sgmv(const void *X, int64_t ldx, const void *W, int64_t ldw, void *Y, int64_t ldy,
+                             const lora_pool *pool, const int32_t *seg_off, const int32_t *seg_ad,
+                             int32_t n_seg, int32_t N, float scale, void *ws, size_t ws_bytes, void *stream);
 
 /*
  * lora_sgmv_expand -- the second half of the segmented product:

@@ -118,8 +118,11 @@ class Oracle:
                                            P, i32, P]
         lib.oracle_route.argtypes = [P, i32, i32, P, P, P, P, P]
         lib.oracle_merge.argtypes = [P, i64, P, P, P, P, P, i32, i32, i32, i32, f64, P, i32, P]
+        lib.oracle_linear_sgmv.argtypes = [P, i64, P, i64, P, P, P, P, P, i32, i32, i32, P, P, i32, i32, f64,
+                                           P, i32, P]
         for f in (lib.oracle_bgmv_delta, lib.oracle_sgmv_shrink, lib.oracle_sgmv_expand,
-                  lib.oracle_sgmv_delta, lib.oracle_apply_multi, lib.oracle_route, lib.oracle_merge):
+                  lib.oracle_sgmv_delta, lib.oracle_apply_multi, lib.oracle_route, lib.oracle_merge,
+                  lib.oracle_linear_sgmv):
             f.restype = ctypes.c_int
         self.lib = lib
         self.path = path
@@ -217,6 +220,24 @@ class Oracle:
         _check(rc, "merge")
         return Wm
 
+    def linear_sgmv(self, X: np.ndarray, W: np.ndarray, pool: HostPool, seg_off: np.ndarray,
+                    seg_ad: np.ndarray, scale: float, rows: Optional[np.ndarray] = None) -> np.ndarray:
+        """Y[k] = W x[n] + scale * B[a] A[a] x[n] (n = rows[k], a = its segment's adapter, -1: none);
+        zero rows outside every segment; unrounded."""
+        X = _c(X, np.uint16)
+        W = _c(W, np.uint16)
+        seg_off = _c(seg_off, np.int32)
+        seg_ad = _c(seg_ad, np.int32)
+        N = int(X.shape[0])
+        rows, n_rows = _rows(rows, N)
+        Y = np.zeros((n_rows, pool.d_out), dtype=np.float64)
+        rc = self.lib.oracle_linear_sgmv(_p(X), X.shape[1], _p(W), W.shape[1], _p(pool.A), _p(pool.A_off),
+                                         _p(pool.B), _p(pool.B_off), _p(pool.rank), pool.n_adapters, pool.d_in,
+                                         pool.d_out, _p(seg_off), _p(seg_ad), int(seg_ad.shape[0]), N,
+                                         float(scale), _p(rows), n_rows, _p(Y))
+        _check(rc, "linear_sgmv")
+        return Y
+
     def route(self, ids: np.ndarray, n_adapters: int):
         """Stable counting sort of ids by adapter: (perm, seg_off, seg_ad); id -1 left out."""
         ids = _c(ids, np.int32)
@@ -269,6 +290,10 @@ def route(*a, **k):
 
 def merge(*a, **k):
     return default().merge(*a, **k)
+
+
+def linear_sgmv(*a, **k):
+    return default().linear_sgmv(*a, **k)
 
 
 def widen_bf16(bits: np.ndarray) -> np.ndarray:

@@ -373,3 +373,53 @@ int oracle_merge(const uint16_t *W, int64_t ldw,
     }
     return status;
 }
+
+/*
+ * A projection with its LoRA delta, computed unmerged (same page, section
+ * "LoRA: merged or alongside": the unmerged layer adds x A^T B^T to x W^T).
+ * For token n = rows[k] in segment g with adapter a = seg_ad[g]:
+ *     Y[k][o] = sum_i W[o][i] * x[n][i] + s * sum_j B[a][o][j] * v_j,
+ *     v_j     = sum_i A[a][j][i] * x[n][i],
+ * and seg_ad[g] == -1 means no adapter (the first sum alone).  W is
+ * [d_out, d_in] (bf16 bit patterns, row stride ldw).  Rows outside every
+ * segment get zeros (the library leaves them untouched).
+ */
+int oracle_linear_sgmv(const uint16_t *X, int64_t ldx, const uint16_t *W, int64_t ldw,
+                       const uint16_t *A, const int64_t *A_off,
+                       const uint16_t *B, const int64_t *B_off, const int32_t *rank,
+                       int32_t n_adapters, int32_t d_in, int32_t d_out,
+                       const int32_t *seg_off, const int32_t *seg_ad, int32_t n_seg, int32_t N,
+                       double scale, const int32_t *rows, int32_t n_rows, double *Y)
+{
+    int status = check_segments(seg_off, n_seg, N);
+    if (status != ORC_OK)
+        return status;
+    if (rows == NULL)
+        n_rows = N;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int32_t k = 0; k < n_rows; ++k) {
+        int32_t n = rows ? rows[k] : k;
+        const uint16_t *x = X + (int64_t)n * ldx;
+        double v[128];
+        double *y_row = Y + (int64_t)k * d_out;
+        for (int32_t o = 0; o < d_out; ++o)
+            y_row[o] = 0.0;
+        int32_t sg = segment_of(seg_off, n_seg, n);
+        if (sg < 0)
+            continue;
+        for (int32_t o = 0; o < d_out; ++o) {
+            double acc = 0.0;
+            for (int32_t i = 0; i < d_in; ++i)
+                acc += widen_bf16(W[(int64_t)o * ldw + i]) * widen_bf16(x[i]);
+            y_row[o] = acc;
+        }
+        if (seg_ad[sg] == -1)
+            continue;
+        int rc = one_adapter(x, A, A_off, B, B_off, rank, n_adapters, d_in, d_out, seg_ad[sg], scale, v, y_row);
+        if (rc != ORC_OK) {
+#pragma omp atomic write
+            status = rc;
+        }
+    }
+    return status;
+}

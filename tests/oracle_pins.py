@@ -352,4 +352,42 @@ def pin_bad_metadata(orc):
         raise AssertionError("non-monotone segments accepted")
 
 
+def pin_linear_is_the_merged_weight_product(orc):
+    """The projection with its LoRA delta equals x (W + s B_a A_a)^T (numpy float64), row
+    by row, for each segment's adapter -- the merged-weight identity of the handbook page
+    -- and the base product x W^T alone for a segment with adapter -1; rows outside every
+    segment are zero.  d_in != d_out != rank, so a transposed W or B fails."""
+    rng = np.random.default_rng(31)
+    d_in, d_out = 40, 24
+    p = rand_host_pool(rng, [16, 8, 24], d_in, d_out)
+    W = rand_x(rng, d_out, d_in)
+    seg_off = np.array([2, 7, 7, 12, 17], np.int32)
+    seg_ad = np.array([2, 0, -1, 1], np.int32)
+    N = 19
+    X = rand_x(rng, N, d_in)
+    s = 0.625
+    Y = orc.linear_sgmv(X, W, p, seg_off, seg_ad, s)
+    Xd, Wd = widen(X), widen(W)
+    want = np.zeros((N, d_out))
+    for k, a in enumerate(seg_ad):
+        Wm = Wd if a == -1 else Wd + s * (B_of(p, a) @ A_of(p, a))
+        for n in range(seg_off[k], seg_off[k + 1]):
+            want[n] = Xd[n] @ Wm.T
+    _close(Y, want)
+    rows = np.array([12, 0, 3, 18], np.int32)
+    _close(orc.linear_sgmv(X, W, p, seg_off, seg_ad, s, rows=rows), want[rows])
+
+
+def pin_linear_zero_B_is_the_base_product(orc):
+    """With every B zero the LoRA part vanishes: y = x W^T exactly as numpy computes it."""
+    rng = np.random.default_rng(32)
+    d_in, d_out = 24, 56
+    p = rand_host_pool(rng, [8, 16], d_in, d_out, zero_B=True)
+    W = rand_x(rng, d_out, d_in)
+    X = rand_x(rng, 10, d_in)
+    seg_off = np.array([0, 4, 10], np.int32)
+    Y = orc.linear_sgmv(X, W, p, seg_off, np.array([1, 0], np.int32), 3.0)
+    _close(Y, widen(X) @ widen(W).T)
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -37,7 +37,7 @@ def test_header_declares_the_entry_points():
     names = set(declared())
     assert {"lora_bgmv", "lora_sgmv_shrink", "lora_sgmv_expand", "lora_apply_multi", "lora_route",
             "lora_workspace_size", "lora_workspace_init", "lora_get_error", "lora_version",
-            "lora_merge", "lora_sgmv_shrink_proj"} <= names
+            "lora_merge", "lora_sgmv_shrink_proj", "lora_linear_sgmv"} <= names
 
 
 def test_every_declared_symbol_is_exported(lib):
@@ -171,3 +171,26 @@ def test_shrink_proj_validates(lib):
     assert sh(FAKE, 64, FAKE, 56, three, 3, FAKE, FAKE, 2, 4, None, 0, None) == WORKSPACE
     # two projections only: ldv 24 is enough
     assert sh(FAKE, 64, FAKE, 24, three, 2, FAKE, FAKE, 2, 4, None, 0, None) == WORKSPACE
+
+
+def test_linear_validates(lib):
+    p = ctypes.byref(_pool())          # d_in 64, d_out 32, max_rank 16
+    ln = lib.lora_linear_sgmv
+    # W missing / W leading dimension below d_in / misaligned W
+    assert ln(FAKE, 64, None, 64, FAKE, 32, p, FAKE, FAKE, 2, 4, 1.0, None, 0, None) == INVALID
+    assert ln(FAKE, 64, FAKE, 32, FAKE, 32, p, FAKE, FAKE, 2, 4, 1.0, None, 0, None) == INVALID
+    assert ln(FAKE, 64, FAKE + 2, 64, FAKE, 32, p, FAKE, FAKE, 2, 4, 1.0, None, 0, None) == UNSUPPORTED
+    # Y and X as elsewhere; segments; workspace
+    assert ln(FAKE, 64, FAKE, 64, FAKE, 16, p, FAKE, FAKE, 2, 4, 1.0, None, 0, None) == INVALID
+    assert ln(FAKE, 64, FAKE, 64, FAKE, 32, p, None, FAKE, 2, 4, 1.0, None, 0, None) == INVALID
+    assert ln(FAKE, 64, FAKE, 64, FAKE, 32, None, FAKE, FAKE, 2, 4, 1.0, None, 0, None) == INVALID
+    assert ln(FAKE, 64, FAKE, 64, FAKE, 32, p, FAKE, FAKE, 2, 4, 1.0, None, 0, None) == WORKSPACE
+
+
+def test_linear_workspace_and_launches(lib):
+    # header + tiles + s V as bf16 high and low parts, max_rank rounded up to 64 per part
+    n = L.lora_workspace_size(L.OP_LINEAR, 1000, 64, 4096, 14336, 64, 8)
+    assert n >= 1000 * 2 * 64 * 2
+    assert L.lora_workspace_size(L.OP_LINEAR, 1000, 64, 4096, 14336, 128, 8) - n >= 1000 * 2 * 64 * 2
+    assert L.lora_kernel_launches(L.OP_LINEAR, 1000, 64, 4096, 8) == 3
+    assert L.lora_kernel_launches(L.OP_LINEAR, 1000, 64, 4096, 0) == 0

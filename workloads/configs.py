@@ -251,6 +251,27 @@ class MergeCall:
 
 
 @dataclass
+class LinearCall:
+    """The projection with its LoRA delta: Y = X W^T + scale * (X A^T B^T per segment's
+    adapter); Y is the output (overwritten)."""
+
+    name: str
+    X: torch.Tensor          # bf16 [N, d_in]
+    W: torch.Tensor          # bf16 [d_out, d_in] (the base weight)
+    Y: torch.Tensor          # bf16 [N, d_out] (output)
+    pool: Pool
+    seg_off: torch.Tensor
+    seg_ad: torch.Tensor
+    seg_off_h: np.ndarray
+    seg_ad_h: np.ndarray
+    scale: float
+
+    @property
+    def n_tokens(self) -> int:
+        return int(self.X.shape[0])
+
+
+@dataclass
 class Workload:
     name: str
     calls: list
@@ -326,6 +347,7 @@ WORKLOAD_NAMES = [
     "diffusion_multi",    # 16 images x 4096 tokens, 1280->1280 x QKVO, r32, 200 adapters, 1-3 per image
     "merge_mlp_up",       # fold one rank-64 adapter into W [14336, 4096] (Llama-3-8B MLP up-proj) in place
     "prefill_qkv",        # the prefill segments over Llama-3-8B q/k/v (4096 -> 4096/1024/1024), r64, X shared
+    "prefill_linear_up",  # the prefill segments through the MLP up-proj W [14336, 4096] with its LoRA, fused
 ]
 
 LLAMA3_8B_PROJ = [  # name, d_in, d_out, which input it reads
@@ -460,4 +482,26 @@ def make_workload(which, device="cpu", seed: Optional[int] = None, y0: str = "ze
                                    seed * 100 + p_i))
         return Workload("prefill_qkv", calls, {"tokens": N, "op": "sgmv_proj", "x_read_once": True,
                                                "requests": n_req})
+    if idx == 7:
+        # the prefill recipe through the whole adapted projection: y = x W^T + s x A^T B^T
+        n_req = overrides.get("n_req", 32)
+        lo, hi = overrides.get("len_range", (128, 1024))
+        d_in = overrides.get("d_in", 4096)
+        d_out = overrides.get("d_out", 14336)
+        r = overrides.get("rank", 64)
+        n_ad = overrides.get("n_adapters", 64)
+        lens = rng.integers(lo, hi + 1, size=n_req).astype(np.int64)
+        req_ids = zipf_ids(rng, n_ad, overrides.get("zipf_s", 1.1), n_req)
+        order = np.argsort(req_ids, kind="stable")
+        tok_ids = np.repeat(req_ids[order], lens[order]).astype(np.int32)
+        seg_off, seg_ad = segments_from_sorted_ids(tok_ids, n_ad, keep_empty=False)
+        N = int(lens.sum())
+        pool = make_pool([r] * n_ad, d_in, d_out, seed, device)
+        X = _x(N, d_in, gen, device)
+        # base weight ~ N(0, 1/d_in), like the adapters' A: x W^T and the delta are both O(1)
+        W = _randn_rows_bf16(d_out, d_in, 1.0 / math.sqrt(d_in), gen, device)
+        Y = torch.zeros(N, d_out, dtype=BF16, device=device)
+        call = LinearCall("up", X, W, Y, pool, torch.tensor(seg_off, device=device),
+                          torch.tensor(seg_ad, device=device), seg_off, seg_ad, overrides.get("scale", 1.0))
+        return Workload("prefill_linear_up", [call], {"tokens": N, "op": "linear", "requests": n_req})
     raise ValueError(f"unknown workload {which!r}")
