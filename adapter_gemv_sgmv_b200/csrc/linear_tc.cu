@@ -4,24 +4,27 @@
 //
 //     Y[n] = W x[n] + s B[a] (A[a] x[n])       (a = the row's segment adapter; -1: none)
 //
-// Unit = (tile of <= 128 rows of one segment, slice of 256 outputs).  One TMEM
-// accumulator D[128 x 256] takes X_tile W_slice^T over d_in in 64-column k-blocks
-// and then, as further k-blocks, (s V)_tile B[a]_slice^T: the tcgen05 shrink has
-// already written s V = s A[a] x as two bf16 parts (high and low), each contracted
-// against the same B columns, so the delta joins the base product in fp32 and y is
-// rounded to bf16 once.  Y is written, never read.
+// Unit = (pair of tiles of <= 128 rows, each inside one segment; slice of 256
+// outputs).  Two TMEM accumulators D0, D1 [128 x 256] take X_tile W_slice^T over
+// d_in in 64-column k-blocks, both tiles against the same W box (so W crosses
+// from L2 once per 256 rows), and then, as further k-blocks, each tile's
+// (s V)_tile B[a]_slice^T: the tcgen05 shrink has already written s V = s A[a] x as
+// two bf16 parts (high and low), each contracted against the same B columns, so
+// the delta joins the base product in fp32 and y is rounded to bf16 once.  Y is
+// written, never read.
 //
 // One persistent CTA per SM, 320 threads, warp specialised:
-//   warp 0     producer: TMA boxes into a four-stage ring of 48 KB stages -- a
-//              128 x 64 x box and a 256 x 64 W box per base k-block; the s V part box
-//              and two 128-row boxes of the adapter's B columns per LoRA k-block;
+//   warp 0     producer: TMA boxes into a three-stage ring of 64 KB stages -- two
+//              128 x 64 x boxes and a 256 x 64 W box per base k-block; the s V part
+//              box and two 128-row boxes of the adapter's B columns per LoRA k-block;
 //   warp 1     one thread issues tcgen05.mma (M = 128, N = 256, K = 16) and commits;
-//   warps 2-9  epilogue: two warps per TMEM lane quarter, 128 columns each --
-//              tcgen05.ld, round to bf16, 16-byte stores.
-// Two 256-column accumulators let one unit's epilogue overlap the next unit's main
-// loop.  Units go out in blocks of all tiles against 8 output slices, and the CTAs
-// take consecutive units, so the units in flight at one time share a few MB of X
-// and W in L2 (the W slices stay there for the whole block).
+//   warps 2-9  epilogue: four warps per tile (one per TMEM lane quarter), 256
+//              columns each -- tcgen05.ld, round to bf16, 16-byte stores.
+// The two accumulators fill all 512 TMEM columns, so a unit's epilogue runs while
+// the producer refills the ring for the next unit.  Units go out in blocks of all
+// tile pairs against 8 output slices, and the CTAs take consecutive units, so the
+// units in flight at one time share a few MB of X and W in L2 (the W slices stay
+// there for the whole block).
 //
 // The LoRA k-blocks read B through the pool views of ranks 16, 32, 64 and 128
 // (adapter offsets multiples of the rank); a segment whose adapter is outside
@@ -37,25 +40,25 @@ namespace {
 constexpr int kLinThreads = 320;            // producer, MMA, 8 epilogue warps
 constexpr int kLinEpiWarps = 8;
 constexpr int kLN = 256;                    // outputs per unit (MMA N)
-constexpr int kLStage = kAtom + kLN * 128;  // x (or s V) atom + W (or B) box: 48 KB
-constexpr int kLStages = 4;
+constexpr int kLStage = 2 * kAtom + kLN * 128;   // two x atoms (a pair of tiles) + W box: 64 KB
+constexpr int kLStages = 3;
 constexpr int kLNsBlock = 8;                // output slices per block of the unit order
 
 struct LinUnit {
-    int tile, ns;
+    int pair, ns;
 };
 
-// Unit u in the blocked order: block k holds every tile against slices
-// 8k .. 8k + 7 (fewer in the last block), tile-major inside the block.
-__device__ __forceinline__ LinUnit lin_unit(int64_t u, int n_tiles, int n_ns)
+// Unit u in the blocked order: block k holds every tile pair against slices
+// 8k .. 8k + 7 (fewer in the last block), pair-major inside the block.
+__device__ __forceinline__ LinUnit lin_unit(int64_t u, int n_pairs, int n_ns)
 {
-    const int64_t per_blk = (int64_t)n_tiles * kLNsBlock;
+    const int64_t per_blk = (int64_t)n_pairs * kLNsBlock;
     const int blk = (int)(u / per_blk);
     const int64_t rem = u - blk * per_blk;
     const int nsb = min(kLNsBlock, n_ns - blk * kLNsBlock);
     LinUnit x;
-    x.tile = (int)(rem / nsb);
-    x.ns = blk * kLNsBlock + (int)(rem - (int64_t)x.tile * nsb);
+    x.pair = (int)(rem / nsb);
+    x.ns = blk * kLNsBlock + (int)(rem - (int64_t)x.pair * nsb);
     return x;
 }
 
@@ -90,12 +93,33 @@ __device__ LinAd lin_adapter(const LinArgs &p, int item, bool report)
 
 __device__ __forceinline__ int lora_kblocks(const LinAd &d) { return d.r ? 2 * ((d.r + 63) >> 6) : 0; }
 
+// The two tiles of pair `pair` (the second may be absent) and their adapters.
+struct LinPair {
+    Group g[2];
+    bool has1;
+    LinAd ad[2];
+    int nl[2];          // LoRA k-blocks of each tile
+};
+
+__device__ __forceinline__ LinPair lin_pair(const LinArgs &p, int pair, int n_tiles, bool report)
+{
+    LinPair x;
+    x.g[0] = p.groups[2 * pair];
+    x.has1 = 2 * pair + 1 < n_tiles;
+    x.g[1] = x.has1 ? p.groups[2 * pair + 1] : x.g[0];
+    x.ad[0] = lin_adapter(p, x.g[0].item, report);
+    x.ad[1] = x.has1 ? lin_adapter(p, x.g[1].item, report) : LinAd{0, 0, 0};
+    x.nl[0] = lora_kblocks(x.ad[0]);
+    x.nl[1] = lora_kblocks(x.ad[1]);
+    return x;
+}
+
 __global__ void __launch_bounds__(kLinThreads, 1) k_tc_linear(const __grid_constant__ LinArgs p)
 {
     extern __shared__ __align__(1024) unsigned char sm_dyn[];
     unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(sm_dyn) + 1023) & ~(uintptr_t)1023);
     __shared__ __align__(8) uint64_t full_bar[kLStages], empty_bar[kLStages];
-    __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2];
+    __shared__ __align__(8) uint64_t acc_full, acc_empty;
     __shared__ uint32_t tmem_base;
     __shared__ int abort_flag;
 
@@ -109,10 +133,8 @@ __global__ void __launch_bounds__(kLinThreads, 1) k_tc_linear(const __grid_const
             mbar_init(&full_bar[s], 1);          // producer's expect_tx
             mbar_init(&empty_bar[s], 1);         // MMA commit
         }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&acc_full[b], 1);          // MMA commit
-            mbar_init(&acc_empty[b], kLinEpiWarps);
-        }
+        mbar_init(&acc_full, 1);                 // MMA commit
+        mbar_init(&acc_empty, kLinEpiWarps);
         abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -125,19 +147,18 @@ __global__ void __launch_bounds__(kLinThreads, 1) k_tc_linear(const __grid_const
     pdl_wait();                                   // tiles (plan) and s V (shrink) are complete
     pdl_trigger();
     const int n_tiles = p.hdr->n_groups;
-    const int64_t n_units = (int64_t)n_tiles * n_ns;
+    const int n_pairs = (n_tiles + 1) / 2;
+    const int64_t n_units = (int64_t)n_pairs * n_ns;
 
     if (warp == 0) {
         // ------------------------------------------------ producer
         int it = 0;
         const uint64_t pol_x = policy_evict_first(), pol_w = policy_evict_last();
         for (int64_t u = blockIdx.x; u < n_units; u += G) {
-            const LinUnit t = lin_unit(u, n_tiles, n_ns);
-            const Group gr = p.groups[t.tile];
-            const LinAd ad = lin_adapter(p, gr.item, lane == 0 && t.ns == 0);
-            const int n_all = n_kb + lora_kblocks(ad);
-            const int o0 = t.ns * kLN;
-            const int w = ad.r < 64 ? ad.r : 64;          // B columns per LoRA k-block
+            const LinUnit un = lin_unit(u, n_pairs, n_ns);
+            const LinPair pr = lin_pair(p, un.pair, n_tiles, lane == 0 && un.ns == 0);
+            const int n_all = n_kb + pr.nl[0] + pr.nl[1];
+            const int o0 = un.ns * kLN;
             for (int kb = 0; kb < n_all; ++kb, ++it) {
                 const int s = it % kLStages;
                 const uint32_t ph = (it / kLStages) & 1;
@@ -145,16 +166,26 @@ __global__ void __launch_bounds__(kLinThreads, 1) k_tc_linear(const __grid_const
                     goto done;
                 if (lane == 0) {
                     unsigned char *xs = sm + s * kLStage;
-                    unsigned char *wsm = xs + kAtom;
+                    unsigned char *wsm = xs + 2 * kAtom;
                     if (kb < n_kb) {
-                        mbar_arrive_expect_tx(&full_bar[s], (uint32_t)kLStage);
-                        tma_load_2d_hint(xs, &p.map_x, &full_bar[s], kb * kBK, gr.p0, pol_x);
+                        mbar_arrive_expect_tx(&full_bar[s], (uint32_t)((pr.has1 ? 2 : 1) * kAtom + kLN * 128));
+                        tma_load_2d_hint(xs, &p.map_x, &full_bar[s], kb * kBK, pr.g[0].p0, pol_x);
+                        if (pr.has1)
+                            tma_load_2d_hint(xs + kAtom, &p.map_x, &full_bar[s], kb * kBK, pr.g[1].p0, pol_x);
                         tma_load_2d_hint(wsm, &p.map_w, &full_bar[s], kb * kBK, o0, pol_w);
                     } else {
-                        // LoRA k-block j: part j % 2 (high, low) of rank columns 64 (j / 2) ..
-                        const int j = kb - n_kb, part = j & 1, c = j >> 1;
+                        // LoRA k-blocks of tile 0, then of tile 1; k-block j of a tile: part
+                        // j % 2 (high, low) of rank columns 64 (j / 2) ..
+                        int j = kb - n_kb;
+                        const int ti = j < pr.nl[0] ? 0 : 1;
+                        if (ti)
+                            j -= pr.nl[0];
+                        const LinAd ad = ti ? pr.ad[1] : pr.ad[0];
+                        const int part = j & 1, c = j >> 1;
+                        const int w = ad.r < 64 ? ad.r : 64;
                         mbar_arrive_expect_tx(&full_bar[s], (uint32_t)(kAtom + 2 * 128 * w * 2));
-                        tma_load_2d_hint(xs, &p.map_v, &full_bar[s], part * p.kv + c * 64, gr.p0, pol_x);
+                        tma_load_2d_hint(xs, &p.map_v, &full_bar[s], part * p.kv + c * 64,
+                                         ti ? pr.g[1].p0 : pr.g[0].p0, pol_x);
                         tma_load_2d_hint(wsm, &p.map_b[ad.m], &full_bar[s], c * 64, ad.brow + o0, pol_w);
                         tma_load_2d_hint(wsm + 128 * w * 2, &p.map_b[ad.m], &full_bar[s], c * 64,
                                          ad.brow + o0 + 128, pol_w);
@@ -168,12 +199,10 @@ __global__ void __launch_bounds__(kLinThreads, 1) k_tc_linear(const __grid_const
         int it = 0, t = 0;
         const uint32_t idesc = idesc_bf16(kBM, kLN);
         for (int64_t u = blockIdx.x; u < n_units; u += G, ++t) {
-            const LinUnit un = lin_unit(u, n_tiles, n_ns);
-            const LinAd ad = lin_adapter(p, p.groups[un.tile].item, false);
-            const int n_all = n_kb + lora_kblocks(ad);
-            const int steps = (ad.r < 64 ? ad.r : 64) >> 4;   // k16 steps of a LoRA k-block
-            const int b = t & 1;
-            if (!warp_wait(&acc_empty[b], ((t >> 1) & 1) ^ 1, &abort_flag, p.err))
+            const LinUnit un = lin_unit(u, n_pairs, n_ns);
+            const LinPair pr = lin_pair(p, un.pair, n_tiles, false);
+            const int n_all = n_kb + pr.nl[0] + pr.nl[1];
+            if (!warp_wait(&acc_empty, (t & 1) ^ 1, &abort_flag, p.err))
                 goto done;
             tc_fence_after();
             for (int kb = 0; kb < n_all; ++kb, ++it) {
@@ -183,19 +212,29 @@ __global__ void __launch_bounds__(kLinThreads, 1) k_tc_linear(const __grid_const
                     goto done;
                 tc_fence_after();
                 if (lane == 0) {
-                    const uint32_t xa = smem_u32(sm + s * kLStage), wa = xa + kAtom;
+                    const uint32_t xa = smem_u32(sm + s * kLStage), wa = xa + 2 * kAtom;
                     if (kb < n_kb) {
 #pragma unroll
                         for (int k = 0; k < kBK / 16; ++k)
-                            tc_mma(tmem + b * kLN, sw128_desc(xa + k * 32), sw128_desc(wa + k * 32), idesc,
+                            tc_mma(tmem, sw128_desc(xa + k * 32), sw128_desc(wa + k * 32), idesc,
                                    (kb > 0 || k > 0) ? 1u : 0u);
+                        if (pr.has1) {
+#pragma unroll
+                            for (int k = 0; k < kBK / 16; ++k)
+                                tc_mma(tmem + kLN, sw128_desc(xa + kAtom + k * 32), sw128_desc(wa + k * 32), idesc,
+                                       (kb > 0 || k > 0) ? 1u : 0u);
+                        }
                     } else {
+                        int j = kb - n_kb;
+                        const int ti = j < pr.nl[0] ? 0 : 1;
+                        const int r = ti ? pr.ad[1].r : pr.ad[0].r;
+                        const int steps = (r < 64 ? r : 64) >> 4;
                         for (int k = 0; k < steps; ++k) {
                             // B columns in the view's swizzle: 128-byte rows from rank 64 up,
                             // 64-byte rows at rank 32, 32-byte rows at rank 16
-                            const uint64_t bdesc = ad.r >= 64 ? sw128_desc(wa + k * 32)
-                                                 : (ad.r == 32 ? sw64_desc(wa + k * 32) : sw32_desc(wa));
-                            tc_mma(tmem + b * kLN, sw128_desc(xa + k * 32), bdesc, idesc, 1u);
+                            const uint64_t bdesc = r >= 64 ? sw128_desc(wa + k * 32)
+                                                 : (r == 32 ? sw64_desc(wa + k * 32) : sw32_desc(wa));
+                            tc_mma(tmem + ti * kLN, sw128_desc(xa + k * 32), bdesc, idesc, 1u);
                         }
                     }
                     tc_commit(&empty_bar[s]);
@@ -203,42 +242,45 @@ __global__ void __launch_bounds__(kLinThreads, 1) k_tc_linear(const __grid_const
                 __syncwarp();
             }
             if (lane == 0)
-                tc_commit(&acc_full[b]);
+                tc_commit(&acc_full);
             __syncwarp();
         }
     } else {
         // ------------------------------------------------ epilogue: D -> y rows
         const int e = warp - 2;                  // 0..7
         const int q = warp & 3;                  // TMEM lane quarter this warp may read
-        const int h = e >> 2;                    // 128-column half of the slice
+        const int ti = e >> 2;                   // tile of the pair (its accumulator)
         const int row = q * 32 + lane;
         int t = 0;
         for (int64_t u = blockIdx.x; u < n_units; u += G, ++t) {
-            const LinUnit un = lin_unit(u, n_tiles, n_ns);
-            const Group gr = p.groups[un.tile];
-            const int b = t & 1;
-            if (!warp_wait(&acc_full[b], (t >> 1) & 1, &abort_flag, p.err))
+            const LinUnit un = lin_unit(u, n_pairs, n_ns);
+            const int tile = 2 * un.pair + ti;
+            if (!warp_wait(&acc_full, t & 1, &abort_flag, p.err))
                 goto done;
             tc_fence_after();
-            const bool valid = row < gr.cnt;
-            __nv_bfloat16 *yrow = p.Y + (int64_t)(gr.p0 + (valid ? row : 0)) * p.ldy;
-            const int o0 = un.ns * kLN + h * 128;
+            if (tile < n_tiles) {
+                const Group gr = p.groups[tile];
+                const bool valid = row < gr.cnt;
+                __nv_bfloat16 *yrow = p.Y + (int64_t)(gr.p0 + (valid ? row : 0)) * p.ldy;
+                const int o0 = un.ns * kLN;
 #pragma unroll 1
-            for (int c0 = 0; c0 < 128; c0 += 32) {
-                float v[32];
-                tmem_ld32(tmem + b * kLN + ((uint32_t)(q * 32) << 16) + h * 128 + c0, v);
-                if (valid) {
+                for (int c0 = 0; c0 < kLN; c0 += 32) {
+                    float v[32];
+                    tmem_ld32(tmem + ti * kLN + ((uint32_t)(q * 32) << 16) + c0, v);
+                    if (valid) {
 #pragma unroll
-                    for (int g = 0; g < 4; ++g) {
-                        const int o = o0 + c0 + 8 * g;
-                        if (o < p.d_out) {
-                            uint32_t w4[4];
+                        for (int g = 0; g < 4; ++g) {
+                            const int o = o0 + c0 + 8 * g;
+                            if (o < p.d_out) {
+                                uint32_t w4[4];
 #pragma unroll
-                            for (int j = 0; j < 4; ++j) {
-                                const __nv_bfloat162 hv = __floats2bfloat162_rn(v[8 * g + 2 * j], v[8 * g + 2 * j + 1]);
-                                w4[j] = *reinterpret_cast<const uint32_t *>(&hv);
+                                for (int jj = 0; jj < 4; ++jj) {
+                                    const __nv_bfloat162 hv =
+                                        __floats2bfloat162_rn(v[8 * g + 2 * jj], v[8 * g + 2 * jj + 1]);
+                                    w4[jj] = *reinterpret_cast<const uint32_t *>(&hv);
+                                }
+                                *reinterpret_cast<uint4 *>(yrow + o) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
                             }
-                            *reinterpret_cast<uint4 *>(yrow + o) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
                         }
                     }
                 }
@@ -246,7 +288,7 @@ __global__ void __launch_bounds__(kLinThreads, 1) k_tc_linear(const __grid_const
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
-                mbar_arrive(&acc_empty[b]);
+                mbar_arrive(&acc_empty);
         }
     }
 done:
