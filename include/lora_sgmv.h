@@ -50,6 +50,15 @@
  *   that share one workspace must be ordered (same stream or events).
  * - Thread safety: the library is stateless; concurrent calls with distinct
  *   workspaces are safe.
+ * - Overlap with the previous kernel: kernels are launched with programmatic
+ *   dependent launch (environment variable LORA_SGMV_NO_PDL=1 turns it off),
+ *   so one may start while the kernel before it on the stream finishes.  Each
+ *   waits for that kernel before touching X, Y, V, W or the workspace; the
+ *   decode kernel of lora_bgmv reads ids and the adapter pool before waiting.
+ *   This matters only when the preceding kernel itself releases its dependents
+ *   early (griddepcontrol.launch_dependents) -- such a kernel must not write
+ *   ids or the pool.  Copies (cudaMemcpyAsync) and ordinary kernels before a
+ *   call are always complete before it starts.
  */
 #ifndef LORA_SGMV_H
 #define LORA_SGMV_H
