@@ -619,20 +619,22 @@ def cpu_baseline(args, wl, budget_s=12.0):
     cores = os.cpu_count() or 1
     oracle.set_threads(cores)
     hc = _host_calls(wl)
-    # calibrate: time one pass over a small row sample, then size the sample to the budget
+    # calibrate on a small row sample (after one untimed pass: the first call starts the
+    # thread pool), size a pass to about a tenth of the budget, then run passes until the
+    # budget is spent
     probe = _rows_sample(hc, min(16, wl.n_tokens), 0)
+    _oracle_pass(oracle, hc, probe)
     t0 = time.perf_counter()
     _oracle_pass(oracle, hc, probe)
     t_probe = max(time.perf_counter() - t0, 1e-4)
     per_tok = t_probe / len(probe[0])
-    n_tok = int(max(1, min(wl.n_tokens, budget_s / per_tok)))
-    passes = max(1, int(budget_s / (per_tok * n_tok)))
+    n_tok = int(max(1, min(wl.n_tokens, 0.1 * budget_s / per_tok)))
     tokens = 0
+    passes = 0
     t0 = time.perf_counter()
-    for p in range(passes):
-        tokens += _oracle_pass(oracle, hc, _rows_sample(hc, n_tok, p + 1))
-        if time.perf_counter() - t0 > 1.5 * budget_s:
-            break
+    while time.perf_counter() - t0 < budget_s and passes < 100000:
+        tokens += _oracle_pass(oracle, hc, _rows_sample(hc, n_tok, passes + 1))
+        passes += 1
     dt = time.perf_counter() - t0
     return {"value": round(tokens / dt, 2), "unit": unit_of(args.workload), "cores": oracle.threads(),
             "kind": "oracle",

@@ -79,3 +79,22 @@ def test_qkv_workload_shares_x_and_counts_it_once():
     separate = sum(accounting.call_cost(c).bytes for c in wl.calls)
     assert accounting.workload_cost(wl).bytes == separate - 2 * 2 * N * 64
     assert accounting.workload_cost(wl).tokens == N
+
+
+def test_bench_counts_the_fused_calls():
+    """Launch counts the bench claims for the shared-input and fused-projection steps
+    follow the library's own rule (one tensor-core shrink per run of projections whose
+    max ranks sum to at most 256)."""
+    import bench
+    assert bench.shrink_proj_passes([64, 64, 64]) == 1
+    assert bench.shrink_proj_passes([128, 128, 128]) == 2
+    assert bench.shrink_proj_passes([128, 8, 128]) == 2
+    assert bench.shrink_proj_passes([16, 16, 16, 16]) == 1
+    wl = make_workload("prefill_qkv", n_req=3, len_range=(200, 300), d_in=64, d_outs=(64, 16, 16), rank=8,
+                       n_adapters=5)
+    assert bench.launches_per_step(wl) == 1 + 1 + 3 * 2          # plan, shrink, 3 x (plan + expand)
+    wl = make_workload("prefill_linear_up", n_req=3, len_range=(4, 9), d_in=64, d_out=48, rank=16,
+                       n_adapters=5)
+    assert bench._is_linear(wl.calls[0]) and bench.launches_per_step(wl) == 3
+    merge = make_workload("merge_mlp_up", d_in=64, d_out=32, rank=16, n_adapters=4).calls[0]
+    assert not bench._is_linear(merge)
