@@ -359,7 +359,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) k_tc_shrink(const __grid_consta
             tc_fence_after();
             const bool valid = row < gr.cnt;
             const int64_t vr = gr.p0 + (valid ? row : 0);
-            float *vrow = p.V + vr * p.ldv;
+            float *vrow = p.Vb ? nullptr : p.V + vr * p.ldv;
             __nv_bfloat16 *brow = p.Vb ? p.Vb + vr * p.ldvb : nullptr;
             for (int c0 = 0; c0 < st.kpad; c0 += 32) {
                 float v[32];
