@@ -15,19 +15,22 @@
 // ranks in total): the shrink produces all of them in one accumulator
 // (N = stacked rank), and the expand contracts over all of them at once
 // (K = stacked rank, each adapter's scale folded into its V columns), so y is
-// read, updated and rounded to bf16 once.
+// read, updated and rounded to bf16 once.  The shrink also stacks the A rows of
+// projections that share x (up to 256 ranks), and can write s V as bf16 high
+// and low parts for the fused projection kernel.
 //
-// Both kernels are persistent (one CTA per SM, 192 threads) and warp
-// specialised:
-//   warp 0     producer: TMA for the dense operands (x tiles for the shrink, y
-//              tiles for the expand; 128-byte swizzle), cp.async for the
-//              per-adapter weight tiles (A rows / B rows, placed in the same
-//              swizzled K-major layout by hand: adapter offsets live in device
-//              memory, so no host-built tensor map can address them);
+// Both kernels are persistent and warp specialised:
+//   warp 0     producer: TMA for every operand -- x tiles (shrink) and y tiles
+//              (expand) with 128-byte swizzle, A rows through the A pool seen
+//              as [A_elems / d_in, d_in] and B slices through the B pool seen as
+//              [B_elems / r, r] per rank r (an adapter whose offset does not fit
+//              those views is gathered with cp.async into the same layout);
 //   warp 1     one thread issues tcgen05.mma (bf16 x bf16 -> fp32 in TMEM,
 //              M = 128) and tracks completion with tcgen05.commit;
-//   warps 2-5  epilogue: tcgen05.ld of the accumulator (each warp owns its
-//              32-lane quarter of TMEM = 32 rows of the tile).
+//   others     epilogue: tcgen05.ld of the accumulator (a warp reads the TMEM
+//              lane quarter of its warp index mod 4) -- four warps writing V
+//              rows in the shrink (192 threads, two CTAs per SM), sixteen
+//              adding D into y in the expand (576 threads, one CTA per SM).
 // Stages hand over through mbarriers; every wait is bounded in time and, if it
 // expires, records LORA_ERR_TIMEOUT and winds the CTA down (TMEM is freed).
 
