@@ -194,3 +194,15 @@ def test_linear_workspace_and_launches(lib):
     assert L.lora_workspace_size(L.OP_LINEAR, 1000, 64, 4096, 14336, 128, 8) - n >= 1000 * 2 * 64 * 2
     assert L.lora_kernel_launches(L.OP_LINEAR, 1000, 64, 4096, 8) == 3
     assert L.lora_kernel_launches(L.OP_LINEAR, 1000, 64, 4096, 0) == 0
+
+
+def test_empty_calls_return_before_any_launch(lib):
+    """N = 0 or no segments: the new entry points validate, then return LORA_OK without
+    touching the device (a fake but large, aligned workspace is never dereferenced)."""
+    p = ctypes.byref(_pool())
+    ws, nb = FAKE, 1 << 20
+    assert lib.lora_linear_sgmv(FAKE, 64, FAKE, 64, FAKE, 32, p, FAKE, FAKE, 2, 0, 1.0, ws, nb, None) == OK
+    assert lib.lora_linear_sgmv(FAKE, 64, FAKE, 64, FAKE, 32, p, FAKE, FAKE, 0, 4, 1.0, ws, nb, None) == OK
+    pools = _pools(_pool(), _pool(max_rank=32))
+    assert lib.lora_sgmv_shrink_proj(FAKE, 64, FAKE, 48, pools, 2, FAKE, FAKE, 2, 0, ws, nb, None) == OK
+    assert lib.lora_sgmv_shrink_proj(FAKE, 64, FAKE, 48, pools, 2, FAKE, FAKE, 0, 4, ws, nb, None) == OK

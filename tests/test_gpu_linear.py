@@ -101,3 +101,24 @@ def test_prefill_linear_full_size_sampled_rows():
     want = oracle.linear_sgmv(to_host(c.X), to_host(c.W), host_pool(c.pool), c.seg_off_h, c.seg_ad_h, c.scale,
                               rows=rows)
     check_parity(widen(to_host(c.Y))[rows], want, "prefill_linear_up")
+
+
+def test_linear_degenerate_segments():
+    """Only empty segments: nothing is written and nothing is reported.  One row in one
+    segment (a tile of one row, boxes reading past the end of x): that row is exact."""
+    rng = np.random.default_rng(6)
+    d_in, d_out = 64, 256
+    hp = rand_host_pool(rng, [16, 32], d_in, d_out)
+    W = _rand_w(rng, d_out, d_in)
+    X = rand_x(rng, 100, d_in)
+    sentinel = np.full((100, d_out), 0x4000, np.uint16)          # 2.0
+    Y = dev_bf16(sentinel)
+    ws = L.lora_linear_sgmv(dev_bf16(X), dev_bf16(W), Y, DevPool(hp), _i32([0, 0, 0]), _i32([0, 1]), 1.0)
+    assert L.lora_get_error(ws) == 0
+    assert np.all(widen(to_host(Y)) == 2.0)
+    X1 = rand_x(rng, 1, d_in)
+    Y1 = torch.zeros((1, d_out), dtype=torch.bfloat16, device=DEV)
+    ws = L.lora_linear_sgmv(dev_bf16(X1), dev_bf16(W), Y1, DevPool(hp), _i32([0, 1]), _i32([1]), 0.5)
+    assert L.lora_get_error(ws) == 0
+    want = oracle.linear_sgmv(X1, W, hp, np.array([0, 1], np.int32), np.array([1], np.int32), 0.5)
+    check_parity(widen(to_host(Y1)), want, "linear, one row")

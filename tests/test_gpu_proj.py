@@ -160,3 +160,14 @@ def test_prefill_qkv_full_size_sampled_rows():
         hp = host_pool(c.pool)
         y_exact = widen(y0)[rows] + oracle.sgmv_delta(X, hp, c.seg_off_h, c.seg_ad_h, c.scale, rows=rows)
         check_parity(widen(to_host(c.Y))[rows], y_exact, f"prefill_qkv {c.name}")
+
+
+def test_shrink_proj_only_empty_segments_writes_nothing():
+    rng = np.random.default_rng(12)
+    hps = [rand_host_pool(rng, [64, 64], 128, d) for d in (128, 64, 64)]
+    N = 300
+    X = rand_x(rng, N, 128)
+    V = torch.full((N, 192), float("nan"), dtype=torch.float32, device=DEV)
+    ws, _ = L.lora_sgmv_shrink_proj(dev_bf16(X), V, [DevPool(hp) for hp in hps], _i32([0, 0, 0]), _i32([0, 1]))
+    assert L.lora_get_error(ws) == 0
+    assert torch.isnan(V).all()
