@@ -350,6 +350,15 @@ def pin_bad_metadata(orc):
         pass
     else:
         raise AssertionError("non-monotone segments accepted")
+    # the projection: an adapter id past the pool (not -1) and non-monotone segments
+    W = rand_x(rng, 16, 16)
+    for seg_off, seg_ad in (([0, 4], [1]), ([0, 3, 2], [0, 0])):
+        try:
+            orc.linear_sgmv(X, W, p, np.array(seg_off, np.int32), np.array(seg_ad, np.int32), 1.0)
+        except OracleError:
+            pass
+        else:
+            raise AssertionError(f"linear segments {seg_off} / adapters {seg_ad} accepted")
 
 
 def pin_linear_is_the_merged_weight_product(orc):
