@@ -18,16 +18,17 @@ import threading
 __all__ = [
     "LoraError", "load", "library_path", "lora_version", "lora_workspace_size", "lora_workspace_init",
     "lora_kernel_launches",
-    "lora_get_error", "lora_route", "lora_bgmv", "lora_sgmv_shrink", "lora_sgmv_shrink_proj", "lora_sgmv_expand",
+    "lora_get_error", "lora_route", "lora_bgmv", "lora_sgmv_shrink", "lora_sgmv_shrink_proj", "lora_sgmv_apply_proj",
+    "lora_sgmv_expand",
     "lora_apply_multi", "lora_apply_multi_static", "make_pool_struct", "Workspace", "OP_BGMV", "OP_SGMV_SHRINK", "OP_SGMV_EXPAND",
-    "OP_APPLY_MULTI", "OP_ROUTE", "OP_MERGE", "OP_LINEAR", "STATUS", "lora_merge", "lora_linear_sgmv",
+    "OP_APPLY_MULTI", "OP_ROUTE", "OP_MERGE", "OP_LINEAR", "OP_APPLY_PROJ", "STATUS", "lora_merge", "lora_linear_sgmv",
     "PoolManager",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 _LIBNAME = "liblora_sgmv.so"
 
-OP_BGMV, OP_SGMV_SHRINK, OP_SGMV_EXPAND, OP_APPLY_MULTI, OP_ROUTE, OP_MERGE, OP_LINEAR = range(7)
+OP_BGMV, OP_SGMV_SHRINK, OP_SGMV_EXPAND, OP_APPLY_MULTI, OP_ROUTE, OP_MERGE, OP_LINEAR, OP_APPLY_PROJ = range(8)
 STATUS = {0: "LORA_OK", 1: "LORA_ERR_INVALID_ARG", 2: "LORA_ERR_UNSUPPORTED", 4: "LORA_ERR_BAD_ADAPTER",
           8: "LORA_ERR_BAD_SEGMENT", 16: "LORA_ERR_CUDA", 32: "LORA_ERR_WORKSPACE", 64: "LORA_ERR_TIMEOUT"}
 MAX_ADS_PER_REQ = 8
@@ -87,6 +88,8 @@ def load():
         lib.lora_sgmv_shrink.argtypes = [P, i64, P, i64, PP, P, P, i32, i32, P, sz, P]
         lib.lora_sgmv_shrink_proj.restype = ctypes.c_int
         lib.lora_linear_sgmv.restype = ctypes.c_int
+        lib.lora_sgmv_apply_proj.restype = ctypes.c_int
+        lib.lora_sgmv_apply_proj.argtypes = [P, i64, P, P, PP, i32, P, P, i32, i32, P, P, sz, P]
         lib.lora_linear_sgmv.argtypes = [P, i64, P, i64, P, i64, PP, P, P, i32, i32, f32, P, sz, P]
         lib.lora_sgmv_shrink_proj.argtypes = [P, i64, P, i64, PP, i32, P, P, i32, i32, P, sz, P]
         lib.lora_sgmv_expand.restype = ctypes.c_int
@@ -298,6 +301,35 @@ def lora_sgmv_shrink_proj(X, V, pools, seg_off, seg_ad, ws: Workspace | None = N
                                   _ptr(seg_ad), n_seg, N, ws.ptr(), ws.nbytes, _stream_ptr(stream)),
         "lora_sgmv_shrink_proj")
     return ws, cols
+
+
+def lora_sgmv_apply_proj(X, Ys, pools, seg_off, seg_ad, scales, ws: Workspace | None = None, stream=None,
+                         max_ranks=None):
+    """Ys[p][n] += scales[p] * B_p[a] A_p[a] X[n] for projections sharing X (q/k/v; gate/up):
+    one plan, one stacked shrink, one expand per projection; V stays in the workspace."""
+    lib = load()
+    pools = list(pools)
+    Ys = list(Ys)
+    _check_dev(X, seg_off, seg_ad, *Ys)
+    if max_ranks is None:
+        max_ranks = [None] * len(pools)
+    structs = [make_pool_struct(p, m) for p, m in zip(pools, max_ranks)]
+    n = len(structs)
+    if n < 1 or len(Ys) != n or len(scales) != n:
+        raise LoraError("one output and one scale per pool", 1)
+    arr = (LoraPoolStruct * n)(*structs)
+    ldx = _mat(X, structs[0].d_in, "X")
+    ys = (ctypes.c_void_p * n)(*[_ptr(Y) for Y in Ys])
+    lds = (ctypes.c_int64 * n)(*[_mat(Y, ps.d_out, "Y") for Y, ps in zip(Ys, structs)])
+    sc = (ctypes.c_float * n)(*[float(s) for s in scales])
+    N = int(X.shape[0])
+    n_seg = int(seg_ad.numel())
+    vcols = sum(ps.max_rank for ps in structs)
+    need = lora_workspace_size(OP_APPLY_PROJ, N, structs[0].n_adapters, structs[0].d_in, 0, vcols, n_seg)
+    ws = ws or _workspace(need, X.device)
+    _rc(lib.lora_sgmv_apply_proj(_ptr(X), ldx, ys, lds, arr, n, _ptr(seg_off), _ptr(seg_ad), n_seg, N, sc,
+                                 ws.ptr(), ws.nbytes, _stream_ptr(stream)), "lora_sgmv_apply_proj")
+    return ws
 
 
 def lora_linear_sgmv(X, W, Y, pool, seg_off, seg_ad, scale: float, ws: Workspace | None = None, stream=None,

@@ -65,8 +65,10 @@ struct Layout {
 bool layout(int op, int32_t N, int32_t n_adapters, int32_t d_in, int32_t max_rank, int32_t n_items,
             int32_t max_ads, Layout *L)
 {
+    // LORA_OP_APPLY_PROJ: max_rank is the V width, the projections' max ranks summed
+    const int32_t rank_cap = op == LORA_OP_APPLY_PROJ ? LORA_MAX_PROJ * LORA_MAX_RANK : LORA_MAX_RANK;
     if (N < 0 || n_adapters < 1 || n_adapters > LORA_MAX_ADAPTERS || d_in <= 0 || max_rank < 8 ||
-        max_rank > LORA_MAX_RANK)
+        max_rank > rank_cap)
         return false;
     const bool routed = op == LORA_OP_BGMV || op == LORA_OP_ROUTE;
     if (!routed && n_items < 0)
@@ -94,6 +96,8 @@ bool layout(int op, int32_t N, int32_t n_adapters, int32_t d_in, int32_t max_ran
         v = (size_t)L->n_chunks * N * max_rank * 4;
     else if (op == LORA_OP_APPLY_MULTI)
         v = (size_t)N * max_ads * max_rank * 4;
+    else if (op == LORA_OP_APPLY_PROJ)
+        v = (size_t)N * max_rank * 4;       // V of all the projections side by side
     else if (op == LORA_OP_LINEAR) {
         L->kv = (max_rank + 63) & ~63;
         v = (size_t)N * 2 * L->kv * 2;      // s V, bf16 high and low parts
@@ -171,6 +175,102 @@ T *at(void *ws, size_t off) { return reinterpret_cast<T *>(static_cast<char *>(w
             return LORA_ERR_CUDA;           \
     } while (0)
 
+// Projections sharing one input: the pools must share d_in and n_adapters; vcol[p]
+// is projection p's first column in V (the earlier pools' max_rank summed).
+lora_status check_proj_pools(const lora_pool *pools, int32_t n_proj, int32_t *vcol, int64_t *vcols)
+{
+    if (!pools || n_proj < 1)
+        return LORA_ERR_INVALID_ARG;
+    if (n_proj > LORA_MAX_PROJ)
+        return LORA_ERR_UNSUPPORTED;
+    *vcols = 0;
+    for (int p = 0; p < n_proj; ++p) {
+        LORA_TRY(check_pool(&pools[p]));
+        if (pools[p].d_in != pools[0].d_in || pools[p].n_adapters != pools[0].n_adapters)
+            return LORA_ERR_INVALID_ARG;
+        vcol[p] = (int32_t)*vcols;
+        *vcols += pools[p].max_rank;
+    }
+    return LORA_OK;
+}
+
+// The plan and the shrinks of projections sharing X into V.  tc (with ta's x map
+// encoded): tiles of 128 rows and one tensor-core launch per run of consecutive
+// projections whose max ranks fit one stacked accumulator (each launch reads X once);
+// else 8-row groups and the CUDA-core shrink once per projection.
+cudaError_t run_proj_shrinks(bool tc, const TcArgs &ta0, const void *X, int64_t ldx, float *V, int64_t ldv,
+                             const lora_pool *pools, int32_t n_proj, const int32_t *vcol, const int32_t *seg_off,
+                             const int32_t *seg_ad, int32_t n_seg, int32_t N, const Layout &L, void *ws,
+                             cudaStream_t s)
+{
+    WsHeader *hdr = at<WsHeader>(ws, L.hdr);
+    Group *groups = at<Group>(ws, L.groups);
+    const int32_t d_in = pools[0].d_in;
+    cudaError_t e;
+    PlanArgs pa = {};
+    pa.mode = kModeSgmv;
+    pa.N = N;
+    pa.item_off = seg_off;
+    pa.n_items = n_seg;
+    pa.groups = groups;
+    pa.max_groups = L.max_groups;
+    pa.group = tc ? kTcGroup : kGroup;
+    pa.hdr = hdr;
+    if ((e = launch_plan(pa, s)) != cudaSuccess)
+        return e;
+    if (tc) {
+        TcArgs ta = ta0;
+        ta.mode = kModeProj;
+        ta.groups = groups;
+        ta.hdr = hdr;
+        ta.seg_ad = seg_ad;
+        ta.max_ads = 1;
+        ta.scale = 1.0f;
+        ta.V = V;
+        ta.ldv = ldv;
+        ta.slot_stride = 0;
+        ta.err = &hdr->err;
+        for (int p0 = 0; p0 < n_proj;) {
+            int p1 = p0, kk = 0;
+            while (p1 < n_proj && kk + pools[p1].max_rank <= kKMaxShrink)
+                kk += pools[p1++].max_rank;
+            TcArgs tp = ta;
+            tp.a_tma = 0;
+            tp.n_proj = p1 - p0;
+            for (int q = p0; q < p1; ++q) {
+                tp.proj[q - p0] = pool_dev(&pools[q]);
+                tp.proj_vcol[q - p0] = vcol[q];
+                tc_encode_a(tp, pools[q].A, pools[q].A_elems, d_in, q - p0);
+            }
+            tp.pool = tp.proj[0];
+            if ((e = launch_tc_shrink(tp, N / kTcGroup + n_seg + 1, kk, s)) != cudaSuccess)
+                return e;
+            p0 = p1;
+        }
+        return cudaSuccess;
+    }
+    for (int p = 0; p < n_proj; ++p) {
+        ShrinkArgs sa = {};
+        sa.X = static_cast<const __nv_bfloat16 *>(X);
+        sa.ldx = ldx;
+        sa.perm = nullptr;
+        sa.groups = groups;
+        sa.hdr = hdr;
+        sa.mode = kModeSgmv;
+        sa.seg_ad = seg_ad;
+        sa.pool = pool_dev(&pools[p]);
+        sa.kc = d_in;
+        sa.V = V + vcol[p];
+        sa.ldv = ldv;
+        sa.chunk_stride = 0;
+        sa.slot_stride = 0;
+        sa.err = &hdr->err;
+        if ((e = launch_shrink(sa, L.max_groups, 1, 1, s)) != cudaSuccess)
+            return e;
+    }
+    return cudaSuccess;
+}
+
 }  // namespace
 
 extern "C" {
@@ -183,7 +283,7 @@ size_t lora_workspace_size(int op, int32_t N, int32_t n_adapters, int32_t d_in, 
     if (op == LORA_OP_MERGE)
         return n_adapters >= 1 && n_adapters <= LORA_MAX_ADAPTERS && N == d_out
                    ? merge_workspace_size(d_in, d_out, max_rank) : 0;
-    if (op < LORA_OP_BGMV || op > LORA_OP_LINEAR || op == LORA_OP_MERGE)
+    if (op < LORA_OP_BGMV || op > LORA_OP_APPLY_PROJ || op == LORA_OP_MERGE)
         return 0;
     Layout L;
     if (!layout(op, N, n_adapters, d_in, max_rank, n_items, max_ads_per_req, &L))
@@ -444,19 +544,9 @@ lora_status lora_sgmv_shrink_proj(const void *X, int64_t ldx, float *V, int64_t 
                                   const int32_t *seg_ad, int32_t n_seg, int32_t N,
                                   void *ws, size_t ws_bytes, void *stream)
 {
-    if (!pools || n_proj < 1)
-        return LORA_ERR_INVALID_ARG;
-    if (n_proj > LORA_MAX_PROJ)
-        return LORA_ERR_UNSUPPORTED;
     int32_t vcol[LORA_MAX_PROJ];
     int64_t vcols = 0;
-    for (int p = 0; p < n_proj; ++p) {
-        LORA_TRY(check_pool(&pools[p]));
-        if (pools[p].d_in != pools[0].d_in || pools[p].n_adapters != pools[0].n_adapters)
-            return LORA_ERR_INVALID_ARG;
-        vcol[p] = (int32_t)vcols;
-        vcols += pools[p].max_rank;
-    }
+    LORA_TRY(check_proj_pools(pools, n_proj, vcol, &vcols));
     const int32_t d_in = pools[0].d_in;
     if (N < 0 || n_seg < 0 || !seg_off || (n_seg > 0 && !seg_ad))
         return LORA_ERR_INVALID_ARG;
@@ -469,75 +559,88 @@ lora_status lora_sgmv_shrink_proj(const void *X, int64_t ldx, float *V, int64_t 
     LORA_TRY(check_ws(ws, ws_bytes, L));
     if (N == 0 || n_seg == 0)
         return LORA_OK;
+    TcArgs ta = {};
+    const bool tc = long_items(N, n_seg) && aligned_v(V, ldv) && tc_encode_x(ta, X, N, d_in, ldx);
+    LORA_CUDA(run_proj_shrinks(tc, ta, X, ldx, V, ldv, pools, n_proj, vcol, seg_off, seg_ad, n_seg, N, L, ws,
+                               (cudaStream_t)stream));
+    return LORA_OK;
+}
+
+lora_status lora_sgmv_apply_proj(const void *X, int64_t ldx, void *const *Y, const int64_t *ldy,
+                                 const lora_pool *pools, int32_t n_proj, const int32_t *seg_off,
+                                 const int32_t *seg_ad, int32_t n_seg, int32_t N, const float *scale,
+                                 void *ws, size_t ws_bytes, void *stream)
+{
+    int32_t vcol[LORA_MAX_PROJ];
+    int64_t vcols = 0;
+    LORA_TRY(check_proj_pools(pools, n_proj, vcol, &vcols));
+    if (!Y || !ldy || !scale)
+        return LORA_ERR_INVALID_ARG;
+    const int32_t d_in = pools[0].d_in;
+    if (N < 0 || n_seg < 0 || !seg_off || (n_seg > 0 && !seg_ad))
+        return LORA_ERR_INVALID_ARG;
+    LORA_TRY(check_mat(X, ldx, d_in, N));
+    for (int p = 0; p < n_proj; ++p)
+        LORA_TRY(check_mat(Y[p], ldy[p], pools[p].d_out, N));
+    Layout L;
+    if (!layout(LORA_OP_APPLY_PROJ, N, pools[0].n_adapters, d_in, (int32_t)vcols, n_seg, 1, &L))
+        return LORA_ERR_INVALID_ARG;
+    LORA_TRY(check_ws(ws, ws_bytes, L));
+    if (N == 0 || n_seg == 0)
+        return LORA_OK;
     cudaStream_t s = (cudaStream_t)stream;
     WsHeader *hdr = at<WsHeader>(ws, L.hdr);
     Group *groups = at<Group>(ws, L.groups);
+    float *V = at<float>(ws, L.V);
+    const int64_t ldv = vcols;
 
-    PlanArgs pa = {};
-    pa.mode = kModeSgmv;
-    pa.N = N;
-    pa.item_off = seg_off;
-    pa.n_items = n_seg;
-    pa.groups = groups;
-    pa.max_groups = L.max_groups;
-    pa.hdr = hdr;
-    if (long_items(N, n_seg) && aligned_v(V, ldv)) {
-        TcArgs ta = {};
-        if (tc_encode_x(ta, X, N, d_in, ldx)) {
-            pa.group = kTcGroup;
-            LORA_CUDA(launch_plan(pa, s));
-            ta.mode = kModeProj;
-            ta.groups = groups;
-            ta.hdr = hdr;
-            ta.seg_ad = seg_ad;
-            ta.max_ads = 1;
-            ta.scale = 1.0f;
-            ta.V = V;
-            ta.ldv = ldv;
-            ta.slot_stride = 0;
-            ta.err = &hdr->err;
-            // one launch per run of consecutive projections whose max_ranks fit
-            // one stacked accumulator: every launch reads X once
-            for (int p0 = 0; p0 < n_proj;) {
-                int p1 = p0, kk = 0;
-                while (p1 < n_proj && kk + pools[p1].max_rank <= kKMaxShrink)
-                    kk += pools[p1++].max_rank;
-                TcArgs tp = ta;
-                tp.a_tma = 0;
-                tp.n_proj = p1 - p0;
-                for (int q = p0; q < p1; ++q) {
-                    tp.proj[q - p0] = pool_dev(&pools[q]);
-                    tp.proj_vcol[q - p0] = vcol[q];
-                    tc_encode_a(tp, pools[q].A, pools[q].A_elems, d_in, q - p0);
-                }
-                tp.pool = tp.proj[0];
-                LORA_CUDA(launch_tc_shrink(tp, N / kTcGroup + n_seg + 1, kk, s));
-                p0 = p1;
-            }
-            return LORA_OK;
-        }
+    // every tensor map is built before the first launch: the path is chosen once
+    TcArgs ta = {};
+    TcArgs te[LORA_MAX_PROJ];
+    bool tc = long_items(N, n_seg) && tc_encode_x(ta, X, N, d_in, ldx);
+    for (int p = 0; p < n_proj && tc; ++p) {
+        te[p] = TcArgs{};
+        tc_encode_b(te[p], pools[p].B, pools[p].B_elems);
+        tc = tc_encode_y(te[p], Y[p], N, pools[p].d_out, ldy[p]);
     }
-
-    // short segments: the CUDA-core shrink, once per projection
-    pa.group = kGroup;
-    LORA_CUDA(launch_plan(pa, s));
+    LORA_CUDA(run_proj_shrinks(tc, ta, X, ldx, V, ldv, pools, n_proj, vcol, seg_off, seg_ad, n_seg, N, L, ws, s));
     for (int p = 0; p < n_proj; ++p) {
-        ShrinkArgs sa = {};
-        sa.X = static_cast<const __nv_bfloat16 *>(X);
-        sa.ldx = ldx;
-        sa.perm = nullptr;
-        sa.groups = groups;
-        sa.hdr = hdr;
-        sa.mode = kModeSgmv;
-        sa.seg_ad = seg_ad;
-        sa.pool = pool_dev(&pools[p]);
-        sa.kc = d_in;
-        sa.V = V + vcol[p];
-        sa.ldv = ldv;
-        sa.chunk_stride = 0;
-        sa.slot_stride = 0;
-        sa.err = &hdr->err;
-        LORA_CUDA(launch_shrink(sa, L.max_groups, 1, 1, s));
+        if (tc) {
+            TcArgs &e = te[p];
+            e.mode = kModeSgmv;
+            e.groups = groups;
+            e.hdr = hdr;
+            e.seg_ad = seg_ad;
+            e.max_ads = 1;
+            e.scale = scale[p];
+            e.pool = pool_dev(&pools[p]);
+            e.V = V + vcol[p];
+            e.ldv = ldv;
+            e.slot_stride = 0;
+            e.Y = static_cast<__nv_bfloat16 *>(Y[p]);
+            e.ldy = ldy[p];
+            e.err = &hdr->err;
+            LORA_CUDA(launch_tc_expand(e, pools[p].max_rank, s));
+        } else {
+            ExpandArgs ea = {};
+            ea.Y = static_cast<__nv_bfloat16 *>(Y[p]);
+            ea.ldy = ldy[p];
+            ea.perm = nullptr;
+            ea.groups = groups;
+            ea.hdr = hdr;
+            ea.mode = kModeSgmv;
+            ea.seg_ad = seg_ad;
+            ea.scale = scale[p];
+            ea.pool = pool_dev(&pools[p]);
+            ea.V = V + vcol[p];
+            ea.ldv = ldv;
+            ea.chunk_stride = 0;
+            ea.n_chunks = 1;
+            ea.slot_stride = 0;
+            ea.max_ads = 1;
+            ea.err = &hdr->err;
+            LORA_CUDA(launch_expand(ea, L.max_groups, s));
+        }
     }
     return LORA_OK;
 }

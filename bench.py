@@ -255,11 +255,8 @@ def shrink_proj_passes(max_ranks, limit=256) -> int:
 def launches_per_step(wl) -> int:
     import adapter_gemv_sgmv_b200 as L
     if wl.desc.get("op") == "sgmv_proj":
-        c0 = wl.calls[0]
-        n = len(c0.seg_ad_h)
-        expands = sum(L.lora_kernel_launches(L.OP_SGMV_EXPAND, c.n_tokens, c.pool.n_adapters, c.pool.d_in, n)
-                      for c in wl.calls)
-        return 1 + shrink_proj_passes([c.pool.max_rank for c in wl.calls]) + expands
+        # lora_sgmv_apply_proj on long segments: one plan, the stacked shrinks, one expand each
+        return 1 + shrink_proj_passes([c.pool.max_rank for c in wl.calls]) + len(wl.calls)
     return sum(launches_per_call(c) for c in wl.calls)
 
 
@@ -269,17 +266,18 @@ def make_step(wl, ws_map, stream):
     import adapter_gemv_sgmv_b200 as L
     fns = []
     if wl.desc.get("op") == "sgmv_proj":
-        # projections sharing X: one shrink over all of them, then each projection's expand
+        # projections sharing X: one call -- one plan, one stacked shrink over all of them
+        # (x read once), then each projection's expand; V stays in the workspace
         c0 = wl.calls[0]
         pools = [c.pool for c in wl.calls]
-        V = torch.empty(c0.X.shape[0], sum(p.max_rank for p in pools), dtype=torch.float32, device=c0.X.device)
-        cols = np.cumsum([0] + [p.max_rank for p in pools])[:-1].tolist()
+        need = L.lora_workspace_size(L.OP_APPLY_PROJ, c0.n_tokens, c0.pool.n_adapters, c0.pool.d_in, 0,
+                                     sum(p.max_rank for p in pools), len(c0.seg_ad_h))
+        ws = ws_map.setdefault(("apply_proj", id(wl)), L.Workspace(need, device=c0.X.device))
+        Ys = [c.Y for c in wl.calls]
+        scales = [c.scale for c in wl.calls]
 
         def proj_step():
-            L.lora_sgmv_shrink_proj(c0.X, V, pools, c0.seg_off, c0.seg_ad, ws=ws_map[id(c0)], stream=stream)
-            for c, col in zip(wl.calls, cols):
-                L.lora_sgmv_expand(V[:, col:], c.Y, c.pool, c.seg_off, c.seg_ad, c.scale, ws=ws_map[id(c)],
-                                   stream=stream)
+            L.lora_sgmv_apply_proj(c0.X, Ys, pools, c0.seg_off, c0.seg_ad, scales, ws=ws, stream=stream)
         return proj_step
     for c in wl.calls:
         ws = ws_map[id(c)]
@@ -377,11 +375,10 @@ def run_ours(args):
         for i in range(max(args.warmup, 3)):
             steps[i % n_sets]()
     stream.synchronize()
-    for wl in sets:
-        for c in wl.calls:
-            err = L.lora_get_error(ws_map[id(c)], stream=stream)
-            if err:
-                raise SystemExit(f"device error {err} during warm-up")
+    for ws in ws_map.values():
+        err = L.lora_get_error(ws, stream=stream)
+        if err:
+            raise SystemExit(f"device error {err} during warm-up")
 
     # one graph = one pass over every input set
     g = torch.cuda.CUDAGraph()

@@ -79,7 +79,7 @@ extern "C" {
 #define LORA_MAX_RANK 128
 #define LORA_MAX_ADAPTERS 32768
 #define LORA_MAX_ADS_PER_REQ 8
-#define LORA_MAX_PROJ 4          /* projections sharing one input in lora_sgmv_shrink_proj */
+#define LORA_MAX_PROJ 4          /* projections sharing one input (lora_sgmv_shrink_proj, _apply_proj) */
 
 /* Status codes.  Host-side codes are returned directly; device-side codes are
  * bits of the workspace error word returned by lora_get_error (OR-ed). */
@@ -119,7 +119,8 @@ typedef enum {
     LORA_OP_APPLY_MULTI = 3,
     LORA_OP_ROUTE = 4,
     LORA_OP_MERGE = 5,
-    LORA_OP_LINEAR = 6
+    LORA_OP_LINEAR = 6,
+    LORA_OP_APPLY_PROJ = 7      /* max_rank = the projections' max_rank summed */
 } lora_op;
 
 /* Bytes of workspace `op` needs for N token rows.  n_items = n_seg for the
@@ -132,7 +133,9 @@ LORA_API size_t lora_workspace_size(int op, int32_t N, int32_t n_adapters, int32
 
 /* Number of kernels one call of `op` launches for these sizes (pure host
  * function): lets a caller budget a CUDA graph or count launches.  0 for
- * arguments the entry point would reject or that launch nothing (N == 0). */
+ * arguments the entry point would reject or that launch nothing (N == 0), and
+ * for LORA_OP_APPLY_PROJ, whose count depends on the pools (see
+ * lora_sgmv_apply_proj). */
 LORA_API int lora_kernel_launches(int op, int32_t N, int32_t n_adapters, int32_t d_in, int32_t n_items);
 
 /* Clear the workspace's error word (cudaMemsetAsync of its 256-byte header on
@@ -214,6 +217,23 @@ LORA_API lora_status lora_sgmv_shrink(const void *X, int64_t ldx, float *V, int6
 LORA_API lora_status lora_sgmv_shrink_proj(const void *X, int64_t ldx, float *V, int64_t ldv,
                              const lora_pool *pools, int32_t n_proj, const int32_t *seg_off,
                              const int32_t *seg_ad, int32_t n_seg, int32_t N,
+                             void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * lora_sgmv_apply_proj -- the whole delta of projections that share their input
+ * (the shrink of lora_sgmv_shrink_proj, then every projection's expand):
+ *   Y_p[n] += scale[p] * B_p[a] (A_p[a] X[n]),  a = seg_ad[k], seg_off[k] <= n < seg_off[k+1],
+ * for p < n_proj.  One plan serves the shrink and all the expands, and the
+ * intermediate stays in the workspace: 1 + (tensor-core shrink launches) +
+ * n_proj kernels on the tensor-core path (long segments), 1 + 2 n_proj on the
+ * CUDA-core path.  Y, ldy, scale: HOST arrays of n_proj entries (Y[p] a device
+ * bf16 [N, ldy[p]] matrix, ldy[p] >= pools[p].d_out).  Pools and segments as
+ * in lora_sgmv_shrink_proj.  Workspace: lora_workspace_size(LORA_OP_APPLY_PROJ,
+ * N, n_adapters, d_in, 0, sum of the pools' max_rank, n_seg, 0).
+ */
+LORA_API lora_status lora_sgmv_apply_proj(const void *X, int64_t ldx, void *const *Y, const int64_t *ldy,
+                             const lora_pool *pools, int32_t n_proj, const int32_t *seg_off,
+                             const int32_t *seg_ad, int32_t n_seg, int32_t N, const float *scale,
                              void *ws, size_t ws_bytes, void *stream);
 
 /*

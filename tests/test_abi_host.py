@@ -37,7 +37,7 @@ def test_header_declares_the_entry_points():
     names = set(declared())
     assert {"lora_bgmv", "lora_sgmv_shrink", "lora_sgmv_expand", "lora_apply_multi", "lora_route",
             "lora_workspace_size", "lora_workspace_init", "lora_get_error", "lora_version",
-            "lora_merge", "lora_sgmv_shrink_proj", "lora_linear_sgmv"} <= names
+            "lora_merge", "lora_sgmv_shrink_proj", "lora_linear_sgmv", "lora_sgmv_apply_proj"} <= names
 
 
 def test_every_declared_symbol_is_exported(lib):
@@ -206,3 +206,30 @@ def test_empty_calls_return_before_any_launch(lib):
     pools = _pools(_pool(), _pool(max_rank=32))
     assert lib.lora_sgmv_shrink_proj(FAKE, 64, FAKE, 48, pools, 2, FAKE, FAKE, 2, 0, ws, nb, None) == OK
     assert lib.lora_sgmv_shrink_proj(FAKE, 64, FAKE, 48, pools, 2, FAKE, FAKE, 0, 4, ws, nb, None) == OK
+
+
+def test_apply_proj_validates(lib):
+    q, k = _pool(), _pool(d_out=16, max_rank=8)
+    two = _pools(q, k)
+    ap = lib.lora_sgmv_apply_proj
+    ys = (ctypes.c_void_p * 2)(FAKE, FAKE)
+    lds = (ctypes.c_int64 * 2)(32, 16)
+    sc = (ctypes.c_float * 2)(1.0, 0.5)
+    # host arrays missing
+    assert ap(FAKE, 64, None, lds, two, 2, FAKE, FAKE, 2, 4, sc, None, 0, None) == INVALID
+    assert ap(FAKE, 64, ys, None, two, 2, FAKE, FAKE, 2, 4, sc, None, 0, None) == INVALID
+    assert ap(FAKE, 64, ys, lds, two, 2, FAKE, FAKE, 2, 4, None, None, 0, None) == INVALID
+    # a projection's leading dimension below its d_out; a misaligned output
+    bad_ld = (ctypes.c_int64 * 2)(32, 8)
+    assert ap(FAKE, 64, ys, bad_ld, two, 2, FAKE, FAKE, 2, 4, sc, None, 0, None) == INVALID
+    bad_y = (ctypes.c_void_p * 2)(FAKE, FAKE + 2)
+    assert ap(FAKE, 64, bad_y, lds, two, 2, FAKE, FAKE, 2, 4, sc, None, 0, None) == UNSUPPORTED
+    # pools that do not share d_in
+    assert ap(FAKE, 64, ys, lds, _pools(q, _pool(d_in=128, d_out=16)), 2, FAKE, FAKE, 2, 4, sc, None, 0,
+              None) == INVALID
+    assert ap(FAKE, 64, ys, lds, two, 2, FAKE, FAKE, 2, 4, sc, None, 0, None) == WORKSPACE
+    # empty: validated, then nothing launched
+    assert ap(FAKE, 64, ys, lds, two, 2, FAKE, FAKE, 2, 0, sc, FAKE, 1 << 20, None) == OK
+    # the workspace holds V for all projections side by side (16 + 8 columns)
+    assert L.lora_workspace_size(L.OP_APPLY_PROJ, 1000, 4, 64, 0, 24, 2) >= 1000 * 24 * 4
+    assert L.lora_workspace_size(L.OP_APPLY_PROJ, 1000, 4, 64, 0, 4 * 128 + 8, 2) == 0

@@ -149,8 +149,8 @@ def test_prefill_qkv_full_size_sampled_rows():
     ws_map = {id(c): bench.workspace_for(c) for c in wl.calls}
     stream = torch.cuda.current_stream()
     bench.make_step(wl, ws_map, stream)()
-    for c in wl.calls:
-        assert L.lora_get_error(ws_map[id(c)]) == 0
+    for ws in ws_map.values():
+        assert L.lora_get_error(ws) == 0
     c0 = wl.calls[0]
     N = c0.X.shape[0]
     rng = np.random.default_rng(1)
@@ -171,3 +171,25 @@ def test_shrink_proj_only_empty_segments_writes_nothing():
     ws, _ = L.lora_sgmv_shrink_proj(dev_bf16(X), V, [DevPool(hp) for hp in hps], _i32([0, 0, 0]), _i32([0, 1]))
     assert L.lora_get_error(ws) == 0
     assert torch.isnan(V).all()
+
+
+@pytest.mark.parametrize("long", [True, False])
+@pytest.mark.parametrize("case", ["qkv_r64", "qkv_r128", "four_r16"])
+def test_apply_proj_every_output(case, long):
+    """One call for the whole delta of projections sharing X: each projection's y against
+    the oracle's delta, with its own scale; rows outside every segment untouched."""
+    rng = np.random.default_rng(len(case) * 11 + long)
+    d_in = 328
+    hps = [rand_host_pool(rng, ranks, d_in, d_out) for d_out, ranks in CASES[case]]
+    seg_off, ads, N = _segments(long)
+    X = rand_x(rng, N, d_in)
+    Y0 = [rand_x(rng, N, hp.d_out) for hp in hps]
+    Ys = [dev_bf16(y) for y in Y0]
+    scales = [0.5 + 0.25 * p for p in range(len(hps))]
+    ws = L.lora_sgmv_apply_proj(dev_bf16(X), Ys, [DevPool(hp) for hp in hps], _i32(seg_off), _i32(ads), scales)
+    assert L.lora_get_error(ws) == 0
+    outside = np.r_[0:seg_off[0], seg_off[-1]:N]
+    for p, (hp, y0, Y) in enumerate(zip(hps, Y0, Ys)):
+        got = widen(to_host(Y))
+        check_parity(got, widen(y0) + oracle.sgmv_delta(X, hp, seg_off, ads, scales[p]), f"apply {case} p{p}")
+        assert np.array_equal(got[outside], widen(y0)[outside])
