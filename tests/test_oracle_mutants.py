@@ -31,6 +31,8 @@ MUTANTS = {
                               "acc += widen_bf16(W[(int64_t)o * ldw + (d_in - 1 - i)]) * widen_bf16(x[i]);"),
     "linear_dropped_base": ("            y_row[o] = acc;\n        }\n        if (seg_ad[sg] == -1)",
                             "            y_row[o] = 0.0 * acc;\n        }\n        if (seg_ad[sg] == -1)"),
+    "linear_dropped_delta": ("        if (seg_ad[sg] == -1)\n            continue;\n        int rc = one_adapter(x,",
+                             "        if (seg_ad[sg] != -3)\n            continue;\n        int rc = one_adapter(x,"),
     "linear_none_gets_delta": ("        if (seg_ad[sg] == -1)\n            continue;\n        int rc = one_adapter(x,",
                                "        if (seg_ad[sg] == -2)\n            continue;\n        int rc = one_adapter(x,"),
     "dropped_last_adapter": ("for (int32_t p = ad_off[q]; p < ad_off[q + 1]; ++p)",
