@@ -11,7 +11,7 @@ import torch
 
 import adapter_gemv_sgmv_b200 as L
 import oracle
-from helpers import DevPool, check_parity, dev_bf16, rand_host_pool, rand_x, widen
+from helpers import DevPool, check_parity, check_rounded, dev_bf16, rand_host_pool, rand_x, widen
 from workloads import bf16_bits, to_host
 
 pytestmark = pytest.mark.gpu
@@ -47,6 +47,7 @@ def test_linear_ragged(d_in, d_out):
     inside = np.r_[seg_off[0]:seg_off[-1]]
     want = oracle.linear_sgmv(X, W, hp, seg_off, np.array(ads, np.int32), 0.75)
     check_parity(got[inside], want[inside], f"linear {d_in}x{d_out}")
+    check_rounded(got[inside], want[inside], f"linear {d_in}x{d_out}")
     outside = np.r_[0:start, seg_off[-1]:N]
     assert np.all(got[outside] == 1.0)
 
@@ -101,6 +102,7 @@ def test_prefill_linear_full_size_sampled_rows():
     want = oracle.linear_sgmv(to_host(c.X), to_host(c.W), host_pool(c.pool), c.seg_off_h, c.seg_ad_h, c.scale,
                               rows=rows)
     check_parity(widen(to_host(c.Y))[rows], want, "prefill_linear_up")
+    check_rounded(widen(to_host(c.Y))[rows], want, "prefill_linear_up")
 
 
 def test_linear_degenerate_segments():

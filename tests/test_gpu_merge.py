@@ -11,7 +11,7 @@ import torch
 
 import adapter_gemv_sgmv_b200 as L
 import oracle
-from helpers import DevPool, dev_bf16, rand_host_pool, rand_x, scatter_pool, widen
+from helpers import DevPool, dev_bf16, half_ulp_bf16, rand_host_pool, rand_x, scatter_pool, widen
 from workloads import make_workload, to_host
 
 pytestmark = pytest.mark.gpu
@@ -24,7 +24,7 @@ def _check_merge(got, exact, what):
     got = np.asarray(got, np.float64)
     exact = np.asarray(exact, np.float64)
     rnd = oracle.round_bf16(exact)
-    bound = 2.0 ** -8 * np.abs(exact) + 1e-4 * (np.sqrt(np.mean(exact ** 2)) + 1e-30)
+    bound = half_ulp_bf16(exact) + 1e-4 * (np.sqrt(np.mean(exact ** 2)) + 1e-30)
     bad = np.abs(got - exact) > bound
     assert not bad.any(), f"{what}: {int(bad.sum())} elements off, worst {np.max(np.abs(got - exact)):.3e}"
     frac = float(np.mean(got == rnd))

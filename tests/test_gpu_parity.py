@@ -3,13 +3,13 @@
 Every call goes through liblora_sgmv.so via the ctypes binding; the oracle
 runs on the host on the same seeded inputs.  The bar (elementwise, against
 the oracle's exact fp64 value y_exact):
-    |y_gpu - y_exact| <= 1e-2 * rms(y_exact) + 1e-3 + 2**-8 * |y_exact|
-(the stated tolerance plus the unit roundoff of the one bf16 rounding of the
-stored output; see helpers.check_parity).  The shrink's fp32 V is held to
-1e-2 * rms + 1e-3 against the oracle's fp64 V.  The decode path, which keeps
-the rank-r intermediate in fp32, must in addition give the correctly rounded
-bf16 of y_exact for at least 99% of the outputs.  Full-size workloads are checked on sampled rows (segment
-boundaries always included); the small ones on every row.
+    |y_gpu - y_exact| <= 1e-2 * rms(y_exact) + 1e-3 + half a bf16 ulp of y_exact
+(the stated tolerance plus the one bf16 rounding of the stored output; see
+helpers.check_parity).  The shrink's fp32 V is held to 1e-2 * rms + 1e-3
+against the oracle's fp64 V.  Every path carries the rank-r intermediate to
+fp32 precision, so each must in addition give the correctly rounded bf16 of
+y_exact for at least 99% of the outputs.  Full-size workloads are checked on
+sampled rows (segment boundaries always included); the small ones on every row.
 """
 import numpy as np
 import pytest
@@ -17,7 +17,8 @@ import torch
 
 import adapter_gemv_sgmv_b200 as L
 import oracle
-from helpers import (check_close_f32, check_parity, compact_from_device_pool, host_pool, widen)
+from helpers import (check_close_f32, check_parity, check_rounded, compact_from_device_pool, host_pool,
+                     widen)
 from workloads import make_workload, to_host
 
 pytestmark = pytest.mark.gpu
@@ -73,6 +74,7 @@ def test_tiny_sgmv_every_row(y0):
     check_close_f32(Vh[m], Vref[m], "tiny shrink V")
     y_exact = _f64(c.Y) + oracle.sgmv_delta(X, hp, c.seg_off_h, c.seg_ad_h, c.scale)
     check_parity(Yh, y_exact, f"tiny sgmv y0={y0}")
+    check_rounded(Yh, y_exact, f"tiny sgmv y0={y0}")
     # the expand alone, fed the GPU's own fp32 V, against the oracle's expand of that V
     Y2 = c.Y.clone()
     V32 = torch.tensor(np.nan_to_num(Vh).astype(np.float32), device=DEV)
@@ -92,7 +94,7 @@ def test_decode_bgmv_full(y0):
     y_exact = _f64(c.Y) + oracle.bgmv_delta(to_host(c.X), hp, c.ids_h, c.scale)
     got = _f64(Y)
     check_parity(got, y_exact, f"decode bgmv y0={y0}")
-    assert np.mean(got == oracle.round_bf16(y_exact)) >= 0.99
+    check_rounded(got, y_exact, f"decode bgmv y0={y0}")
 
 
 def test_prefill_sgmv_full_size_sampled_rows():
@@ -107,6 +109,7 @@ def test_prefill_sgmv_full_size_sampled_rows():
     check_close_f32(Vh, Vref, "prefill shrink V")
     y_exact = _f64(c.Y)[rows] + oracle.sgmv_delta(X, hp, c.seg_off_h, c.seg_ad_h, c.scale, rows=rows)
     check_parity(Yh, y_exact, "prefill sgmv")
+    check_rounded(Yh, y_exact, "prefill sgmv")
 
 
 def test_mixed_rank_layer_every_row():
@@ -119,6 +122,7 @@ def test_mixed_rank_layer_every_row():
         ids = np.where(c.ids_h >= 0, remap[np.maximum(c.ids_h, 0)], -1).astype(np.int32)
         y_exact = _f64(c.Y) + oracle.bgmv_delta(to_host(c.X), hp, ids, c.scale)
         check_parity(_f64(Y), y_exact, f"mixed-rank layer {c.name}")
+        check_rounded(_f64(Y), y_exact, f"mixed-rank layer {c.name}")
         del Y
     del wl
     torch.cuda.empty_cache()
@@ -135,3 +139,4 @@ def test_diffusion_multi_sampled_rows():
         d = oracle.apply_multi_delta(to_host(c.X), hp, c.req_off_h, c.ad_off_h, c.ad_id_h, c.ad_scale_h,
                                      rows=rows)
         check_parity(_f64(Y)[rows], _f64(c.Y)[rows] + d, f"diffusion multi {c.name}")
+        check_rounded(_f64(Y)[rows], _f64(c.Y)[rows] + d, f"diffusion multi {c.name}")

@@ -11,7 +11,7 @@ import torch
 
 import adapter_gemv_sgmv_b200 as L
 import oracle
-from helpers import (DevPool, check_close_f32, check_parity, dev_bf16, rand_host_pool, rand_x,
+from helpers import (DevPool, check_close_f32, check_parity, check_rounded, dev_bf16, rand_host_pool, rand_x,
                      scatter_pool, widen)
 from workloads import to_host
 
@@ -160,6 +160,7 @@ def test_prefill_qkv_full_size_sampled_rows():
         hp = host_pool(c.pool)
         y_exact = widen(y0)[rows] + oracle.sgmv_delta(X, hp, c.seg_off_h, c.seg_ad_h, c.scale, rows=rows)
         check_parity(widen(to_host(c.Y))[rows], y_exact, f"prefill_qkv {c.name}")
+        check_rounded(widen(to_host(c.Y))[rows], y_exact, f"prefill_qkv {c.name}")
 
 
 def test_shrink_proj_only_empty_segments_writes_nothing():
@@ -191,5 +192,7 @@ def test_apply_proj_every_output(case, long):
     outside = np.r_[0:seg_off[0], seg_off[-1]:N]
     for p, (hp, y0, Y) in enumerate(zip(hps, Y0, Ys)):
         got = widen(to_host(Y))
-        check_parity(got, widen(y0) + oracle.sgmv_delta(X, hp, seg_off, ads, scales[p]), f"apply {case} p{p}")
+        want = widen(y0) + oracle.sgmv_delta(X, hp, seg_off, ads, scales[p])
+        check_parity(got, want, f"apply {case} p{p}")
+        check_rounded(got, want, f"apply {case} p{p}")
         assert np.array_equal(got[outside], widen(y0)[outside])

@@ -10,7 +10,7 @@ import torch
 
 import adapter_gemv_sgmv_b200 as L
 import oracle
-from helpers import (DevPool, check_close_f32, check_parity, dev_bf16, rand_host_pool, rand_x,
+from helpers import (DevPool, check_close_f32, check_parity, check_rounded, dev_bf16, rand_host_pool, rand_x,
                      scatter_pool, widen)
 from workloads import to_host
 
@@ -54,6 +54,7 @@ def test_tc_sgmv_ragged(d_in, d_out, packed):
     assert L.lora_get_error(ws) == 0
     got = widen(to_host(Y))
     check_parity(got, widen(Y0) + oracle.sgmv_delta(X, hp, seg_off, ads, 1.25), "tc sgmv")
+    check_rounded(got, widen(Y0) + oracle.sgmv_delta(X, hp, seg_off, ads, 1.25), "tc sgmv")
     outside = np.r_[0:start, seg_off[-1]:N]
     assert np.array_equal(got[outside], widen(Y0)[outside])
 
@@ -82,6 +83,7 @@ def test_tc_multi_stacked_adapters(packed):
     assert L.lora_get_error(ws) == 0
     got = widen(to_host(Y))
     check_parity(got, widen(Y0) + oracle.apply_multi_delta(X, hp, req_off, ad_off, ad_id, ad_sc), "tc multi")
+    check_rounded(got, widen(Y0) + oracle.apply_multi_delta(X, hp, req_off, ad_off, ad_id, ad_sc), "tc multi")
     untouched = np.r_[req_off[1]:req_off[2], req_off[-1]:N, req_off[3]:req_off[3]]   # empty list, outside
     assert np.array_equal(got[req_off[2]:req_off[3]], widen(Y0)[req_off[2]:req_off[3]])  # request with no adapters
     assert np.array_equal(got[untouched], widen(Y0)[untouched])

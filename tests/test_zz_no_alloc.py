@@ -11,7 +11,8 @@ import pytest
 import torch
 
 import adapter_gemv_sgmv_b200 as L
-from helpers import check_parity, widen
+import oracle
+from helpers import check_parity, check_rounded, host_pool, widen
 from workloads import make_pool, make_workload, to_host
 
 pytestmark = pytest.mark.gpu
@@ -22,23 +23,28 @@ def _case(seed):
                          projections=["q"], y0="normal").calls[0]
 
 
-def test_static_scratch_matches_the_workspace_entry_point_on_two_calls():
-    for seed in (11, 12):   # two calls in a row on the same fixed scratch
+def test_static_scratch_matches_the_oracle_on_two_calls():
+    """Two calls in a row on the one fixed scratch, each against the oracle's exact
+    multi-adapter delta (the bar every parity test uses), and against what
+    lora_apply_multi gives with a caller workspace on the same inputs."""
+    for seed in (11, 12):
         c = _case(seed)
-        y_ref = c.Y.clone()
-        ws = L.lora_apply_multi(c.X, y_ref, c.pool, c.req_off, c.ad_off, c.ad_id, c.ad_scale, max_ads_per_req=3)
-        assert L.lora_get_error(ws) == 0
         y = c.Y.clone()
         err = torch.full((1,), -1, dtype=torch.int32, device="cuda")
         L.lora_apply_multi_static(c.X, y, c.pool, c.req_off, c.ad_off, c.ad_id, c.ad_scale, max_ads_per_req=3,
                                   err_out=err)
         torch.cuda.synchronize()
         assert int(err.item()) == 0
-        got, want = widen(to_host(y)), widen(to_host(y_ref))
-        # both sides are bf16 results (the workspace entry point may take the tensor-core
-        # path, whose rank-r intermediate is bf16), so both roundings are allowed for
-        check_parity(got, want, f"static scratch vs workspace, call seed {seed}", ref_rounded=True)
-        assert np.max(np.abs(want - widen(to_host(c.Y)))) > 0   # the call did change y
+        y_exact = widen(to_host(c.Y)) + oracle.apply_multi_delta(to_host(c.X), host_pool(c.pool), c.req_off_h,
+                                                                 c.ad_off_h, c.ad_id_h, c.ad_scale_h)
+        got = widen(to_host(y))
+        check_parity(got, y_exact, f"static scratch, call seed {seed}")
+        check_rounded(got, y_exact, f"static scratch, call seed {seed}")
+        assert np.max(np.abs(got - widen(to_host(c.Y)))) > 0   # the call did change y
+        y_ws = c.Y.clone()
+        ws = L.lora_apply_multi(c.X, y_ws, c.pool, c.req_off, c.ad_off, c.ad_id, c.ad_scale, max_ads_per_req=3)
+        assert L.lora_get_error(ws) == 0
+        check_parity(widen(to_host(y_ws)), y_exact, f"workspace entry point, call seed {seed}")
 
 
 def test_static_scratch_rejects_calls_that_do_not_fit():
