@@ -23,17 +23,6 @@ import numpy as np
 BF16_BYTES = 2
 
 
-def lora_costs(d_model: int, layers: int, adapted_per_layer: int, rank: int, n_tokens: int,
-               hbm_gbps: float = 3350.0, dtype: int = 2):
-    """The handbook's cost model: (extra FLOP fraction, merge ms, LoRA size in MiB)."""
-    base_flops = 2 * n_tokens * d_model * d_model * adapted_per_layer * layers
-    lora = lora_flops(n_tokens, rank, d_model, d_model) * adapted_per_layer * layers
-    weight_bytes = d_model * d_model * dtype * adapted_per_layer * layers
-    merge_ms = merge_bytes(weight_bytes) / (hbm_gbps * 1e9) * 1e3
-    lora_mb = adapter_elems(rank, d_model, d_model) * dtype * adapted_per_layer * layers / 2 ** 20
-    return lora / base_flops, merge_ms, lora_mb
-
-
 def lora_flops(n_tokens: int, rank: int, d_in: int, d_out: int) -> int:
     """Shrink (2*N*d_in*r) plus expand (2*N*r*d_out)."""
     return 2 * int(n_tokens) * int(rank) * (int(d_in) + int(d_out))

@@ -1,10 +1,10 @@
 // Grouping of a batch by adapter and construction of the work-group list.
 //
-// "Serving several LoRAs, ControlNet and IP-Adapter", exercise 2's answer:
-// group the batch's activations by LoRA index, let one kernel handle every
-// group, and add the results back in the original order.  For an unsorted
-// decode batch this is a stable counting sort of the adapter ids (histogram
-// -> exclusive scan -> stable scatter).  Prefill segments and multi-adapter
+// "Serving several LoRAs, ControlNet and IP-Adapter", exercise 2's answer: a
+// stable counting sort of the tokens by adapter id, one kernel over all the
+// resulting runs, and the results scattered back to token order.  For an
+// unsorted decode batch the sort is histogram -> exclusive scan -> stable
+// scatter.  Prefill segments and multi-adapter
 // requests arrive already grouped; the plan kernel only validates their
 // offsets.  In every mode it then cuts each item (segment / request) into
 // work groups of at most `group` tokens.

@@ -10,9 +10,9 @@ IP-Adapter", section "LoRA: merged or alongside", unless stated):
 * W' = W + BA with A r x d, B d x r; unmerged each layer adds x A^T B^T
   to x W^T  -> dense special case, merged-weight identity, zero B.
 * the LoRA weight is a runtime scalar swapped per step -> linearity in s.
-* exercise 2's answer: group by LoRA index, one kernel for all groups, add
-  back in the original order; two requests on one LoRA fall in one group
-  -> permutation invariance, segment-split independence, SGMV == BGMV,
+* exercise 2's answer (tokens sorted stably by adapter, one kernel over all
+  runs, results returned in token order; tokens sharing an adapter share a
+  run) -> permutation invariance, segment-split independence, SGMV == BGMV,
   the stable grouping (route) and integer-coded routing.
 * table row "Stacking several LoRAs": a few more alongside computations
   -> additivity and rank stacking.

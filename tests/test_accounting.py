@@ -21,16 +21,24 @@ def _rows():
     return out
 
 
-def test_lora_costs_table():
+def test_cost_formulas_reproduce_the_printed_flux_table():
+    """The page's table, recomputed from the library's per-layer formulas: FLUX has
+    57 layers with a LoRA on each of 4 attention projections (d = 3072, square),
+    4608 tokens, bf16 weights and an HBM of 3350 GB/s.  Each table column is one
+    ratio or sum of those formulas, so a wrong term in any of them shows here."""
+    d, n_proj, n_tok, hbm = 3072, 57 * 4, 4608, 3350e9
     rows = _rows()
     assert [r[0] for r in rows] == [8, 16, 64, 128]
     for rank, pct, mb, ms in rows:
-        extra, merge_ms, lora_mb = acc.lora_costs(3072, 57, 4, rank, 4608)
+        base = 2 * n_tok * d * d                        # one projection's x W^T
+        extra = acc.lora_flops(n_tok, rank, d, d) / base
+        size_mib = acc.adapter_elems(rank, d, d) * acc.BF16_BYTES * n_proj / 2 ** 20
+        merge_s = acc.merge_bytes(d * d * acc.BF16_BYTES * n_proj) / hbm
         assert f"{extra:.1%}" == f"{pct:.1f}%"
-        assert round(lora_mb) == mb
-        assert round(merge_ms) == ms
+        assert round(size_mib) == mb
+        assert round(merge_s * 1e3) == ms
         # the extra fraction is exactly 2r/d
-        assert abs(extra - 2 * rank / 3072) < 1e-15
+        assert abs(extra - 2 * rank / d) < 1e-15
 
 
 def test_bgmv_cost_counts_distinct_adapters_once():
