@@ -9,8 +9,10 @@
 // and the rank updates on the caller's stream, so kernels later on that stream see
 // the batch's adapters in place.
 
+#include <algorithm>
 #include <mutex>
 #include <unordered_map>
+#include <unordered_set>
 #include <vector>
 
 #include "lora_internal.cuh"
@@ -41,6 +43,9 @@ struct HostAdapter {
 
 }  // namespace
 
+struct lora_pool_mgr;
+static bool copy_in(lora_pool_mgr *m, const std::vector<std::pair<int, int64_t>> &loads, cudaStream_t st);
+
 struct lora_pool_mgr {
     std::mutex mu;
     lora_pool pool;               // the caller's device storage
@@ -48,11 +53,40 @@ struct lora_pool_mgr {
     SlotCache cache;
     std::unordered_map<int64_t, HostAdapter> reg;
     std::vector<int32_t> slot_rank;
+    CoOccurrence co;              // requests' adapter sets seen so far
+    int32_t top_k = 0;            // partners of each acquired key preloaded (0: off)
+    int32_t preloaded = 0;        // adapters the last acquire preloaded
 
     explicit lora_pool_mgr(const lora_pool &p)
         : pool(p), a_slot((int64_t)p.max_rank * p.d_in), b_slot((int64_t)p.d_out * p.max_rank),
           cache(p.n_adapters), slot_rank(p.n_adapters, 0) {}
 };
+
+// Copies (slot, key) pairs in on `st`: A, B, then the slot's rank.  On a failed
+// copy the failing key and every later one are rolled back (not resident).
+static bool copy_in(lora_pool_mgr *m, const std::vector<std::pair<int, int64_t>> &loads, cudaStream_t st)
+{
+    char *A = static_cast<char *>(const_cast<void *>(m->pool.A));
+    char *B = static_cast<char *>(const_cast<void *>(m->pool.B));
+    for (size_t i = 0; i < loads.size(); ++i) {
+        const int slot = loads[i].first;
+        const HostAdapter &h = m->reg[loads[i].second];
+        const size_t a_bytes = (size_t)h.rank * m->pool.d_in * 2, b_bytes = (size_t)m->pool.d_out * h.rank * 2;
+        cudaError_t e = cudaMemcpyAsync(A + (size_t)slot * m->a_slot * 2, h.A, a_bytes, cudaMemcpyHostToDevice, st);
+        if (e == cudaSuccess)
+            e = cudaMemcpyAsync(B + (size_t)slot * m->b_slot * 2, h.B, b_bytes, cudaMemcpyHostToDevice, st);
+        if (e == cudaSuccess) {
+            k_pm_set_rank<<<1, 1, 0, st>>>(const_cast<int32_t *>(m->pool.rank), slot, h.rank);
+            e = cudaGetLastError();
+        }
+        if (e != cudaSuccess) {
+            m->cache.rollback(loads, i);
+            return false;
+        }
+        m->slot_rank[slot] = h.rank;
+    }
+    return true;
+}
 
 extern "C" {
 
@@ -114,26 +148,27 @@ lora_status lora_pm_acquire(lora_pool_mgr *m, const int64_t *keys, int32_t n, in
     if (!m->cache.assign(keys, n, s.data(), &loads))
         return LORA_ERR_UNSUPPORTED;       // more distinct keys than slots: nothing changes
     cudaStream_t st = (cudaStream_t)stream;
-    const char *A = static_cast<const char *>(m->pool.A);
-    const char *B = static_cast<const char *>(m->pool.B);
-    for (const auto &ld : loads) {
-        const int slot = ld.first;
-        const HostAdapter &h = m->reg[ld.second];
-        const size_t a_bytes = (size_t)h.rank * m->pool.d_in * 2, b_bytes = (size_t)m->pool.d_out * h.rank * 2;
-        cudaError_t e = cudaMemcpyAsync(const_cast<char *>(A) + (size_t)slot * m->a_slot * 2, h.A, a_bytes,
-                                        cudaMemcpyHostToDevice, st);
-        if (e == cudaSuccess)
-            e = cudaMemcpyAsync(const_cast<char *>(B) + (size_t)slot * m->b_slot * 2, h.B, b_bytes,
-                                cudaMemcpyHostToDevice, st);
-        if (e == cudaSuccess) {
-            k_pm_set_rank<<<1, 1, 0, st>>>(const_cast<int32_t *>(m->pool.rank), slot, h.rank);
-            e = cudaGetLastError();
+    if (!copy_in(m, loads, st))
+        return LORA_ERR_CUDA;
+    m->preloaded = 0;
+    if (m->top_k > 0) {
+        // the top-k co-occurring partners of the batch's keys, registered and not in
+        // the batch, in order of first appearance, come in while slots allow
+        std::vector<int64_t> want, partners;
+        std::unordered_set<int64_t> in_batch(keys, keys + n);
+        for (int32_t i = 0; i < n; ++i) {
+            if (i > 0 && std::find(keys, keys + i, keys[i]) != keys + i)
+                continue;
+            m->co.top(keys[i], m->top_k, &partners);
+            for (int64_t p : partners)
+                if (!in_batch.count(p) && m->reg.count(p) && std::find(want.begin(), want.end(), p) == want.end())
+                    want.push_back(p);
         }
-        if (e != cudaSuccess) {
-            m->cache.drop(ld.second);      // not resident after all
+        std::vector<std::pair<int, int64_t>> pre;
+        m->cache.preload(want.data(), (int)want.size(), &pre);
+        if (!copy_in(m, pre, st))
             return LORA_ERR_CUDA;
-        }
-        m->slot_rank[slot] = h.rank;
+        m->preloaded = (int32_t)pre.size();
     }
     if (slots)
         for (int32_t i = 0; i < n; ++i)
@@ -141,6 +176,32 @@ lora_status lora_pm_acquire(lora_pool_mgr *m, const int64_t *keys, int32_t n, in
     if (n_loaded)
         *n_loaded = (int32_t)loads.size();
     return LORA_OK;
+}
+
+lora_status lora_pm_observe(lora_pool_mgr *m, const int64_t *keys, int32_t n)
+{
+    if (!m || n < 0 || (n > 0 && !keys))
+        return LORA_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lock(m->mu);
+    m->co.observe(keys, n);
+    return LORA_OK;
+}
+
+lora_status lora_pm_set_preload(lora_pool_mgr *m, int32_t top_k)
+{
+    if (!m || top_k < 0)
+        return LORA_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lock(m->mu);
+    m->top_k = top_k;
+    return LORA_OK;
+}
+
+int32_t lora_pm_preloaded(lora_pool_mgr *m)
+{
+    if (!m)
+        return -1;
+    std::lock_guard<std::mutex> lock(m->mu);
+    return m->preloaded;
 }
 
 }  // extern "C"

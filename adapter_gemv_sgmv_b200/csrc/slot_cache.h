@@ -9,8 +9,10 @@
 // rejected before anything changes.
 #pragma once
 
+#include <algorithm>
 #include <cstdint>
 #include <unordered_map>
+#include <unordered_set>
 #include <vector>
 
 namespace lora {
@@ -39,6 +41,15 @@ public:
         slot_of_.erase(key);
         key_[s] = -1;
         last_[s] = 0;
+    }
+
+    // Undo part of an assignment: the keys of loads[from..] were marked resident
+    // by assign() but their copies never happened, so they become missing again
+    // (their slots free) and the next batch that needs them loads them.
+    void rollback(const std::vector<std::pair<int, int64_t>> &loads, size_t from)
+    {
+        for (size_t i = from; i < loads.size(); ++i)
+            drop(loads[i].second);
     }
 
     // Assign slots to keys[0..n); slots[i] receives keys[i]'s slot.  `loads`
@@ -93,11 +104,96 @@ public:
         return true;
     }
 
+    // Bring keys[0..n) in ahead of need, after this tick's assign(): each one not
+    // resident takes a free slot, else the least recently used slot that no key of
+    // this tick holds (the batch's keys and earlier preloads are never evicted);
+    // it stops when no such slot is left.  `loads` receives (slot, key) per key.
+    void preload(const int64_t *keys, int n, std::vector<std::pair<int, int64_t>> *loads)
+    {
+        loads->clear();
+        const uint64_t tick = clock_;
+        for (int i = 0; i < n; ++i) {
+            if (find(keys[i]) >= 0)
+                continue;
+            int victim = -1;
+            for (int s = 0; s < n_slots(); ++s) {
+                if (last_[s] == tick && key_[s] >= 0)
+                    continue;
+                if (key_[s] < 0) {
+                    victim = s;
+                    break;
+                }
+                if (victim < 0 || last_[s] < last_[victim])
+                    victim = s;
+            }
+            if (victim < 0)
+                return;
+            if (key_[victim] >= 0)
+                slot_of_.erase(key_[victim]);
+            key_[victim] = keys[i];
+            slot_of_[keys[i]] = victim;
+            last_[victim] = tick;
+            loads->emplace_back(victim, keys[i]);
+        }
+    }
+
 private:
     std::vector<int64_t> key_;                // key held by each slot (-1: free)
     std::vector<uint64_t> last_;              // batch tick of each slot's last use
     std::unordered_map<int64_t, int> slot_of_;
     uint64_t clock_ = 0;
+};
+
+// Co-occurrence of adapters in requests ("Co-occurrence Patterns of LoRA Adapters in
+// Production Diffusion Model Inference Services", abstract: requests that carry
+// several adapters combine them in recurring patterns, and preloading each adapter's
+// top-k co-occurring partners covers most of them).  Counts, for every pair of
+// distinct keys, the requests that carried both; top() ranks a key's partners.
+class CoOccurrence {
+public:
+    // one request's keys (duplicates count once)
+    void observe(const int64_t *keys, int n)
+    {
+        std::vector<int64_t> d;
+        for (int i = 0; i < n; ++i)
+            if (std::find(d.begin(), d.end(), keys[i]) == d.end())
+                d.push_back(keys[i]);
+        for (size_t i = 0; i < d.size(); ++i)
+            for (size_t j = 0; j < d.size(); ++j)
+                if (i != j)
+                    ++count_[d[i]][d[j]];
+    }
+
+    // up to k partners of `key`, most frequent first (ties: smaller key first)
+    void top(int64_t key, int k, std::vector<int64_t> *out) const
+    {
+        out->clear();
+        auto it = count_.find(key);
+        if (it == count_.end() || k <= 0)
+            return;
+        std::vector<std::pair<uint64_t, int64_t>> v;
+        v.reserve(it->second.size());
+        for (const auto &e : it->second)
+            v.emplace_back(e.second, e.first);
+        const size_t m = std::min<size_t>((size_t)k, v.size());
+        std::partial_sort(v.begin(), v.begin() + m, v.end(), [](const auto &a, const auto &b) {
+            return a.first != b.first ? a.first > b.first : a.second < b.second;
+        });
+        for (size_t i = 0; i < m; ++i)
+            out->push_back(v[i].second);
+    }
+
+    uint64_t pairs(int64_t a, int64_t b) const
+    {
+        auto it = count_.find(a);
+        if (it == count_.end())
+            return 0;
+        auto jt = it->second.find(b);
+        return jt == it->second.end() ? 0 : jt->second;
+    }
+
+private:
+    std::unordered_map<int64_t, std::unordered_map<int64_t, uint64_t>> count_;
 };
 
 }  // namespace lora

@@ -68,6 +68,39 @@ def test_reregistering_replaces_the_adapter():
     check_parity(widen(to_host(Y)), want, "re-registered adapter")
 
 
+def test_preloaded_partners_give_oracle_exact_batches():
+    """Co-occurrence preloading on the GPU: after requests that pair adapter 0 with 3 and
+    1 with 4, acquiring {0, 1} also brings 3 and 4 in (on the same stream); a batch over
+    3 and 4 then loads nothing, and its decode through the managed pool matches the oracle."""
+    rng = np.random.default_rng(35)
+    d_in, d_out = 384, 256
+    ranks = [16, 32, 8, 64, 24, 16]
+    hp = rand_host_pool(rng, ranks, d_in, d_out)
+    pm = L.PoolManager(4, d_in, d_out, 64)
+    for a in range(len(ranks)):
+        pm.register(a, *_host_ab(hp, a))
+    for req in ([0, 3], [0, 3], [1, 4], [0, 5], [1, 4, 2]):
+        pm.observe(req)
+    pm.set_preload(1)
+    slots01, n = pm.acquire([0, 1, 0])
+    assert n == 2 and pm.preloaded() == 2              # partners 3 (of 0) and 4 (of 1)
+    slots34, n = pm.acquire([3, 4, 4, 3])
+    assert n == 0 and pm.preloaded() == 0              # already resident; their partners 0 and 1 too
+    tok = np.array([3, 4, 4, 3, 3, 4, 3, 3], np.int64)
+    slot_of = {3: int(slots34[0]), 4: int(slots34[1])}
+    ids = np.array([slot_of[int(k)] for k in tok], np.int32)
+    X = rand_x(rng, len(tok), d_in)
+    Y0 = rand_x(rng, len(tok), d_out)
+    Y = dev_bf16(Y0)
+    ws = L.lora_bgmv(dev_bf16(X), Y, pm, torch.tensor(ids, device=DEV), 0.75)
+    assert L.lora_get_error(ws) == 0
+    want = widen(Y0) + oracle.bgmv_delta(X, hp, tok.astype(np.int32), 0.75)
+    check_parity(widen(to_host(Y)), want, "preloaded adapters")
+    pm.set_preload(0)
+    pm.acquire([5])
+    assert pm.preloaded() == 0
+
+
 def test_oversize_batch_and_unknown_key_change_nothing():
     rng = np.random.default_rng(33)
     hp = rand_host_pool(rng, [8, 8, 8], 64, 64)

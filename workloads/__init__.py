@@ -8,5 +8,5 @@ the CPU oracle's tests take their inputs from here.
 from .configs import (  # noqa: F401
     Pool, BgmvCall, SgmvCall, MultiCall, Workload,
     make_pool, bgmv_call, sgmv_call, multi_call, zipf_ids,
-    make_workload, WORKLOAD_NAMES, bf16_bits, to_host,
+    make_workload, WORKLOAD_NAMES, bf16_bits, to_host, cooccurrence_requests,
 )

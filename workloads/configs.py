@@ -357,6 +357,33 @@ LLAMA3_8B_PROJ = [  # name, d_in, d_out, which input it reads
 ]
 
 
+def cooccurrence_requests(seed: int, n_requests: int = 20000, n_adapters: int = 200, n_bundles: int = 64,
+                          p_bundle: float = 0.8, zipf_s: float = 1.1):
+    """A stream of requests' adapter lists with recurring combinations, standing in
+    for the production traces of "Co-occurrence Patterns of LoRA Adapters in
+    Production Diffusion Model Inference Services" (not available here).
+
+    Each request carries k in {1, 2, 3} adapters with P = 0.5 / 0.3 / 0.2 (the
+    diffusion workload's mix).  A single adapter is Zipf(zipf_s) over the pool.  A
+    multi-adapter request, with probability p_bundle, takes the first k adapters of
+    one of n_bundles fixed bundles (three distinct adapters each, drawn once; the
+    bundle picked Zipf(zipf_s)); otherwise k distinct adapters uniformly.  The first
+    adapter of a list is its primary one."""
+    rng = _rng(seed)
+    bundles = [rng.choice(n_adapters, size=3, replace=False) for _ in range(n_bundles)]
+    ks = rng.choice(np.array([1, 2, 3]), size=n_requests, p=[0.5, 0.3, 0.2])
+    out = []
+    for k in ks:
+        if k == 1:
+            out.append(zipf_ids(rng, n_adapters, zipf_s, 1).astype(np.int64))
+        elif rng.random() < p_bundle:
+            b = bundles[int(zipf_ids(rng, n_bundles, zipf_s, 1)[0])]
+            out.append(np.asarray(b[:k], np.int64))
+        else:
+            out.append(rng.choice(n_adapters, size=int(k), replace=False).astype(np.int64))
+    return out
+
+
 def make_workload(which, device="cpu", seed: Optional[int] = None, y0: str = "zeros",
                   **overrides) -> Workload:
     """Build one of the named workloads (index or name).  seed defaults to the index.
