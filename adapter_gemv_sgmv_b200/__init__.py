@@ -22,7 +22,7 @@ __all__ = [
     "lora_sgmv_expand",
     "lora_apply_multi", "lora_apply_multi_static", "make_pool_struct", "Workspace", "OP_BGMV", "OP_SGMV_SHRINK", "OP_SGMV_EXPAND",
     "OP_APPLY_MULTI", "OP_ROUTE", "OP_MERGE", "OP_LINEAR", "OP_APPLY_PROJ", "STATUS", "lora_merge", "lora_linear_sgmv",
-    "PoolManager",
+    "PoolManager", "lora_test_stall",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -72,6 +72,8 @@ def load():
         PP = ctypes.POINTER(LoraPoolStruct)
         lib.lora_version.restype = ctypes.c_char_p
         lib.lora_version.argtypes = []
+        lib.lora_test_stall.restype = None
+        lib.lora_test_stall.argtypes = [ctypes.c_int, ctypes.c_double]
         lib.lora_workspace_size.restype = sz
         lib.lora_workspace_size.argtypes = [ctypes.c_int, i32, i32, i32, i32, i32, i32, i32]
         lib.lora_kernel_launches.restype = ctypes.c_int
@@ -108,8 +110,20 @@ def load():
         lib.lora_pm_register.argtypes = [P, i64, P, P, i32]
         lib.lora_pm_acquire.restype = ctypes.c_int
         lib.lora_pm_acquire.argtypes = [P, P, i32, P, P, P]
+        lib.lora_pm_observe.restype = ctypes.c_int
+        lib.lora_pm_observe.argtypes = [P, P, i32]
+        lib.lora_pm_set_preload.restype = ctypes.c_int
+        lib.lora_pm_set_preload.argtypes = [P, i32]
+        lib.lora_pm_preloaded.restype = ctypes.c_int32
+        lib.lora_pm_preloaded.argtypes = [P]
         _lib = lib
     return _lib
+
+
+def lora_test_stall(stall: bool, wait_seconds: float = 0.0) -> None:
+    """Testing hook: while set, the pipelined kernels issue no loads and every wait
+    inside a kernel gives up after wait_seconds (the call reports LORA_ERR_TIMEOUT)."""
+    load().lora_test_stall(1 if stall else 0, float(wait_seconds))
 
 
 def lora_version() -> str:
@@ -477,6 +491,20 @@ class PoolManager:
         _rc(load().lora_pm_acquire(self._h, keys.ctypes.data, len(keys), slots.ctypes.data,
                                    ctypes.byref(n_loaded), _stream_ptr(stream)), "lora_pm_acquire")
         return slots[:len(keys)], int(n_loaded.value)
+
+    def observe(self, keys):
+        """Record one request's adapter keys for co-occurrence preloading."""
+        import numpy as np
+        keys = np.ascontiguousarray(np.asarray(keys, dtype=np.int64))
+        _rc(load().lora_pm_observe(self._h, keys.ctypes.data, len(keys)), "lora_pm_observe")
+
+    def set_preload(self, top_k: int):
+        """Preload the top_k co-occurring partners of every acquired key (0: off)."""
+        _rc(load().lora_pm_set_preload(self._h, int(top_k)), "lora_pm_set_preload")
+
+    def preloaded(self) -> int:
+        """Adapters the last acquire preloaded."""
+        return int(load().lora_pm_preloaded(self._h))
 
     def close(self):
         if self._h:

@@ -27,9 +27,11 @@
 // there for the whole block).
 //
 // The LoRA k-blocks read B through the pool views of ranks 16, 32, 64 and 128
-// (adapter offsets multiples of the rank); a segment whose adapter is outside
-// those (or fails the pool checks) gets the base product only and sets
-// LORA_ERR_BAD_ADAPTER.  Every wait is bounded as in the other tcgen05 kernels.
+// when the adapter's offset is a multiple of its rank, and gather it with 16-byte
+// cp.async copies into the same swizzled layout otherwise (any rank that is a
+// multiple of 8); a segment whose adapter fails the pool checks gets the base
+// product only and sets LORA_ERR_BAD_ADAPTER.  Every wait is bounded as in the
+// other tcgen05 kernels.
 
 #include "lora_internal.cuh"
 #include "tc_ptx.cuh"
@@ -63,31 +65,37 @@ __device__ __forceinline__ LinUnit lin_unit(int64_t u, int n_pairs, int n_ns)
 }
 
 struct LinAd {
-    int r;      // rank, 0: no LoRA k-blocks
-    int brow;   // row of output 0 in the B view of rank r
-    int m;      // that view's index
+    int r;          // rank, 0: no LoRA k-blocks
+    int brow;       // TMA: row of output 0 in the B view of rank r
+    int m;          // TMA: that view's index; -1: B rows gathered with cp.async
+    int64_t boff;   // gather: element offset of the adapter's B
 };
 
-// The segment's adapter as the LoRA k-blocks use it.
+// The segment's adapter as the LoRA k-blocks use it: B through the pool's view of
+// its rank when there is one (ranks 16, 32, 64, 128, offset a multiple of the
+// rank), else gathered row by row.
 __device__ LinAd lin_adapter(const LinArgs &p, int item, bool report)
 {
-    LinAd d = {0, 0, 0};
+    LinAd d = {0, 0, 0, 0};
     const int32_t a = p.seg_ad[item];
     if (a == -1)
         return d;
     int32_t r = 0;
     int64_t ao = 0, bo = 0;
-    bool ok = pool_adapter_ok(p.pool, a, &r, &ao, &bo);
-    const int m = ok ? b_map(r) : -1;
-    ok = ok && m >= 0 && ((p.b_tma >> m) & 1) && (bo % r) == 0;
-    if (!ok) {
+    if (!pool_adapter_ok(p.pool, a, &r, &ao, &bo)) {
         if (report)
             atomicOr(p.err, (uint32_t)LORA_ERR_BAD_ADAPTER);
         return d;
     }
+    const int m = b_map(r);
     d.r = r;
-    d.brow = (int)(bo / r);
-    d.m = m;
+    d.boff = bo;
+    if (m >= 0 && ((p.b_tma >> m) & 1) && (bo % r) == 0 && bo / r <= 0x7fffffffLL) {
+        d.brow = (int)(bo / r);
+        d.m = m;
+    } else {
+        d.m = -1;
+    }
     return d;
 }
 
@@ -108,7 +116,7 @@ __device__ __forceinline__ LinPair lin_pair(const LinArgs &p, int pair, int n_ti
     x.has1 = 2 * pair + 1 < n_tiles;
     x.g[1] = x.has1 ? p.groups[2 * pair + 1] : x.g[0];
     x.ad[0] = lin_adapter(p, x.g[0].item, report);
-    x.ad[1] = x.has1 ? lin_adapter(p, x.g[1].item, report) : LinAd{0, 0, 0};
+    x.ad[1] = x.has1 ? lin_adapter(p, x.g[1].item, report) : LinAd{0, 0, 0, 0};
     x.nl[0] = lora_kblocks(x.ad[0]);
     x.nl[1] = lora_kblocks(x.ad[1]);
     return x;
@@ -119,7 +127,7 @@ __global__ void __launch_bounds__(kLinThreads, 1) k_tc_linear(const __grid_const
     extern __shared__ __align__(1024) unsigned char sm_dyn[];
     unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(sm_dyn) + 1023) & ~(uintptr_t)1023);
     __shared__ __align__(8) uint64_t full_bar[kLStages], empty_bar[kLStages];
-    __shared__ __align__(8) uint64_t acc_full, acc_empty;
+    __shared__ __align__(8) uint64_t acc_full, acc_empty, mma_drain;
     __shared__ uint32_t tmem_base;
     __shared__ int abort_flag;
 
@@ -130,11 +138,12 @@ __global__ void __launch_bounds__(kLinThreads, 1) k_tc_linear(const __grid_const
 
     if (tid == 0) {
         for (int s = 0; s < kLStages; ++s) {
-            mbar_init(&full_bar[s], 1);          // producer's expect_tx
+            mbar_init(&full_bar[s], 33);         // producer lane 0's expect_tx + 32 cp.async arrivals
             mbar_init(&empty_bar[s], 1);         // MMA commit
         }
         mbar_init(&acc_full, 1);                 // MMA commit
         mbar_init(&acc_empty, kLinEpiWarps);
+        mbar_init(&mma_drain, 1);                // the MMA issuer's last commit before TMEM is freed
         abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -149,10 +158,13 @@ __global__ void __launch_bounds__(kLinThreads, 1) k_tc_linear(const __grid_const
     const int n_tiles = p.hdr->n_groups;
     const int n_pairs = (n_tiles + 1) / 2;
     const int64_t n_units = (int64_t)n_pairs * n_ns;
+    int issued = 0;                               // producer: stage fills issued
 
     if (warp == 0) {
         // ------------------------------------------------ producer
         int it = 0;
+        if (p.test_stall)
+            goto done;
         const uint64_t pol_x = policy_evict_first(), pol_w = policy_evict_last();
         for (int64_t u = blockIdx.x; u < n_units; u += G) {
             const LinUnit un = lin_unit(u, n_pairs, n_ns);
@@ -162,7 +174,7 @@ __global__ void __launch_bounds__(kLinThreads, 1) k_tc_linear(const __grid_const
             for (int kb = 0; kb < n_all; ++kb, ++it) {
                 const int s = it % kLStages;
                 const uint32_t ph = (it / kLStages) & 1;
-                if (!warp_wait(&empty_bar[s], ph ^ 1, &abort_flag, p.err))
+                if (!warp_wait(&empty_bar[s], ph ^ 1, &abort_flag, p.err, p.wait_ns))
                     goto done;
                 if (lane == 0) {
                     unsigned char *xs = sm + s * kLStage;
@@ -183,15 +195,42 @@ __global__ void __launch_bounds__(kLinThreads, 1) k_tc_linear(const __grid_const
                         const LinAd ad = ti ? pr.ad[1] : pr.ad[0];
                         const int part = j & 1, c = j >> 1;
                         const int w = ad.r < 64 ? ad.r : 64;
-                        mbar_arrive_expect_tx(&full_bar[s], (uint32_t)(kAtom + 2 * 128 * w * 2));
+                        mbar_arrive_expect_tx(&full_bar[s], (uint32_t)(kAtom + (ad.m >= 0 ? 2 * 128 * w * 2 : 0)));
                         tma_load_2d_hint(xs, &p.map_v, &full_bar[s], part * p.kv + c * 64,
                                          ti ? pr.g[1].p0 : pr.g[0].p0, pol_x);
-                        tma_load_2d_hint(wsm, &p.map_b[ad.m], &full_bar[s], c * 64, ad.brow + o0, pol_w);
-                        tma_load_2d_hint(wsm + 128 * w * 2, &p.map_b[ad.m], &full_bar[s], c * 64,
-                                         ad.brow + o0 + 128, pol_w);
+                        if (ad.m >= 0) {
+                            tma_load_2d_hint(wsm, &p.map_b[ad.m], &full_bar[s], c * 64, ad.brow + o0, pol_w);
+                            tma_load_2d_hint(wsm + 128 * w * 2, &p.map_b[ad.m], &full_bar[s], c * 64,
+                                             ad.brow + o0 + 128, pol_w);
+                        }
                     }
                 }
                 __syncwarp();
+                if (kb >= n_kb) {
+                    // a LoRA k-block whose adapter has no B view: all lanes gather its
+                    // 256 output rows x 64 rank columns (16-byte chunks, 128-byte swizzle,
+                    // the layout of the rank >= 64 views); ranks past r and outputs past
+                    // d_out are zero-filled
+                    int j = kb - n_kb;
+                    const int ti = j < pr.nl[0] ? 0 : 1;
+                    if (ti)
+                        j -= pr.nl[0];
+                    const LinAd ad = ti ? pr.ad[1] : pr.ad[0];
+                    if (ad.m < 0) {
+                        const int rc0 = (j >> 1) * 64;
+                        const uint32_t wbase = smem_u32(sm + s * kLStage + 2 * kAtom);
+                        for (int idx = lane; idx < kLN * 8; idx += 32) {
+                            const int o = idx >> 3, cc = idx & 7;
+                            const int col = rc0 + cc * 8;
+                            const bool ok = o0 + o < p.d_out && col < ad.r;
+                            const __nv_bfloat16 *src = ok ? p.pool.B + ad.boff + (int64_t)(o0 + o) * ad.r + col
+                                                          : p.pool.B;
+                            cp_async16(wbase + (o >> 7) * kAtom + sw128_off(o & 127, cc), src, ok);
+                        }
+                    }
+                }
+                cp_async_arrive(&full_bar[s]);
+                issued = it + 1;
             }
         }
     } else if (warp == 1) {
@@ -202,14 +241,16 @@ __global__ void __launch_bounds__(kLinThreads, 1) k_tc_linear(const __grid_const
             const LinUnit un = lin_unit(u, n_pairs, n_ns);
             const LinPair pr = lin_pair(p, un.pair, n_tiles, false);
             const int n_all = n_kb + pr.nl[0] + pr.nl[1];
-            if (!warp_wait(&acc_empty, (t & 1) ^ 1, &abort_flag, p.err))
+            if (!warp_wait(&acc_empty, (t & 1) ^ 1, &abort_flag, p.err, p.wait_ns))
                 goto done;
             tc_fence_after();
             for (int kb = 0; kb < n_all; ++kb, ++it) {
                 const int s = it % kLStages;
                 const uint32_t ph = (it / kLStages) & 1;
-                if (!warp_wait(&full_bar[s], ph, &abort_flag, p.err))
+                if (!warp_wait(&full_bar[s], ph, &abort_flag, p.err, p.wait_ns))
                     goto done;
+                if (kb >= n_kb)
+                    fence_async_smem();             // B may have been written by cp.async (generic proxy)
                 tc_fence_after();
                 if (lane == 0) {
                     const uint32_t xa = smem_u32(sm + s * kLStage), wa = xa + 2 * kAtom;
@@ -227,12 +268,17 @@ __global__ void __launch_bounds__(kLinThreads, 1) k_tc_linear(const __grid_const
                     } else {
                         int j = kb - n_kb;
                         const int ti = j < pr.nl[0] ? 0 : 1;
-                        const int r = ti ? pr.ad[1].r : pr.ad[0].r;
-                        const int steps = (r < 64 ? r : 64) >> 4;
+                        if (ti)
+                            j -= pr.nl[0];
+                        const LinAd ad = ti ? pr.ad[1] : pr.ad[0];
+                        const int r = ad.r;
+                        const int left = r - (j >> 1) * 64;          // ranks in this k-block
+                        const int steps = ((left < 64 ? left : 64) + 15) >> 4;
                         for (int k = 0; k < steps; ++k) {
-                            // B columns in the view's swizzle: 128-byte rows from rank 64 up,
-                            // 64-byte rows at rank 32, 32-byte rows at rank 16
-                            const uint64_t bdesc = r >= 64 ? sw128_desc(wa + k * 32)
+                            // B columns in the view's swizzle: 128-byte rows from rank 64 up
+                            // (and for every gathered block), 64-byte rows at rank 32,
+                            // 32-byte rows at rank 16
+                            const uint64_t bdesc = (r >= 64 || ad.m < 0) ? sw128_desc(wa + k * 32)
                                                  : (r == 32 ? sw64_desc(wa + k * 32) : sw32_desc(wa));
                             tc_mma(tmem + ti * kLN, sw128_desc(xa + k * 32), bdesc, idesc, 1u);
                         }
@@ -255,7 +301,7 @@ __global__ void __launch_bounds__(kLinThreads, 1) k_tc_linear(const __grid_const
         for (int64_t u = blockIdx.x; u < n_units; u += G, ++t) {
             const LinUnit un = lin_unit(u, n_pairs, n_ns);
             const int tile = 2 * un.pair + ti;
-            if (!warp_wait(&acc_full, t & 1, &abort_flag, p.err))
+            if (!warp_wait(&acc_full, t & 1, &abort_flag, p.err, p.wait_ns))
                 goto done;
             tc_fence_after();
             if (tile < n_tiles) {
@@ -292,6 +338,11 @@ __global__ void __launch_bounds__(kLinThreads, 1) k_tc_linear(const __grid_const
         }
     }
 done:
+    // nothing may land in shared memory or TMEM after this CTA lets go of them
+    if (warp == 0)
+        drain_fills(full_bar, kLStages, issued, p.err, p.wait_ns);
+    if (warp == 1 && lane == 0)
+        drain_mma(&mma_drain, 0, p.err, p.wait_ns);
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
@@ -316,8 +367,11 @@ bool lin_encode(LinArgs &a, const void *X, int64_t ldx, int32_t N, const void *W
     return true;
 }
 
-cudaError_t launch_tc_linear(const LinArgs &a, int max_units, cudaStream_t s)
+cudaError_t launch_tc_linear(const LinArgs &a_in, int max_units, cudaStream_t s)
 {
+    LinArgs a = a_in;
+    a.wait_ns = wait_bound_ns();
+    a.test_stall = test_stall_mode();
     static bool attr_set[64] = {};
     const int smem = kLStages * kLStage + 1024;
     int dev = 0;

@@ -5,6 +5,8 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <atomic>
+
 #include "lora_internal.cuh"
 
 using namespace lora;
@@ -33,7 +35,28 @@ bool tc_enabled()
     return on;
 }
 
+namespace {
+std::atomic<int> g_test_stall{0};
+std::atomic<unsigned long long> g_wait_ns{kWaitBoundNs};
+}  // namespace
+
+int test_stall_mode() { return g_test_stall.load(std::memory_order_relaxed); }
+unsigned long long wait_bound_ns() { return g_wait_ns.load(std::memory_order_relaxed); }
+
 }  // namespace lora
+
+extern "C" LORA_API void lora_test_stall(int stall, double wait_seconds)
+{
+    using namespace lora;
+    if (stall) {
+        const double ns = wait_seconds > 0 ? wait_seconds * 1e9 : 0.0;
+        g_wait_ns.store(ns < 1e3 ? 1000ull : (ns > 2e9 ? kWaitBoundNs : (unsigned long long)ns));
+        g_test_stall.store(1);
+    } else {
+        g_test_stall.store(0);
+        g_wait_ns.store(kWaitBoundNs);
+    }
+}
 
 namespace {
 
@@ -297,7 +320,7 @@ int lora_kernel_launches(int op, int32_t N, int32_t n_adapters, int32_t d_in, in
         return 0;
     switch (op) {
     case LORA_OP_BGMV:
-        return fused_bgmv_supported(N, n_adapters, d_in) ? 1 : 3;
+        return stream_bgmv_supported(N, n_adapters) || fused_bgmv_supported(N, n_adapters, d_in) ? 1 : 3;
     case LORA_OP_SGMV_SHRINK:
     case LORA_OP_SGMV_EXPAND:
         return n_items > 0 ? 2 : 0;
@@ -385,6 +408,30 @@ lora_status lora_bgmv(const void *X, int64_t ldx, void *Y, int64_t ldy, const lo
         return LORA_OK;
     cudaStream_t s = (cudaStream_t)stream;
     WsHeader *hdr = at<WsHeader>(ws, L.hdr);
+    if (stream_bgmv_supported(N, pool->n_adapters)) {
+        StreamBgmvArgs sa = {};
+        sa.X = static_cast<const __nv_bfloat16 *>(X);
+        sa.ldx = ldx;
+        sa.Y = static_cast<__nv_bfloat16 *>(Y);
+        sa.ldy = ldy;
+        sa.ids = ids;
+        sa.N = N;
+        sa.pool = pool_dev(pool);
+        sa.scale = scale;
+        sa.V = at<float>(ws, L.V);
+        sa.ldv = pool->max_rank;
+        sa.plane = (int64_t)N * pool->max_rank;
+        sa.max_parts = L.n_chunks;
+        sa.hdr = hdr;
+        sa.test_stall = test_stall_mode();
+        sa.wait_ns = wait_bound_ns();
+        const cudaError_t e = launch_bgmv_stream(sa, s, pdl_enabled());
+        if (e == cudaSuccess)
+            return LORA_OK;
+        if (e != cudaErrorNotSupported)
+            return LORA_ERR_CUDA;
+        // the kernel does not fit this device: the kernels below take the call
+    }
     if (fused_bgmv_supported(N, pool->n_adapters, pool->d_in)) {
         FusedBgmvArgs fa = {};
         fa.X = static_cast<const __nv_bfloat16 *>(X);

@@ -48,6 +48,7 @@ constexpr int kEpiWarps = 16;
 // heights of the A-pool TMA boxes (map_a[m])
 __host__ __device__ constexpr int abox_rows(int m) { return m == 0 ? 64 : (m == 1 ? 32 : 8); }
 constexpr int kBN = 128;            // expand: outputs per unit
+constexpr int kZeroCol = 1 << 30;          // shrink epilogue: a V column written as zeros
 constexpr int kMaxShrinkStages = 6;
 constexpr int kExpandBStages = 2;
 
@@ -180,7 +181,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) k_tc_shrink(const __grid_consta
     // 1024-byte alignment for the swizzle atoms
     unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(sm_dyn) + 1023) & ~(uintptr_t)1023);
     __shared__ __align__(8) uint64_t full_bar[kMaxShrinkStages], empty_bar[kMaxShrinkStages];
-    __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2];
+    __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2], mma_drain;
     __shared__ __align__(8) StackSm stk[kTcThreads / 32];
     __shared__ const __nv_bfloat16 *arow[kKMaxShrink];   // producer, cp.async path: stacked row j's A row
     __shared__ int4 abox[kKMaxShrink / 8];   // producer, TMA path: (stacked row, pool row, map) of each A box
@@ -204,6 +205,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) k_tc_shrink(const __grid_consta
             mbar_init(&acc_full[b], 1);      // MMA commit
             mbar_init(&acc_empty[b], 4);     // one arrival per epilogue warp
         }
+        mbar_init(&mma_drain, 1);            // the MMA issuer's last commit before TMEM is freed
         abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -217,11 +219,14 @@ __global__ void __launch_bounds__(kTcThreads, 2) k_tc_shrink(const __grid_consta
     pdl_trigger();
     const int n_units = p.hdr->n_groups;
     const int u0 = (int)((int64_t)blockIdx.x * n_units / G), u1 = (int)((int64_t)(blockIdx.x + 1) * n_units / G);
+    int issued = 0;                              // producer: stage fills issued
 
     if (warp == 0) {
         // ------------------------------------------------ producer
         StackSm &st = stk[0];
         int it = 0;
+        if (p.test_stall)
+            goto done;
         for (int u = u0; u < u1; ++u) {
             const Group gr = p.groups[u];
             warp_build_stack(p, gr.item, st, false, kKMaxShrink);
@@ -267,7 +272,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) k_tc_shrink(const __grid_consta
                 const int s = it % n_st;
                 const uint32_t ph = (it / n_st) & 1;
                 TC_STAMP(0, it, 0);
-                if (!warp_wait(&empty_bar[s], ph ^ 1, &abort_flag, p.err))
+                if (!warp_wait(&empty_bar[s], ph ^ 1, &abort_flag, p.err, p.wait_ns))
                     goto done;
                 TC_STAMP(0, it, 1);
                 unsigned char *xs = sm + s * p.s_stage;
@@ -290,6 +295,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) k_tc_shrink(const __grid_consta
                         cp_async16(abase + sw128_off(j, c), in ? arow[j] + col : p.pool.A, in);
                 }
                 cp_async_arrive(&full_bar[s]);
+                issued = it + 1;
                 TC_STAMP(0, it, 2);
             }
         }
@@ -303,7 +309,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) k_tc_shrink(const __grid_consta
             const int kpad = st.kpad;
             const bool a_tma = st.a_tma;
             const int b = t & 1;
-            if (!warp_wait(&acc_empty[b], ((t >> 1) & 1) ^ 1, &abort_flag, p.err))
+            if (!warp_wait(&acc_empty[b], ((t >> 1) & 1) ^ 1, &abort_flag, p.err, p.wait_ns))
                 goto done;
             tc_fence_after();
             const uint32_t idesc = idesc_bf16(kBM, kpad > 0 ? kpad : 16);
@@ -311,7 +317,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) k_tc_shrink(const __grid_consta
                 const int s = it % n_st;
                 const uint32_t ph = (it / n_st) & 1;
                 TC_STAMP(1, it, 0);
-                if (!warp_wait(&full_bar[s], ph, &abort_flag, p.err))
+                if (!warp_wait(&full_bar[s], ph, &abort_flag, p.err, p.wait_ns))
                     goto done;
                 TC_STAMP(1, it, 1);
                 if (!a_tma)
@@ -352,12 +358,16 @@ __global__ void __launch_bounds__(kTcThreads, 2) k_tc_shrink(const __grid_consta
                 if (k < st.ktot) {
                     const int e = stack_entry(st, k);
                     c = st.vc0[e] + (k - st.kb[e]);
+                } else if (p.Vb && st.n == 1 && k < ((st.ktot + 15) & ~15)) {
+                    // bf16-pair output: the columns up to the next 16 are written as zeros,
+                    // since the projection's MMAs read V in steps of 16 ranks
+                    c = (st.vc0[0] + k) | kZeroCol;
                 }
                 vc[g] = c;
             }
             __syncwarp();
             const int b = t & 1;
-            if (!warp_wait(&acc_full[b], (t >> 1) & 1, &abort_flag, p.err))
+            if (!warp_wait(&acc_full[b], (t >> 1) & 1, &abort_flag, p.err, p.wait_ns))
                 goto done;
             tc_fence_after();
             const bool valid = row < gr.cnt;
@@ -370,9 +380,15 @@ __global__ void __launch_bounds__(kTcThreads, 2) k_tc_shrink(const __grid_consta
                 if (valid) {
 #pragma unroll
                     for (int g = 0; g < 8; ++g) {
-                        const int col = vc[(c0 >> 2) + g];
+                        int col = vc[(c0 >> 2) + g];
                         if (col < 0)
                             continue;
+                        if (col & kZeroCol) {
+                            col &= ~kZeroCol;
+                            *reinterpret_cast<uint2 *>(brow + col) = make_uint2(0u, 0u);
+                            *reinterpret_cast<uint2 *>(brow + p.vb_lo + col) = make_uint2(0u, 0u);
+                            continue;
+                        }
                         if (brow) {
                             // s v as a high and a low bf16 part (the fused projection's LoRA operand)
                             uint32_t hi[2], lo[2];
@@ -401,6 +417,12 @@ __global__ void __launch_bounds__(kTcThreads, 2) k_tc_shrink(const __grid_consta
         }
     }
 done:
+    // nothing may land in shared memory or TMEM after this CTA lets go of them:
+    // the producer waits for its fills, the MMA issuer for its last MMAs
+    if (warp == 0)
+        drain_fills(full_bar, n_st, issued, p.err, p.wait_ns);
+    if (warp == 1 && lane == 0)
+        drain_mma(&mma_drain, 0, p.err, p.wait_ns);
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
@@ -443,6 +465,7 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_tc_expand(const __grid_co
     __shared__ int vsrc[kEpiWarps][kKMax / 8];   // epilogue warp e: V column of stacked chunk c (-1: zero)
     __shared__ float vsc[kEpiWarps][kKMax / 8];  // and its adapter's scale
     __shared__ uint32_t tmem_base;
+    __shared__ __align__(8) uint64_t mma_drain;
     __shared__ int abort_flag;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -471,6 +494,7 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_tc_expand(const __grid_co
         }
         mbar_init(&v_full, kEpiWarps);       // epilogue warps, after staging V
         mbar_init(&v_empty, 1);              // MMA commit after a tile's last unit
+        mbar_init(&mma_drain, 1);            // the MMA issuer's last commit before TMEM is freed
         abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -484,11 +508,14 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_tc_expand(const __grid_co
     pdl_trigger();
     const int64_t n_units = (int64_t)p.hdr->n_groups * n_ns;
     const int64_t u0 = (int64_t)blockIdx.x * n_units / G, u1 = (int64_t)(blockIdx.x + 1) * n_units / G;
+    int y_issued = 0, b_issued = 0;              // producer: y and B stage fills issued
 
     if (warp == 0) {
         // ------------------------------------------------ producer: y tiles and B slices
         StackSm &st = stk[0];
         int it = 0;
+        if (p.test_stall)
+            goto done;
         int64_t prev_tile = -1;
         int nch = 0, o_l = 0, c_l = 0, dq = 0, dr = 0;
         int p0 = 0;
@@ -536,7 +563,7 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_tc_expand(const __grid_co
             const int o0 = ns * kBN;
             const int sy = it % n_ys;
             TC_STAMP(0, it, 0);
-            if (!warp_wait(&y_empty[sy], ((it / n_ys) & 1) ^ 1, &abort_flag, p.err))
+            if (!warp_wait(&y_empty[sy], ((it / n_ys) & 1) ^ 1, &abort_flag, p.err, p.wait_ns))
                 goto done;
             TC_STAMP(0, it, 1);
             unsigned char *ys = smY + sy * kY;
@@ -545,8 +572,9 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_tc_expand(const __grid_co
                 tma_load_2d_hint(ys, &p.map_y, &y_full[sy], o0, p0, pol_y);
                 tma_load_2d_hint(ys + kAtom, &p.map_y, &y_full[sy], o0 + 64, p0, pol_y);
             }
+            y_issued = it + 1;
             const int sb = it % kExpandBStages;
-            if (!warp_wait(&b_empty[sb], ((it / kExpandBStages) & 1) ^ 1, &abort_flag, p.err))
+            if (!warp_wait(&b_empty[sb], ((it / kExpandBStages) & 1) ^ 1, &abort_flag, p.err, p.wait_ns))
                 goto done;
             TC_STAMP(0, it, 2);
             unsigned char *bs = smB + sb * szB;
@@ -583,6 +611,7 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_tc_expand(const __grid_co
                 }
             }
             cp_async_arrive(&b_full[sb]);
+            b_issued = it + 1;
             TC_STAMP(0, it, 3);
         }
     } else if (warp == 1) {
@@ -623,17 +652,17 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_tc_expand(const __grid_co
                         bd[k16] = sw128_desc((k >> 6) * kAtom + ((k & 63) >> 4) * 32);
                     }
                 }
-                if (!warp_wait(&v_full, vt & 1, &abort_flag, p.err))
+                if (!warp_wait(&v_full, vt & 1, &abort_flag, p.err, p.wait_ns))
                     goto done;
                 ++vt;
             }
             const int b = it & 1;
             TC_STAMP(1, it, 0);
-            if (!warp_wait(&acc_empty[b], ((it >> 1) & 1) ^ 1, &abort_flag, p.err))
+            if (!warp_wait(&acc_empty[b], ((it >> 1) & 1) ^ 1, &abort_flag, p.err, p.wait_ns))
                 goto done;
             TC_STAMP(1, it, 1);
             const int sb = it % kExpandBStages;
-            if (!warp_wait(&b_full[sb], (it / kExpandBStages) & 1, &abort_flag, p.err))
+            if (!warp_wait(&b_full[sb], (it / kExpandBStages) & 1, &abort_flag, p.err, p.wait_ns))
                 goto done;
             TC_STAMP(1, it, 2);
             if (!b_tma)
@@ -699,7 +728,7 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_tc_expand(const __grid_co
                 }
                 __syncwarp();
                 // wait until the MMAs of the previous tile stopped reading V
-                if (vt > 0 && !warp_wait(&v_empty, (vt - 1) & 1, &abort_flag, p.err))
+                if (vt > 0 && !warp_wait(&v_empty, (vt - 1) & 1, &abort_flag, p.err, p.wait_ns))
                     goto done;
                 // V[vr][stacked k] = s_e * V_e[vr][k - kb_e] (s_e = 1 for one adapter), zero outside the
                 // tile's rows and the stack, as two bf16 parts: hi = bf16(v) and lo = bf16(v - hi), so
@@ -742,11 +771,11 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_tc_expand(const __grid_co
             const int sy = it % n_ys;
             if (warp == 2)
                 TC_STAMP(2, it, 0);
-            if (!warp_wait(&acc_full[b], (it >> 1) & 1, &abort_flag, p.err))
+            if (!warp_wait(&acc_full[b], (it >> 1) & 1, &abort_flag, p.err, p.wait_ns))
                 goto done;
             if (warp == 2)
                 TC_STAMP(2, it, 1);
-            if (!warp_wait(&y_full[sy], (it / n_ys) & 1, &abort_flag, p.err))
+            if (!warp_wait(&y_full[sy], (it / n_ys) & 1, &abort_flag, p.err, p.wait_ns))
                 goto done;
             if (warp == 2)
                 TC_STAMP(2, it, 2);
@@ -822,6 +851,13 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_tc_expand(const __grid_co
         }
     }
 done:
+    // nothing may land in shared memory or TMEM after this CTA lets go of them
+    if (warp == 0) {
+        drain_fills(y_full, n_ys, y_issued, p.err, p.wait_ns);
+        drain_fills(b_full, kExpandBStages, b_issued, p.err, p.wait_ns);
+    }
+    if (warp == 1 && lane == 0)
+        drain_mma(&mma_drain, 0, p.err, p.wait_ns);
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
@@ -922,6 +958,8 @@ cudaError_t launch_tc_shrink(const TcArgs &args, int max_tiles, int kk, cudaStre
         return e;
     const int room = optin - (int)fa.sharedSizeBytes - 1024;
     TcArgs a = args;
+    a.wait_ns = wait_bound_ns();
+    a.test_stall = test_stall_mode();
     const int a_rows = (kk + 15) & ~15;
     const bool wide = kk > kKMax;
     a.s_stage = kAtom + a_rows * 128;
@@ -960,6 +998,8 @@ cudaError_t launch_tc_expand(const TcArgs &args, int kk, cudaStream_t s)
     if ((e = cudaFuncGetAttributes(&fa, k_tc_expand)) != cudaSuccess)
         return e;
     TcArgs a = args;
+    a.wait_ns = wait_bound_ns();
+    a.test_stall = test_stall_mode();
     a.e_natoms = kk > 64 ? 2 : 1;
     const int fixed = (2 + kExpandBStages) * a.e_natoms * kAtom + kStaging + 1024;
     const int room = optin - (int)fa.sharedSizeBytes - fixed;

@@ -21,7 +21,6 @@ __host__ __device__ constexpr int b_map(int r) { return r == 16 ? 0 : (r == 32 ?
 constexpr int kBM = 128;            // rows per tile
 constexpr int kBK = 64;             // d_in per k-block (one 128-byte swizzle atom)
 constexpr int kAtom = kBM * 128;    // bytes of a 128-row x 64-column bf16 swizzle atom
-constexpr unsigned long long kWaitNs = 2000000000ull;   // 2 s bound on any single wait
 
 // ------------------------------------------------------------------ PTX glue
 __device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
@@ -60,9 +59,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
 }
 
 // Bounded wait for the phase with the given parity.  Returns false if the CTA
-// is already aborting or the bound expires (then it marks the abort itself).
+// is already aborting or `limit_ns` passes (then it marks the abort itself).
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
-                                          uint32_t *err)
+                                          uint32_t *err, unsigned long long limit_ns)
 {
     if (mbar_try_wait(bar, parity))
         return true;
@@ -70,10 +69,10 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity))
             return true;
-        if ((i & 255) == 0) {
+        if ((i & 63) == 0) {
             if (*abort_flag)
                 return false;
-            if (now_ns() - t0 > kWaitNs) {
+            if (now_ns() - t0 > limit_ns) {
                 *abort_flag = 1;
                 atomicOr(err, (uint32_t)LORA_ERR_TIMEOUT);
                 return false;
@@ -83,9 +82,42 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
 }
 
 // The whole warp waits; all lanes leave together (all succeed or all give up).
-__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag, uint32_t *err)
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag, uint32_t *err,
+                                          unsigned long long limit_ns)
 {
-    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, err));
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, err, limit_ns));
+}
+
+// Before a CTA that gave up may exit: every fill of a ring of `n_stages` barriers
+// issued so far (fills 0 .. issued-1, fill i on barrier i % n_stages) must have
+// landed, whether or not a consumer got to it.  Bounded like every wait.
+__device__ __forceinline__ void drain_fills(uint64_t *bars, int n_stages, int issued, uint32_t *err,
+                                            unsigned long long limit_ns)
+{
+    for (int i = issued > n_stages ? issued - n_stages : 0; i < issued; ++i) {
+        const unsigned long long t0 = now_ns();
+        while (!mbar_try_wait(&bars[i % n_stages], (uint32_t)((i / n_stages) & 1))) {
+            if (now_ns() - t0 > limit_ns) {
+                atomicOr(err, (uint32_t)LORA_ERR_TIMEOUT);
+                break;
+            }
+        }
+    }
+}
+
+// Before TMEM is freed: every tcgen05.mma this thread issued has completed
+// (a commit to `bar`, a fresh phase of a barrier of count 1).  Bounded.
+__device__ __forceinline__ void drain_mma(uint64_t *bar, uint32_t parity, uint32_t *err, unsigned long long limit_ns)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+    const unsigned long long t0 = now_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (now_ns() - t0 > limit_ns) {
+            atomicOr(err, (uint32_t)LORA_ERR_TIMEOUT);
+            break;
+        }
+    }
 }
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d)

@@ -61,12 +61,6 @@ WORKLOAD_DESC = {
 }
 
 
-# DRAM traffic of the step's only kernel, from one ncu capture of the current kernel
-# (dram__bytes_read.sum + dram__bytes_write.sum of one launch); None where the step has
-# several kernels or no capture of the current kernel exists.
-NCU_TRAFFIC = {"decode_bgmv": 21_570_560}
-
-
 def unit_of(workload: str) -> str:
     """The merge streams weight rows; every other workload, token rows."""
     return "weight rows/s" if workload == "merge_mlp_up" else "tokens/s"
@@ -212,10 +206,12 @@ def load_peaks():
 # ----------------------------------------------------------------------------
 # workload steps
 # ----------------------------------------------------------------------------
+# workload overrides for profiling one part of a workload (set by --only-proj)
+OVERRIDES = {}
+
+
 def build_sets(name, device, rank, n_sets):
-    from workloads import make_workload, WORKLOAD_NAMES
-    idx = WORKLOAD_NAMES.index(name)
-    return [make_workload(idx, device=device, seed=rank_seed(idx, rank, s)) for s in range(n_sets)]
+    return build_sets_from(name, device, rank, 0, n_sets)
 
 
 def _is_linear(call) -> bool:
@@ -328,12 +324,188 @@ def workspace_for(call):
 
 
 # ----------------------------------------------------------------------------
+# traffic of a step's dominant kernel, from a committed ncu summary
+# ----------------------------------------------------------------------------
+def profile_traffic(workload: str):
+    """DRAM bytes (read + write) per launch of the workload's dominant kernel, from
+    the committed ncu summary that records it -- only while the kernel's source
+    file is byte-identical to the one profiled (its sha256 is in the summary's
+    record line), else None."""
+    import glob
+    import hashlib
+    import re
+    pat = re.compile(r"^traffic-record: workload=(\S+) kernel=(\S+) bytes_per_launch=(\d+) "
+                     r"source=(\S+) sha256=([0-9a-f]{16})\s*$")
+    for f in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
+        for line in open(f):
+            m = pat.match(line.strip())
+            if not m or m.group(1) != workload:
+                continue
+            src = os.path.join(ROOT, m.group(4))
+            if not os.path.exists(src):
+                return None
+            h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+            if h != m.group(5):
+                return None
+            return {"bytes": int(m.group(3)), "kernel": m.group(2), "profile": os.path.relpath(f, ROOT)}
+    return None
+
+
+def config_of(workload: str, tokens: int, world: int) -> dict:
+    """The line's `config`: the workload itself, the same in both arms."""
+    desc = WORKLOAD_DESC[workload]
+    if workload in OVERRIDES:
+        desc += f" -- restricted for profiling: {OVERRIDES[workload]}"
+    return {"workload": desc, "tokens_per_step_per_gpu": int(tokens),
+            "parallelism": f"dp{world} (independent batches per GPU, no collective)"}
+
+
+# ----------------------------------------------------------------------------
 # our arm
 # ----------------------------------------------------------------------------
+L2_BYTES = 126 * 2 ** 20
+
+
+class Bench:
+    """One workload's input sets on the device, one CUDA graph per set (a step =
+    one graph replay), and the accounting of a step."""
+
+    def __init__(self, name, dev, rank, stream, max_sets=16, min_set_total=4 * L2_BYTES):
+        import torch
+        from adapter_gemv_sgmv_b200 import accounting
+        self.name = name
+        self.stream = stream
+        self.sets = build_sets(name, dev, rank, 1)
+        self.set_bytes = self._bytes(self.sets[0])
+        # enough independent sets that a step never finds the previous steps' inputs in L2
+        n_sets = int(min(max_sets, max(2, -(-min_set_total // max(self.set_bytes, 1)))))
+        if n_sets > 1:
+            self.sets += build_sets_from(name, dev, rank, 1, n_sets)
+        self.ws_map = {}
+        for wl in self.sets:
+            for c in wl.calls:
+                self.ws_map[id(c)] = workspace_for(c)
+        self.steps = [make_step(wl, self.ws_map, stream) for wl in self.sets]
+        self.cost = accounting.workload_cost(self.sets[0])
+        self.tokens = self.sets[0].n_tokens
+        self.launches = launches_per_step(self.sets[0])
+        self.graphs = []
+        torch.cuda.synchronize()
+
+    @staticmethod
+    def _bytes(wl):
+        n, seen_x = 0, set()
+        for c in wl.calls:
+            if _is_linear(c):
+                io = (c.X.numel() + c.W.numel() + c.Y.numel()) * 2
+            elif hasattr(c, "W"):
+                io = c.W.numel() * 2
+            else:
+                io = c.Y.numel() * 2 + (0 if c.X.data_ptr() in seen_x else c.X.numel() * 2)
+                seen_x.add(c.X.data_ptr())
+            n += c.pool.A.numel() * 2 + c.pool.B.numel() * 2 + io
+        return n
+
+    def warm(self, warmup):
+        import torch
+        import adapter_gemv_sgmv_b200 as L
+        # eager warm-up (also sets per-device function attributes before capture)
+        with torch.cuda.stream(self.stream):
+            for i in range(max(warmup, 3)):
+                self.steps[i % len(self.steps)]()
+        self.stream.synchronize()
+        for ws in self.ws_map.values():
+            err = L.lora_get_error(ws, stream=self.stream)
+            if err:
+                raise SystemExit(f"{self.name}: device error {err} during warm-up")
+
+    def capture(self, steps):
+        """One CUDA graph of `steps` consecutive steps rotating over the input sets
+        (consecutive kernels overlap their prologues as they would in a model's
+        graph), replayed once untimed."""
+        import torch
+        self.graphs.clear()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=self.stream):
+            for i in range(steps):
+                self.steps[i % len(self.steps)]()
+        self.graphs.append(g)
+        self.graph_steps = steps
+        with torch.cuda.stream(self.stream):
+            g.replay()
+        torch.cuda.synchronize()
+
+    def timed(self, replays=1):
+        """Device time (ms) of `replays` replays of the captured graph (each
+        `graph_steps` steps), CUDA events on the launching stream."""
+        import torch
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(self.stream):
+            e0.record(self.stream)
+            for _ in range(replays):
+                self.graphs[0].replay()
+            e1.record(self.stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1)
+
+    def check_errors(self):
+        import adapter_gemv_sgmv_b200 as L
+        for ws in self.ws_map.values():
+            err = L.lora_get_error(ws, stream=self.stream)
+            if err:
+                raise SystemExit(f"{self.name}: device error {err} in the timed steps")
+
+    def release(self):
+        import torch
+        self.graphs.clear()
+        self.steps.clear()
+        self.ws_map.clear()
+        self.sets.clear()
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+
+
+def build_sets_from(name, device, rank, start, stop):
+    from workloads import make_workload, WORKLOAD_NAMES
+    idx = WORKLOAD_NAMES.index(name)
+    ov = OVERRIDES.get(name, {})
+    return [make_workload(idx, device=device, seed=rank_seed(idx, rank, s), **ov) for s in range(start, stop)]
+
+
+def roofline_of(name, cost, ms_per_step, clk, peaks, peak_src):
+    """Algorithmic bytes (FLOPs for the fused projection) per step over the measured
+    step time, against the measured peak."""
+    t = ms_per_step * 1e-3
+    gbs = cost.bytes / t / 1e9
+    tflops = cost.flops / t / 1e12
+    tr = profile_traffic(name)
+    traffic = None
+    if tr is not None:
+        traffic = tr["bytes"]
+    if name == "prefill_linear_up":
+        # a dense projection: tensor-bound.  The burst cuBLAS peak while the SM clock
+        # stayed near its maximum, the sustained (power-capped) one once it fell below 85 %
+        capped = (clk.get("sm_mhz") or 0) < 0.85 * (clk.get("sm_max_mhz") or 1)
+        key = "bf16_tflops_sustained" if capped else "bf16_tflops"
+        pk = peaks.get(key, peaks["bf16_tflops"])
+        return {"bound": "tensor", "achieved": round(tflops, 1), "peak": pk, "unit": "TFLOP/s",
+                "frac": round(tflops / pk, 4), "traffic": traffic,
+                "peak_source": f"{peak_src} (MEASURED_PEAKS.json {key})" if peak_src == "measured" else "fallback",
+                "algorithmic_flops_per_step": cost.flops, "algorithmic_bytes_per_step": cost.bytes}
+    return {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": traffic,
+            "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else "fallback",
+            "algorithmic_bytes_per_step": cost.bytes}
+
+
+ALL_WORKLOADS = ["tiny_sgmv", "decode_bgmv", "prefill_sgmv", "mixed_rank_layer", "diffusion_multi",
+                 "prefill_qkv", "merge_mlp_up", "prefill_linear_up"]
+
+
 def run_ours(args):
     import torch
     import adapter_gemv_sgmv_b200 as L
-    from adapter_gemv_sgmv_b200 import accounting
 
     world, rank, local = dist_env()
     if world != args.gpus:
@@ -343,126 +515,109 @@ def run_ours(args):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     L.load()
-
-    n_sets = args.sets
-    sets = build_sets(args.workload, dev, rank, n_sets)
     stream = torch.cuda.Stream(device=dev)
-    ws_map = {}
-    for wl in sets:
-        for c in wl.calls:
-            ws_map[id(c)] = workspace_for(c)
-    steps = [make_step(wl, ws_map, stream) for wl in sets]
-    torch.cuda.synchronize()
+    peaks, peak_src = load_peaks()
 
-    cost = accounting.workload_cost(sets[0])
-    tokens_per_step = sets[0].n_tokens
-    set_bytes = 0
-    for wl in sets:
-        seen_x = set()
-        for c in wl.calls:
-            if _is_linear(c):
-                io = (c.X.numel() + c.W.numel() + c.Y.numel()) * 2
-            elif hasattr(c, "W"):
-                io = c.W.numel() * 2
-            else:
-                io = c.Y.numel() * 2 + (0 if c.X.data_ptr() in seen_x else c.X.numel() * 2)
-                seen_x.add(c.X.data_ptr())
-            set_bytes += c.pool.A.numel() * 2 + c.pool.B.numel() * 2 + io
-    launches_step = launches_per_step(sets[0])
-
-    # eager warm-up (also sets per-device function attributes before capture)
-    with torch.cuda.stream(stream):
-        for i in range(max(args.warmup, 3)):
-            steps[i % n_sets]()
-    stream.synchronize()
-    for ws in ws_map.values():
-        err = L.lora_get_error(ws, stream=stream)
-        if err:
-            raise SystemExit(f"device error {err} during warm-up")
-
-    # one graph = one pass over every input set
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g, stream=stream):
-        for s in steps:
-            s()
-    reps = max(1, (args.steps + n_sets - 1) // n_sets)
-    K = reps * n_sets
-    # CUDAGraph.replay() launches on the current stream: make it the timed stream
-    with torch.cuda.stream(stream):
-        for _ in range(2):
-            g.replay()
-    torch.cuda.synchronize()
-
+    bench = Bench(args.workload, dev, rank, stream, max_sets=args.sets)
+    bench.warm(args.warmup)
+    K = args.steps
+    bench.capture(K)
     clocks = ClockSampler(local).start()
     time.sleep(0.25)
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
     t_wall0 = time.time()
-    with torch.cuda.stream(stream):
-        e0.record(stream)
-        for _ in range(reps):
-            g.replay()
-        e1.record(stream)
-    torch.cuda.synchronize()
+    ms_local = bench.timed(1)
     t_wall1 = time.time()
     if dist is not None:
         dist.barrier()
     clocks.stop()
-    ms_local = e0.elapsed_time(e1)
-    ms_per_step, job_tokens_s = job_time_and_throughput(ms_local, K, tokens_per_step, world, dist, dev)
+    bench.check_errors()
+    ms_per_step, job_tokens_s = job_time_and_throughput(ms_local, K, bench.tokens, world, dist, dev)
+    clk = clocks.summary(t_wall0, t_wall1)
 
     # end to end through the public call, host buffers, copies inside the timed region
-    e2e = run_e2e(args, sets, ws_map, stream, dist, dev, world)
+    e2e = run_e2e(args, bench.sets, bench.ws_map, stream, dist, dev, world)
 
-    peaks, peak_src = load_peaks()
+    roof = roofline_of(args.workload, bench.cost, ms_per_step, clk, peaks, peak_src)
+    roof["scope"] = "whole step (one pass of the path), algorithmic bytes per step / step time"
     t_step = ms_per_step * 1e-3
-    gbs = cost.bytes / t_step / 1e9
-    tflops = cost.flops / t_step / 1e12
-    clk = clocks.summary(t_wall0, t_wall1)
-    if any(_is_linear(c) for c in sets[0].calls):
-        # a dense projection: tensor-bound.  Peak: the burst cuBLAS figure while the SM clock
-        # stayed near its maximum over the timed region, the sustained (power-capped) one
-        # once it fell below 85 % of it
-        capped = (clk.get("sm_mhz") or 0) < 0.85 * (clk.get("sm_max_mhz") or 1)
-        key = "bf16_tflops_sustained" if capped else "bf16_tflops"
-        pk = peaks.get(key, peaks["bf16_tflops"])
-        roof = {"bound": "tensor", "achieved": round(tflops, 1), "peak": pk, "unit": "TFLOP/s",
-                "frac": round(tflops / pk, 4), "traffic": NCU_TRAFFIC.get(args.workload),
-                "peak_source": f"{peak_src} (MEASURED_PEAKS.json {key})" if peak_src == "measured" else "fallback",
-                "scope": "whole step, algorithmic FLOPs per step / step time",
-                "algorithmic_flops_per_step": cost.flops, "algorithmic_bytes_per_step": cost.bytes}
-    else:
-        roof = {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": NCU_TRAFFIC.get(args.workload),
-                "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else "fallback",
-                "scope": "whole step, algorithmic bytes per step / step time",
-                "algorithmic_bytes_per_step": cost.bytes}
     out = {
         "metric": METRIC, "value": round(job_tokens_s, 1), "unit": unit_of(args.workload),
         "n_gpus": world, "steps": K, "warmup": max(args.warmup, 3), "ms_per_step": round(ms_per_step, 6),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded; random-init adapters of the stated shapes)",
-        "config": {"workload": WORKLOAD_DESC[args.workload], "tokens_per_step_per_gpu": tokens_per_step,
-                   "parallelism": f"dp{world} (independent batches per GPU, no collective)",
-                   "l2": f"rotating {n_sets} independent input sets ({set_bytes / 1e6:.0f} MB > 126 MB L2)",
-                   "timing": "CUDA-graph replays of all input sets, CUDA events on the launching stream"},
-        "hbm_gbs": round(gbs, 1), "tflops": round(tflops, 3),
+        "config": config_of(args.workload, bench.tokens, world),
+        "timing": {"l2": f"inputs larger than L2: {len(bench.sets)} independent input sets rotated "
+                         f"({len(bench.sets) * bench.set_bytes / 1e6:.0f} MB in total > 126 MB L2)",
+                   "method": "one CUDA graph holding the K steps (input sets rotated), replayed once; "
+                             "CUDA events on the launching stream, max over ranks"},
+        "hbm_gbs": round(bench.cost.bytes / t_step / 1e9, 1), "tflops": round(bench.cost.flops / t_step / 1e12, 3),
         "roofline": roof,
-        "gpu_launches": K * launches_step,
+        "gpu_launches": K * bench.launches,
         "clocks": clk,
         "e2e": e2e,
     }
+    bench.release()
+    del bench
+    if args.workloads != "none":
+        names = ALL_WORKLOADS if args.workloads == "all" else args.workloads.split(",")
+        out["workloads"] = {n: time_one_workload(n, dev, rank, stream, args, peaks, peak_src, dist, world)
+                            for n in names}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(args, sets[0], budget_s=args.cpu_seconds)
+        import gc
+        gc.collect()
+        wl0 = build_sets(args.workload, dev, rank, 1)[0]
+        out["cpu_baseline"] = cpu_baseline(args, wl0, budget_s=args.cpu_seconds)
+        del wl0
     if rank == 0:
         print(json.dumps(out), flush=True)
-    del g
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def time_one_workload(name, dev, rank, stream, args, peaks, peak_src, dist, world):
+    """One workload of the table, timed in this run: its own input sets, warm-up,
+    enough graph replays for a timed region of about 0.2 s (at least --steps),
+    clocks sampled over that region."""
+    import torch
+    b = Bench(name, dev, rank, stream, max_sets=args.sets)
+    b.warm(args.warmup)
+    b.capture(len(b.sets))
+    est = b.timed(1) / b.graph_steps
+    # a graph of up to 2000 steps, replayed for a timed region of about 0.2 s
+    per_graph = int(max(len(b.sets), min(2000, args.steps)))
+    replays = int(max(1, min(200, 200.0 / max(est * per_graph, 1e-4))))
+    b.capture(per_graph)
+    steps = per_graph * replays
+    clocks = ClockSampler(dev.index if dev.index is not None else 0).start()
+    time.sleep(0.25)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = time.time()
+    ms = b.timed(replays)
+    t1 = time.time()
+    if dist is not None:
+        dist.barrier()
+    clocks.stop()
+    b.check_errors()
+    ms_per_step, tok_s = job_time_and_throughput(ms, steps, b.tokens, world, dist, dev)
+    clk = clocks.summary(t0, t1)
+    roof = roofline_of(name, b.cost, ms_per_step, clk, peaks, peak_src)
+    res = {"desc": WORKLOAD_DESC[name], "ms_per_step": round(ms_per_step, 6),
+           "value": round(tok_s, 1), "unit": unit_of(name), "steps": steps,
+           "tokens_per_step_per_gpu": b.tokens,
+           "algorithmic_bytes_per_step": b.cost.bytes, "algorithmic_flops_per_step": b.cost.flops,
+           "hbm_gbs": round(b.cost.bytes / (ms_per_step * 1e-3) / 1e9, 1),
+           "tflops": round(b.cost.flops / (ms_per_step * 1e-3) / 1e12, 3),
+           "roofline": roof, "gpu_launches_per_step": b.launches, "clocks": clk,
+           "input_sets": len(b.sets), "input_bytes": len(b.sets) * b.set_bytes}
+    b.release()
+    del b
+    return res
 
 
 def run_e2e(args, sets, ws_map, stream, dist, dev, world):
@@ -633,11 +788,31 @@ def cpu_baseline(args, wl, budget_s=12.0):
         tokens += _oracle_pass(oracle, hc, _rows_sample(hc, n_tok, passes + 1))
         passes += 1
     dt = time.perf_counter() - t0
-    return {"value": round(tokens / dt, 2), "unit": unit_of(args.workload), "cores": oracle.threads(),
-            "kind": "oracle",
-            "sample": f"{tokens} tokens ({n_tok} sampled rows x {passes} passes) of one "
-                      f"{args.workload} batch, all projections, fp64 C loops, OpenMP over rows",
-            "seconds": round(dt, 2)}
+    out = {"value": round(tokens / dt, 2), "unit": unit_of(args.workload), "cores": oracle.threads(),
+           "kind": "oracle",
+           "sample": f"{tokens} tokens ({n_tok} sampled rows x {passes} passes) of one "
+                     f"{args.workload} batch, all projections, fp64 C loops, OpenMP over rows",
+           "seconds": round(dt, 2)}
+    # one host thread on the tiny and decode workloads (the whole batch per pass)
+    one = {}
+    oracle.set_threads(1)
+    try:
+        from workloads import make_workload, WORKLOAD_NAMES
+        for name in ("tiny_sgmv", "decode_bgmv"):
+            idx = WORKLOAD_NAMES.index(name)
+            w = make_workload(idx, device=wl.calls[0].pool.A.device, seed=rank_seed(idx, 0, 0))
+            h = _host_calls(w)
+            rows = [np.arange(w.n_tokens, dtype=np.int32) for _ in h]
+            _oracle_pass(oracle, h, rows)
+            n, t0 = 0, time.perf_counter()
+            while time.perf_counter() - t0 < args.one_thread_seconds:
+                n += _oracle_pass(oracle, h, rows)
+            one[name] = {"value": round(n / (time.perf_counter() - t0), 2), "unit": "tokens/s", "cores": 1,
+                         "sample": f"whole {name} batch ({w.n_tokens} tokens) per pass"}
+    finally:
+        oracle.set_threads(os.cpu_count() or 1)
+    out["one_thread"] = one
+    return out
 
 
 def run_reference(args):
@@ -677,7 +852,8 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / max(args.steps, 1) * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded)",
-        "config": {"workload": WORKLOAD_DESC[args.workload], "tokens_per_step": n_tok},
+        "config": config_of(args.workload, wl.n_tokens, args.gpus),
+        "sample": f"{n_tok} token rows per step",
         "cpu_baseline": {"value": round(v, 3), "unit": unit_of(args.workload), "cores": oracle.threads(),
                          "kind": "oracle",
                          "sample": sample},
@@ -697,8 +873,18 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--reference-seconds", type=float, default=60.0)
+    ap.add_argument("--one-thread-seconds", type=float, default=3.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workloads", default="all",
+                    help="'all', 'none' or a comma list: workloads timed in the same run next to the headline")
+    ap.add_argument("--only-proj", default=None,
+                    help="mixed_rank_layer only: keep just these projections (comma list, e.g. 'gate'); "
+                         "for profiling one kernel on a smaller device footprint")
     args = ap.parse_args(argv)
+    if args.only_proj:
+        from workloads.configs import LLAMA3_8B_PROJ
+        keep = args.only_proj.split(",")
+        OVERRIDES["mixed_rank_layer"] = {"projections": [p for p in LLAMA3_8B_PROJ if p[0] in keep]}
     if args.impl == "reference":
         run_reference(args)
     else:

@@ -138,8 +138,10 @@ LORA_API size_t lora_workspace_size(int op, int32_t N, int32_t n_adapters, int32
  * lora_sgmv_apply_proj). */
 LORA_API int lora_kernel_launches(int op, int32_t N, int32_t n_adapters, int32_t d_in, int32_t n_items);
 
-/* Clear the workspace's error word (cudaMemsetAsync of its 256-byte header on
- * `stream`).  Call once on a fresh workspace. */
+/* Clear the workspace's header (cudaMemsetAsync of its first 4096 bytes on
+ * `stream`): the error word and the progress counters the decode kernel of
+ * lora_bgmv keeps there.  Call once on a fresh workspace, unless the memory is
+ * already zero; the library keeps the header consistent from then on. */
 LORA_API lora_status lora_workspace_init(void *ws, void *stream);
 
 /* Synchronise `stream`, read the workspace's error word, clear it, and return
@@ -169,11 +171,15 @@ LORA_API lora_status lora_route(const int32_t *ids, int32_t N, int32_t n_adapter
  * lora_bgmv -- decode: one token per request, each with its own adapter.
  *   Y[n] += scale * B[ids[n]] A[ids[n]] X[n]   for ids[n] != -1
  * ids: device int32 [N], unsorted, -1 = no adapter (row untouched).  The
- * grouping runs inside the call, so every distinct adapter's A and B are
- * streamed from HBM once per group of up to 8 tokens sharing it.  For
- * N <= 8192, n_adapters <= 8192 and d_in <= 32768 the whole call is one
- * kernel launch (thread-block clusters of 8 CTAs; only the workspace's error
- * word is used); larger calls take a three-kernel path through the workspace.
+ * grouping runs inside the call: tokens are sorted stably by adapter and cut
+ * into items of up to 16 tokens, and each item's A and B rows cross HBM once
+ * (the items of one adapter re-read them from L2).  The whole call is one
+ * kernel launch when the grouping fits the kernel's shared memory (about
+ * N <= 2000 tokens with up to a few thousand adapters): the rank-r partial
+ * products go through the workspace, and the kernel's CTAs hand them over with
+ * progress counters kept in the workspace header, so calls sharing a workspace
+ * must not overlap on the GPU.  Larger calls take a three-kernel path through
+ * the workspace.
  */
 LORA_API lora_status lora_bgmv(const void *X, int64_t ldx, void *Y, int64_t ldy, const lora_pool *pool,
                       const int32_t *ids, int32_t N, float scale,
@@ -249,9 +255,10 @@ LORA_API lora_status lora_sgmv_apply_proj(const void *X, int64_t ldx, void *cons
  * W: device bf16 [d_out, d_in] row-major (a torch Linear weight), leading
  * dimension ldw >= d_in, multiple of 8, 16-byte aligned; X [N, ldx] and
  * Y [N, ldy] as elsewhere; pool->d_in / d_out give the projection's shape.
- * Adapters in the LoRA part must have rank 16, 32, 64 or 128 with B_off[a]
- * a multiple of the rank (what a packed pool of those ranks gives); a segment
- * whose adapter fails this or the usual device checks gets Y = W X and sets
+ * Adapters may have any rank the pool allows (a multiple of 8 up to
+ * max_rank): B is read through a tensor map when the rank is 16, 32, 64 or 128
+ * and B_off[a] a multiple of it, and gathered with 16-byte copies otherwise.
+ * A segment whose adapter fails the usual device checks gets Y = W X and sets
  * LORA_ERR_BAD_ADAPTER.  Workspace: lora_workspace_size(LORA_OP_LINEAR, N,
  * n_adapters, d_in, d_out, max_rank, n_seg, 0) (it holds s V).  Launches
  * three kernels (plan, tcgen05 shrink, tcgen05 projection).  Needs the
@@ -389,6 +396,39 @@ LORA_API lora_status lora_pm_register(lora_pool_mgr *m, int64_t key, const void 
                                       int32_t rank);
 LORA_API lora_status lora_pm_acquire(lora_pool_mgr *m, const int64_t *keys, int32_t n, int32_t *slots,
                                      int32_t *n_loaded, void *stream);
+
+/*
+ * Co-occurrence preloading ("Co-occurrence Patterns of LoRA Adapters in
+ * Production Diffusion Model Inference Services", abstract: requests that
+ * combine adapters do so in recurring patterns, and preloading the top-k
+ * co-occurring adapters covers most of them).
+ *
+ * lora_pm_observe: records one request's adapter keys[0..n) (duplicates count
+ *   once): every pair of distinct keys in it co-occurred once more.  Host only.
+ * lora_pm_set_preload: top_k > 0 makes every later lora_pm_acquire, after the
+ *   batch's own keys, also bring in the top_k partners of each batch key (most
+ *   requests in common first, ties to the smaller key) that are registered, not
+ *   resident and not in the batch -- into free slots, else least recently used
+ *   slots that no key of this acquire holds, until none is left; the copies go
+ *   on the acquire's stream like the batch's own.  0 (the default) turns it off.
+ * lora_pm_preloaded: adapters the last acquire preloaded (-1 for a NULL manager).
+ */
+LORA_API lora_status lora_pm_observe(lora_pool_mgr *m, const int64_t *keys, int32_t n);
+LORA_API lora_status lora_pm_set_preload(lora_pool_mgr *m, int32_t top_k);
+LORA_API int32_t lora_pm_preloaded(lora_pool_mgr *m);
+
+/*
+ * lora_test_stall -- testing hook for the timeout path (no counterpart on the
+ * pages).  While `stall` is non-zero, the kernels that stream their operands
+ * through a load pipeline (the decode kernel of lora_bgmv and the tensor-core
+ * kernels of the SGMV, multi-adapter, projection and merge calls) issue no loads
+ * at all, and every wait inside a kernel gives up after `wait_seconds`
+ * (clamped to [1 us, 2 s]): such a call changes none of its outputs, reports
+ * LORA_ERR_TIMEOUT through lora_get_error, and leaves the device ready for the
+ * next call.  stall = 0 restores normal operation (waits bounded by 2 s).
+ * Process-wide; not for production use.
+ */
+LORA_API void lora_test_stall(int stall, double wait_seconds);
 
 LORA_API const char *lora_version(void);
 

@@ -52,22 +52,32 @@ def test_linear_ragged(d_in, d_out):
     assert np.all(got[outside] == 1.0)
 
 
-def test_linear_rank_outside_the_fused_views_is_reported():
-    """Rank 24 (a multiple of 8, valid for the delta kernels) has no B view in the fused
-    projection: its segments get the base product alone and LORA_ERR_BAD_ADAPTER."""
-    rng = np.random.default_rng(3)
+@pytest.mark.parametrize("scatter", [False, True])
+def test_linear_any_rank_multiple_of_8(scatter):
+    """Ranks 8, 24, 40, 96 and 120 (no pool view: B gathered row by row) next to
+    16/64/128 (views), mixed in one call -- and, on a scattered pool (offsets no
+    longer multiples of the rank), every adapter through the gather -- against the
+    oracle's x (W + s B_a A_a)^T."""
+    from helpers import scatter_pool
+    rng = np.random.default_rng(3 + scatter)
     d_in, d_out = 192, 264
-    hp = rand_host_pool(rng, [32, 24, 64], d_in, d_out)
-    seg_off = np.array([0, 200, 330, 500], np.int32)
-    ads = np.array([0, 1, 2], np.int32)
-    N = 500
+    ranks = [8, 24, 40, 16, 96, 64, 120, 128]
+    hp = rand_host_pool(rng, ranks, d_in, d_out)
+    if scatter:
+        hp = scatter_pool(hp)
+    lens = [130, 200, 64, 150, 129, 90, 200, 140]
+    seg_off = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    ads = np.arange(len(ranks), dtype=np.int32)
+    N = int(seg_off[-1])
     X = rand_x(rng, N, d_in)
     W = _rand_w(rng, d_out, d_in)
     Y = torch.zeros((N, d_out), dtype=torch.bfloat16, device=DEV)
-    ws = L.lora_linear_sgmv(dev_bf16(X), dev_bf16(W), Y, DevPool(hp), _i32(seg_off), _i32(ads), 1.0)
-    assert L.lora_get_error(ws) == 4                          # LORA_ERR_BAD_ADAPTER
-    want = oracle.linear_sgmv(X, W, hp, seg_off, np.array([0, -1, 2], np.int32), 1.0)
-    check_parity(widen(to_host(Y)), want, "linear, rank 24 segment base only")
+    ws = L.lora_linear_sgmv(dev_bf16(X), dev_bf16(W), Y, DevPool(hp), _i32(seg_off), _i32(ads), 1.5)
+    assert L.lora_get_error(ws) == 0
+    want = oracle.linear_sgmv(X, W, hp, seg_off, ads, 1.5)
+    got = widen(to_host(Y))
+    check_parity(got, want, f"linear, ranks {ranks} scatter={scatter}")
+    check_rounded(got, want, f"linear, ranks {ranks} scatter={scatter}")
 
 
 def test_linear_scale_zero_and_no_adapter_are_the_base_product():
