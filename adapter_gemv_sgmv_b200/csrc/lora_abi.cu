@@ -320,7 +320,7 @@ int lora_kernel_launches(int op, int32_t N, int32_t n_adapters, int32_t d_in, in
         return 0;
     switch (op) {
     case LORA_OP_BGMV:
-        return stream_bgmv_supported(N, n_adapters) || fused_bgmv_supported(N, n_adapters, d_in) ? 1 : 3;
+        return fused_bgmv_supported(N, n_adapters, d_in) ? 1 : 3;
     case LORA_OP_SGMV_SHRINK:
     case LORA_OP_SGMV_EXPAND:
         return n_items > 0 ? 2 : 0;
@@ -408,30 +408,6 @@ lora_status lora_bgmv(const void *X, int64_t ldx, void *Y, int64_t ldy, const lo
         return LORA_OK;
     cudaStream_t s = (cudaStream_t)stream;
     WsHeader *hdr = at<WsHeader>(ws, L.hdr);
-    if (stream_bgmv_supported(N, pool->n_adapters)) {
-        StreamBgmvArgs sa = {};
-        sa.X = static_cast<const __nv_bfloat16 *>(X);
-        sa.ldx = ldx;
-        sa.Y = static_cast<__nv_bfloat16 *>(Y);
-        sa.ldy = ldy;
-        sa.ids = ids;
-        sa.N = N;
-        sa.pool = pool_dev(pool);
-        sa.scale = scale;
-        sa.V = at<float>(ws, L.V);
-        sa.ldv = pool->max_rank;
-        sa.plane = (int64_t)N * pool->max_rank;
-        sa.max_parts = L.n_chunks;
-        sa.hdr = hdr;
-        sa.test_stall = test_stall_mode();
-        sa.wait_ns = wait_bound_ns();
-        const cudaError_t e = launch_bgmv_stream(sa, s, pdl_enabled());
-        if (e == cudaSuccess)
-            return LORA_OK;
-        if (e != cudaErrorNotSupported)
-            return LORA_ERR_CUDA;
-        // the kernel does not fit this device: the kernels below take the call
-    }
     if (fused_bgmv_supported(N, pool->n_adapters, pool->d_in)) {
         FusedBgmvArgs fa = {};
         fa.X = static_cast<const __nv_bfloat16 *>(X);

@@ -18,22 +18,16 @@ constexpr int kExpandPerThread = 8;  // consecutive outputs per thread in the ex
 constexpr int kExpandTile = kThreads * kExpandPerThread;
 constexpr int kBgmvChunk = 512;      // split of d_in across CTAs in the decode shrink
 
-constexpr int kMaxStreamCtas = 504;  // CTAs of the streamed decode kernel (progress slots in the header)
 constexpr unsigned long long kWaitBoundNs = 2000000000ull;   // bound of any single wait in a kernel (2 s)
 
-// Head of every workspace (4096 bytes, zeroed by lora_workspace_init).
+// Head of every workspace (256 bytes).
 struct WsHeader {
     uint32_t err;       // device error bits (lora_status values), sticky until lora_get_error
     int32_t n_seg;      // distinct adapters found by the grouping
     int32_t n_groups;   // work groups written by the plan kernel
-    uint32_t epoch;     // streamed decode: calls completed on this workspace
-    uint32_t done;      // streamed decode: CTAs of the running call that have finished
-    int32_t pad[11];
-    // streamed decode: shrink units finished by each CTA of the running call,
-    // tagged with the call's epoch in the high 32 bits
-    unsigned long long progress[kMaxStreamCtas];
+    int32_t pad[61];
 };
-static_assert(sizeof(WsHeader) == 4096, "header is 4096 bytes");
+static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
 
 // A run of at most kGroup tokens that share one item (segment or request).
 // Tokens are positions p0 .. p0+cnt-1: row indices, or indices into perm.
@@ -219,38 +213,6 @@ struct FusedBgmvArgs {
 };
 
 size_t fused_smem_bytes(int32_t N, int32_t n_adapters, int32_t max_rank, int32_t Wo);
-
-// ------------------------------------- streamed decode (one launch, bulk copies)
-constexpr int kStreamMaxTokens = 8192;
-constexpr size_t kStreamMaxSmem = 224 * 1024;   // dynamic; the static shared variables fit beside it
-constexpr int kStreamMaxSlots = 6;
-constexpr int kStreamMinSlots = 3;
-
-struct StreamBgmvArgs {
-    CUtensorMap map_a;         // the A pool as [A_elems / d_in, d_in], boxes of 256 columns x 16 rows (set by the launcher)
-    int32_t a_tma;             // map_a is valid
-    const __nv_bfloat16 *X;
-    int64_t ldx;
-    __nv_bfloat16 *Y;
-    int64_t ldy;
-    const int32_t *ids;
-    int32_t N;
-    PoolDev pool;
-    float scale;
-    float *V;                  // workspace: planes of the rank-r partials, [plane][token][ldv] fp32
-    int64_t ldv;               // max_rank
-    int64_t plane;             // N * ldv
-    int32_t max_parts;         // planes the workspace holds
-    WsHeader *hdr;
-    int32_t n_slots;           // set by the launcher
-    int32_t test_stall;        // the producer issues nothing (tests the timeout path)
-    unsigned long long wait_ns;  // bound of every wait
-};
-
-// Grid of the streamed decode kernel for this batch (0 if its shared memory does not fit).
-int stream_grid(int32_t N, int32_t n_adapters, int *n_slots_out, size_t *smem_out);
-bool stream_bgmv_supported(int32_t N, int32_t n_adapters);
-cudaError_t launch_bgmv_stream(const StreamBgmvArgs &a, cudaStream_t s, bool pdl);
 bool fused_bgmv_supported(int32_t N, int32_t n_adapters, int32_t d_in);
 cudaError_t launch_bgmv_fused(const FusedBgmvArgs &a, cudaStream_t s, bool pdl);
 bool pdl_enabled();

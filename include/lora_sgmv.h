@@ -138,10 +138,8 @@ LORA_API size_t lora_workspace_size(int op, int32_t N, int32_t n_adapters, int32
  * lora_sgmv_apply_proj). */
 LORA_API int lora_kernel_launches(int op, int32_t N, int32_t n_adapters, int32_t d_in, int32_t n_items);
 
-/* Clear the workspace's header (cudaMemsetAsync of its first 4096 bytes on
- * `stream`): the error word and the progress counters the decode kernel of
- * lora_bgmv keeps there.  Call once on a fresh workspace, unless the memory is
- * already zero; the library keeps the header consistent from then on. */
+/* Clear the workspace's error word (cudaMemsetAsync of its 256-byte header on
+ * `stream`).  Call once on a fresh workspace. */
 LORA_API lora_status lora_workspace_init(void *ws, void *stream);
 
 /* Synchronise `stream`, read the workspace's error word, clear it, and return
@@ -173,13 +171,11 @@ LORA_API lora_status lora_route(const int32_t *ids, int32_t N, int32_t n_adapter
  * ids: device int32 [N], unsorted, -1 = no adapter (row untouched).  The
  * grouping runs inside the call: tokens are sorted stably by adapter and cut
  * into items of up to 16 tokens, and each item's A and B rows cross HBM once
- * (the items of one adapter re-read them from L2).  The whole call is one
- * kernel launch when the grouping fits the kernel's shared memory (about
- * N <= 2000 tokens with up to a few thousand adapters): the rank-r partial
- * products go through the workspace, and the kernel's CTAs hand them over with
- * progress counters kept in the workspace header, so calls sharing a workspace
- * must not overlap on the GPU.  Larger calls take a three-kernel path through
- * the workspace.
+ * (the items of one adapter re-read them from L2).  For N <= 8192,
+ * n_adapters <= 8192 and d_in <= 32768 (and a grouping that fits the kernel's
+ * shared memory) the whole call is one kernel launch (thread-block clusters of
+ * 8 CTAs; only the workspace's error word is used); larger calls take a
+ * three-kernel path through the workspace.
  */
 LORA_API lora_status lora_bgmv(const void *X, int64_t ldx, void *Y, int64_t ldy, const lora_pool *pool,
                       const int32_t *ids, int32_t N, float scale,
@@ -420,8 +416,8 @@ LORA_API int32_t lora_pm_preloaded(lora_pool_mgr *m);
 /*
  * lora_test_stall -- testing hook for the timeout path (no counterpart on the
  * pages).  While `stall` is non-zero, the kernels that stream their operands
- * through a load pipeline (the decode kernel of lora_bgmv and the tensor-core
- * kernels of the SGMV, multi-adapter, projection and merge calls) issue no loads
+ * through a load pipeline (the tensor-core kernels of the SGMV, multi-adapter,
+ * projection and merge calls) issue no loads
  * at all, and every wait inside a kernel gives up after `wait_seconds`
  * (clamped to [1 us, 2 s]): such a call changes none of its outputs, reports
  * LORA_ERR_TIMEOUT through lora_get_error, and leaves the device ready for the

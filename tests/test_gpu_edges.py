@@ -217,3 +217,51 @@ def test_bgmv_three_kernel_path_beyond_fused_limits(N, n_ad):
     ws = L.lora_bgmv(dev_bf16(X), Y, DevPool(hp), _i32(ids), 0.5)
     assert L.lora_get_error(ws) == 0
     check_parity(_f64(Y), widen(Y0) + oracle.bgmv_delta(X, hp, ids, 0.5), f"3-kernel bgmv N={N}")
+
+
+def test_output_ties_round_to_even():
+    """Outputs that land exactly halfway between two bf16 values come back rounded to
+    the even one (round to nearest even), through the decode path and the tensor-core
+    SGMV path.  A[a] row 0 holds (256, v1) so v_0 = 256 + v1 exactly; B[a][o][0] = 1;
+    scale 2^-8: y = y0 + (256 + v1) / 256, with v1 = 1 giving 1 + 2^-8 (a tie, even
+    neighbour 1.0) and v1 = 3 giving 1 + 3 * 2^-8 (a tie, even neighbour 1 + 2^-6)."""
+    from workloads import bf16_bits
+    d_in, d_out, r = 64, 48, 8
+    ranks = np.array([r, r], np.int32)
+    A = np.zeros((2, r, d_in), np.float32)
+    A[0, 0, 0], A[0, 0, 1] = 256.0, 1.0
+    A[1, 0, 0], A[1, 0, 1] = 256.0, 3.0
+    B = np.zeros((2, d_out, r), np.float32)
+    B[:, :, 0] = 1.0
+    hp = oracle.HostPool(A=bf16_bits(A.reshape(-1)), B=bf16_bits(B.reshape(-1)),
+                         A_off=np.array([0, r * d_in], np.int64), B_off=np.array([0, r * d_out], np.int64),
+                         rank=ranks, d_in=d_in, d_out=d_out)
+    N = 300
+    X = np.zeros((N, d_in), np.float32)
+    X[:, 0] = X[:, 1] = 1.0
+    Xb = bf16_bits(X)
+    ids = (np.arange(N) % 2).astype(np.int32)
+    want = np.where(ids[:, None] == 0, 1.0, 1.0 + 2.0 ** -6) * np.ones((1, d_out))
+    # y0 = 0: the delta itself is the tie
+    Y = torch.zeros(N, d_out, dtype=torch.bfloat16, device=DEV)
+    ws = L.lora_bgmv(dev_bf16(Xb), Y, DevPool(hp), _i32(ids), 2.0 ** -8)
+    assert L.lora_get_error(ws) == 0
+    assert np.array_equal(_f64(Y), want)
+    # the same through the SGMV tensor-core path (segments of 150 rows)
+    order = np.argsort(ids, kind="stable")
+    seg_off = np.array([0, 150, 300], np.int32)
+    Xs = Xb[order]
+    V = torch.zeros(N, r, dtype=torch.float32, device=DEV)
+    ws = L.lora_sgmv_shrink(dev_bf16(Xs), V, DevPool(hp), _i32(seg_off), _i32([0, 1]))
+    assert L.lora_get_error(ws) == 0
+    Y = torch.zeros(N, d_out, dtype=torch.bfloat16, device=DEV)
+    ws = L.lora_sgmv_expand(V, Y, DevPool(hp), _i32(seg_off), _i32([0, 1]), 2.0 ** -8)
+    assert L.lora_get_error(ws) == 0
+    assert np.array_equal(_f64(Y), want[order])
+    # a nonzero y0 in the same pass: y = -2 - (256 + v1) / 256, rounded once
+    Y0 = np.full((N, d_out), bf16_bits(np.float32(-2.0)), np.uint16)
+    Y = dev_bf16(Y0)
+    ws = L.lora_bgmv(dev_bf16(Xb), Y, DevPool(hp), _i32(ids), -2.0 ** -8)
+    assert L.lora_get_error(ws) == 0
+    exact = -2.0 - np.where(ids[:, None] == 0, 257.0, 259.0) / 256.0 * np.ones((1, d_out))
+    assert np.array_equal(_f64(Y), oracle.round_bf16(exact))
