@@ -12,8 +12,14 @@
 // * every CTA rebuilds the grouping in shared memory (ids -> per-adapter
 //   counts -> exclusive scan of groups per adapter); item k is the k-th
 //   (adapter, group of up to 16 tokens) pair in adapter order.  Clusters are
-//   persistent: the grid holds as many clusters as fit on the GPU at once and
-//   cluster c takes items c, c + n_clusters, ...
+//   persistent: the grid holds as many clusters as fit on the GPU at once.  The
+//   items are dealt out heaviest first: ordered by rank class (ranks 65-128,
+//   33-64, 17-32, 8-16; adapter order inside a class), round k of the clusters
+//   takes positions k * n_clusters .. in alternating direction (cluster c gets
+//   positions c, 2 n_clusters - 1 - c, 2 n_clusters + c, ...), so that a cluster
+//   with a heavy first item gets a light second one.  With cluster c taking
+//   items c, c + n_clusters, ... instead, the mixed-rank gate projection (about
+//   230 items on 86 clusters) ran 1.6x longer than its average cluster load.
 // * an item is a 16-row tile of tokens, so both halves are tiny dense
 //   contractions done with warp-level tensor-core MMAs (m16n8k16, bf16 in,
 //   fp32 accumulate): with CUDA-core FMAs the instruction issue, not HBM,
@@ -139,6 +145,16 @@ __device__ __forceinline__ bool adapter_ok(const PoolDev &P, int32_t a, int32_t 
     *aoff = ao;
     *boff = bo;
     return true;
+}
+
+// Scheduling class of adapter a by rank (its L2 copy of the metadata is warm):
+// 3 for ranks 65-128 .. 0 for 8-16 and for an adapter that fails its checks.
+__device__ __forceinline__ int rank_class(const PoolDev &P, int a)
+{
+    const int r = __ldg(P.rank + a);
+    if (r < 8 || r > P.max_rank || (r & 7))
+        return 0;
+    return r <= 16 ? 0 : r <= 32 ? 1 : r <= 64 ? 2 : 3;
 }
 
 // Shrink of one warp: NT rank tiles (8 ranks each, from rank tile nt0) over
@@ -352,6 +368,7 @@ __global__ void __launch_bounds__(kFThreads, 5) k_bgmv_fused(FusedBgmvArgs p)
     const FusedSmem L = fused_smem_layout(p.N, p.pool.n_adapters, p.pool.max_rank, p.Wo);
     const int vs = L.vs;
     int16_t *item_ad = reinterpret_cast<int16_t *>(sm_raw + L.items);   // adapter of items < L.n_tab
+    int16_t *order = reinterpret_cast<int16_t *>(sm_raw + L.order);    // item at each schedule position
     const int mr = p.pool.max_rank < kMaxRank ? p.pool.max_rank : kMaxRank;
     int32_t *ids_s = reinterpret_cast<int32_t *>(sm_raw + L.ids);
     int32_t *ipre = reinterpret_cast<int32_t *>(sm_raw + L.cnt);    // [n_ad + 1]
@@ -366,6 +383,7 @@ __global__ void __launch_bounds__(kFThreads, 5) k_bgmv_fused(FusedBgmvArgs p)
     __shared__ int32_t s_ad, s_g, s_cnt, s_bad, s_r;
     __shared__ int64_t s_aoff, s_boff;
     __shared__ int32_t sm_scan[kFWarps + 1];
+    __shared__ unsigned long long sm_cls[kFWarps + 1];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, qd = lane & 3;    // MMA fragment row group and quad position
@@ -403,38 +421,72 @@ __global__ void __launch_bounds__(kFThreads, 5) k_bgmv_fused(FusedBgmvArgs p)
     __syncthreads();
     PHASE(1);
     {
-        // counts -> exclusive prefix of groups per adapter, ipre[n_ad] = total
+        // counts -> exclusive prefix of groups per adapter, ipre[n_ad] = total; and the
+        // same prefix per rank class (four 16-bit fields of one 64-bit scan: class 3 =
+        // ranks 65-128 .. class 0 = ranks 8-16, or an adapter that fails its checks)
         const int per = (n_ad + kFThreads - 1) / kFThreads;
         const int b = tid * per, e = min(n_ad, b + per);
         int local = 0;
-        for (int a = b; a < e; ++a)
-            local += (ipre[a] + kFT - 1) / kFT;
+        unsigned long long lcls = 0;
+        for (int a = b; a < e; ++a) {
+            const int gr = (ipre[a] + kFT - 1) / kFT;
+            local += gr;
+            if (gr)
+                lcls += (unsigned long long)gr << (16 * rank_class(p.pool, a));
+        }
         int incl = local;
+        unsigned long long icls = lcls;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
             const int v = __shfl_up_sync(0xffffffffu, incl, off);
-            if (lane >= off)
+            const unsigned long long w = __shfl_up_sync(0xffffffffu, icls, off);
+            if (lane >= off) {
                 incl += v;
+                icls += w;
+            }
         }
-        if (lane == 31)
+        if (lane == 31) {
             sm_scan[warp] = incl;
+            sm_cls[warp] = icls;
+        }
         __syncthreads();
         if (tid == 0) {
             int run = 0;
+            unsigned long long runc = 0;
             for (int w = 0; w < kFWarps; ++w) {
                 const int t = sm_scan[w];
+                const unsigned long long tc = sm_cls[w];
                 sm_scan[w] = run;
+                sm_cls[w] = runc;
                 run += t;
+                runc += tc;
             }
             sm_scan[kFWarps] = run;
+            sm_cls[kFWarps] = runc;
         }
         __syncthreads();
         int run = sm_scan[warp] + incl - local;
+        unsigned long long runc = sm_cls[warp] + icls - lcls;
+        // schedule position of the first item of each class: heaviest class first
+        const unsigned long long tot = sm_cls[kFWarps];
+        int cbase[4];
+        cbase[3] = 0;
+        cbase[2] = (int)(tot >> 48);
+        cbase[1] = cbase[2] + (int)((tot >> 32) & 0xFFFF);
+        cbase[0] = cbase[1] + (int)((tot >> 16) & 0xFFFF);
         for (int a = b; a < e; ++a) {
             const int gr = (ipre[a] + kFT - 1) / kFT;
             ipre[a] = run;
-            for (int j = 0; j < gr && run + j < L.n_tab; ++j)
-                item_ad[run + j] = (int16_t)a;
+            if (gr) {
+                const int c = rank_class(p.pool, a);
+                const int pos = cbase[c] + (int)((runc >> (16 * c)) & 0xFFFF);
+                for (int j = 0; j < gr && run + j < L.n_tab; ++j) {
+                    item_ad[run + j] = (int16_t)a;
+                    if (pos + j < L.n_tab)
+                        order[pos + j] = (int16_t)(run + j);
+                }
+                runc += (unsigned long long)gr << (16 * c);
+            }
             run += gr;
         }
         if (tid == 0)
@@ -448,7 +500,14 @@ __global__ void __launch_bounds__(kFThreads, 5) k_bgmv_fused(FusedBgmvArgs p)
     const int o0 = min(d_out, (int)crank * p.Wo), o1 = min(d_out, o0 + p.Wo);
     bool waited = false;
 
-    for (int item = (int)cluster_id_x(); item < n_items; item += n_cl) {
+    // the schedule (above) needs every item in the tables; else items in index order
+    const bool sched = n_items <= L.n_tab;
+    const int cid = (int)cluster_id_x();
+    for (int rnd = 0;; ++rnd) {
+        const int pos = rnd * n_cl + ((rnd & 1) ? n_cl - 1 - cid : cid);
+        if (pos >= n_items)
+            break;
+        const int item = sched ? order[pos] : pos;
         // ---- the item's adapter, metadata and tokens (immutable inputs only)
         if (tid == 0) {
             int lo = 0;
@@ -522,14 +581,10 @@ __global__ void __launch_bounds__(kFThreads, 5) k_bgmv_fused(FusedBgmvArgs p)
             const __nv_bfloat16 *src = Ba + (int64_t)o0 * r;
             for (int c = tid; c < nch; c += kFThreads)
                 cp_async16(bst + c * 8, src + c * 8);
-        } else if (tid == 32 && o1 > o0) {   // this CTA's B chunk towards L2 (immutable input)
-            prefetch_l2(Ba + (int64_t)o0 * r, (uint32_t)((o1 - o0) * r * 2));
         }
-        // the tokens' y rows towards L2: a prefetch only fills L2, which is the
-        // point of coherence, so it cannot expose data older than a write that
-        // the previous kernel completes later
-        if (!L.staged && tid >= 32 && tid < 32 + cnt && o1 > o0)
-            prefetch_l2(p.Y + (int64_t)tok[tid - 32] * p.ldy + o0, (uint32_t)((o1 - o0) * 2));
+        // (a chunk too large to stage is not prefetched: its expand streams at the
+        // HBM rate anyway, and one bulk prefetch of a few hundred KB holds the SM's copy
+        // engine for microseconds, blocking every copy and prefetch issued after it)
         PHASE(3);
 
         // ---- shrink work split: rank tiles of 8 in groups of up to 4 per warp;
@@ -542,10 +597,17 @@ __global__ void __launch_bounds__(kFThreads, 5) k_bgmv_fused(FusedBgmvArgs p)
         const int b0 = my_kp * nblk / kparts, b1 = (my_kp + 1) * nblk / kparts;
 
         // ---- shrink: V_c[16 x r] = X_tile[16 x chunk] A[:, chunk]^T; this
-        // CTA's A rows are requested into L2 first (immutable input)
-        if (k1 > k0)
-            for (int j = tid; j < r; j += kFThreads)
-                prefetch_l2(Aa + (int64_t)j * d_in + k0, (uint32_t)((k1 - k0) * 2));
+        // CTA's A rows are requested into L2 first (immutable input), one 128-byte
+        // line per prefetch instruction (these do not queue behind bulk copies)
+        if (k1 > k0) {
+            const uint32_t lpr = (uint32_t)((k1 - k0) * 2 + 127) >> 7;    // lines per row
+            for (uint32_t e = (uint32_t)tid; e < (uint32_t)r * lpr; e += kFThreads) {
+                const uint32_t j = e / lpr, l = e - j * lpr;
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<const char *>(
+                                                            Aa + (int64_t)j * d_in + k0) + ((size_t)l << 7))
+                             : "memory");
+            }
+        }
         if (!waited) {
             pdl_trigger();
             pdl_wait();   // from here on x, y and the workspace may be touched
@@ -601,7 +663,7 @@ __global__ void __launch_bounds__(kFThreads, 5) k_bgmv_fused(FusedBgmvArgs p)
             pdl_wait();
             waited = true;
         }
-        if (s_bad && blockIdx.x == 0 && tid == 0 && item == (int)cluster_id_x())
+        if (s_bad && blockIdx.x == 0 && tid == 0 && rnd == 0)
             atomicOr(p.err, (uint32_t)LORA_ERR_BAD_ADAPTER);
         PHASE(4);
         __syncthreads();

@@ -149,8 +149,8 @@ constexpr size_t kFMaxSmem = 200 * 1024;
 constexpr int kFItemTable = 1024;   // most items whose adapter the grouping writes into a table
 
 struct FusedSmem {
-    size_t ids, cnt, items, vpart, vsum, bst, yst, total;
-    int n_tab;       // entries of the item -> adapter table (int16)
+    size_t ids, cnt, items, order, vpart, vsum, bst, yst, total;
+    int n_tab;       // entries of the item -> adapter table and of the item order (int16)
     int vs;          // bf16 row stride of the staged rank-r vectors
     bool staged;     // this CTA's B chunk and the item's y rows are copied to shared memory
 };
@@ -175,6 +175,8 @@ __host__ __device__ inline FusedSmem fused_smem_layout(int32_t N, int32_t n_adap
     const int64_t max_items = (int64_t)(N < n_adapters ? N : n_adapters) + N / kFT + 1;
     L.n_tab = (int)(max_items < kFItemTable ? max_items : kFItemTable);
     L.items = off;
+    off = fused_align16(off + 2 * (size_t)L.n_tab);
+    L.order = off;
     off = fused_align16(off + 2 * (size_t)L.n_tab);
     L.vpart = off;
     off = fused_align16(off + 4 * (size_t)mr * kFT);
