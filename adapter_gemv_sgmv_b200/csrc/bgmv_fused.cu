@@ -14,12 +14,15 @@
 //   (adapter, group of up to 16 tokens) pair in adapter order.  Clusters are
 //   persistent: the grid holds as many clusters as fit on the GPU at once.  The
 //   items are dealt out heaviest first: ordered by rank class (ranks 65-128,
-//   33-64, 17-32, 8-16; adapter order inside a class), round k of the clusters
-//   takes positions k * n_clusters .. in alternating direction (cluster c gets
-//   positions c, 2 n_clusters - 1 - c, 2 n_clusters + c, ...), so that a cluster
-//   with a heavy first item gets a light second one.  With cluster c taking
-//   items c, c + n_clusters, ... instead, the mixed-rank gate projection (about
-//   230 items on 86 clusters) ran 1.6x longer than its average cluster load.
+//   33-64, 17-32, 8-16; adapter order inside a class), cluster c starts with
+//   position c and then takes the next free position from a counter in the
+//   workspace header (rank 0 of the cluster draws it during the item and writes
+//   it into every CTA of the cluster before the cluster barrier that ends the
+//   item).  With cluster c taking items c, c + n_clusters, ... instead, the
+//   mixed-rank gate projection (about 230 items on 86 clusters) ran 1.6x longer
+//   than its average cluster load.  The last cluster to finish puts the counter
+//   back to zero; a launch draws from it only after griddepcontrol.wait, i.e.
+//   after the previous launch on the stream has finished.
 // * an item is a 16-row tile of tokens, so both halves are tiny dense
 //   contractions done with warp-level tensor-core MMAs (m16n8k16, bf16 in,
 //   fp32 accumulate): with CUDA-core FMAs the instruction issue, not HBM,
@@ -384,6 +387,7 @@ __global__ void __launch_bounds__(kFThreads, 5) k_bgmv_fused(FusedBgmvArgs p)
     __shared__ int64_t s_aoff, s_boff;
     __shared__ int32_t sm_scan[kFWarps + 1];
     __shared__ unsigned long long sm_cls[kFWarps + 1];
+    __shared__ int s_next;          // the cluster's next schedule position (written by cluster rank 0)
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, qd = lane & 3;    // MMA fragment row group and quad position
@@ -503,10 +507,26 @@ __global__ void __launch_bounds__(kFThreads, 5) k_bgmv_fused(FusedBgmvArgs p)
     // the schedule (above) needs every item in the tables; else items in index order
     const bool sched = n_items <= L.n_tab;
     const int cid = (int)cluster_id_x();
-    for (int rnd = 0;; ++rnd) {
-        const int pos = rnd * n_cl + ((rnd & 1) ? n_cl - 1 - cid : cid);
-        if (pos >= n_items)
-            break;
+    // rank 0 of the cluster draws the next position (early, so that the atomic's round
+    // trip overlaps the shrink) and later hands it to every CTA of the cluster, which
+    // read it after the next cluster barrier
+    int drawn = -1;
+    auto draw = [&]() {
+        if (crank == 0 && tid == 0 && drawn < 0)
+            drawn = (int)atomicAdd(p.sched, 1u) + n_cl;
+    };
+    auto publish = [&]() {
+        if (crank == 0 && tid == 0) {
+            namespace cg = cooperative_groups;
+            cg::cluster_group cl = cg::this_cluster();
+#pragma unroll
+            for (int c = 0; c < kFC; ++c)
+                *cl.map_shared_rank(&s_next, c) = drawn;
+            drawn = -1;
+        }
+    };
+    int pos = cid;                  // the first round: the heaviest items, one per cluster
+    for (bool first_item = true; pos < n_items; first_item = false) {
         const int item = sched ? order[pos] : pos;
         // ---- the item's adapter, metadata and tokens (immutable inputs only)
         if (tid == 0) {
@@ -570,6 +590,11 @@ __global__ void __launch_bounds__(kFThreads, 5) k_bgmv_fused(FusedBgmvArgs p)
             }
             if (crank == 0 && tid == 0)
                 atomicOr(p.err, (uint32_t)LORA_ERR_BAD_ADAPTER);
+            draw();
+            publish();
+            cluster_arrive();
+            cluster_wait();
+            pos = s_next;
             __syncthreads();
             continue;
         }
@@ -613,6 +638,7 @@ __global__ void __launch_bounds__(kFThreads, 5) k_bgmv_fused(FusedBgmvArgs p)
             pdl_wait();   // from here on x, y and the workspace may be touched
             waited = true;
         }
+        draw();
         PHASE(11);
         if (L.staged) {
             // the item's y rows into shared memory: land during the shrink and the exchange
@@ -663,7 +689,7 @@ __global__ void __launch_bounds__(kFThreads, 5) k_bgmv_fused(FusedBgmvArgs p)
             pdl_wait();
             waited = true;
         }
-        if (s_bad && blockIdx.x == 0 && tid == 0 && rnd == 0)
+        if (s_bad && blockIdx.x == 0 && tid == 0 && first_item)
             atomicOr(p.err, (uint32_t)LORA_ERR_BAD_ADAPTER);
         PHASE(4);
         __syncthreads();
@@ -704,6 +730,7 @@ __global__ void __launch_bounds__(kFThreads, 5) k_bgmv_fused(FusedBgmvArgs p)
                 }
             }
         }
+        publish();          // lands before the barrier that ends this item
         cluster_arrive();   // our reads of the other CTAs' partials are done
         cp_async_wait_all();
         __syncthreads();
@@ -748,12 +775,21 @@ __global__ void __launch_bounds__(kFThreads, 5) k_bgmv_fused(FusedBgmvArgs p)
         cluster_wait();     // no CTA reuses its partials while another may still read them
         PHASE(8);
         first = false;
+        pos = s_next;
     }
     if (!waited) {
         pdl_trigger();
         pdl_wait();
         if (s_bad && blockIdx.x == 0 && tid == 0)
             atomicOr(p.err, (uint32_t)LORA_ERR_BAD_ADAPTER);
+    }
+    // the last cluster out puts the item counter back to zero for the next launch
+    if (crank == 0 && tid == 0) {
+        __threadfence();
+        if (atomicAdd(p.sched + 1, 1u) == (unsigned)n_cl - 1u) {
+            atomicExch(p.sched, 0u);
+            atomicExch(p.sched + 1, 0u);
+        }
     }
 }
 

@@ -421,6 +421,7 @@ lora_status lora_bgmv(const void *X, int64_t ldx, void *Y, int64_t ldy, const lo
         fa.Wk = fused_chunk(pool->d_in);
         fa.Wo = fused_chunk(pool->d_out);
         fa.err = &hdr->err;
+        fa.sched = hdr->sched;
         LORA_CUDA(launch_bgmv_fused(fa, s, pdl_enabled()));
         return LORA_OK;
     }

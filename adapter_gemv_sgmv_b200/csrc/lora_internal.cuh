@@ -25,7 +25,9 @@ struct WsHeader {
     uint32_t err;       // device error bits (lora_status values), sticky until lora_get_error
     int32_t n_seg;      // distinct adapters found by the grouping
     int32_t n_groups;   // work groups written by the plan kernel
-    int32_t pad[61];
+    uint32_t sched[2];  // decode kernel: next item position handed out, clusters finished
+                        // (both back to zero when the launch ends)
+    int32_t pad[59];
 };
 static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
 
@@ -212,6 +214,7 @@ struct FusedBgmvArgs {
     float scale;
     int32_t Wk, Wo;
     uint32_t *err;
+    uint32_t *sched;     // the workspace header's item counter pair
 };
 
 size_t fused_smem_bytes(int32_t N, int32_t n_adapters, int32_t max_rank, int32_t Wo);
