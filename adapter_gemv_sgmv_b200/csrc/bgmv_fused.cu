@@ -150,14 +150,21 @@ __device__ __forceinline__ bool adapter_ok(const PoolDev &P, int32_t a, int32_t 
     return true;
 }
 
-// Scheduling class of adapter a by rank (its L2 copy of the metadata is warm):
-// 3 for ranks 65-128 .. 0 for 8-16 and for an adapter that fails its checks.
-__device__ __forceinline__ int rank_class(const PoolDev &P, int a)
+// Scheduling class of a rank: 3 for ranks 65-128 .. 0 for 8-16 and for a rank that
+// fails the checks.
+__device__ __forceinline__ int rank_class(const PoolDev &P, int r)
 {
-    const int r = __ldg(P.rank + a);
     if (r < 8 || r > P.max_rank || (r & 7))
         return 0;
     return r <= 16 ? 0 : r <= 32 ? 1 : r <= 64 ? 2 : 3;
+}
+
+// The ranks of adapters a0 .. a0 + 7 (below e), eight loads in flight together.
+__device__ __forceinline__ void load_ranks8(const PoolDev &P, int a0, int e, int (&rk)[8])
+{
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+        rk[u] = a0 + u < e ? __ldg(P.rank + a0 + u) : 0;
 }
 
 // Shrink of one warp: NT rank tiles (8 ranks each, from rank tile nt0) over
@@ -432,11 +439,19 @@ __global__ void __launch_bounds__(kFThreads, 5) k_bgmv_fused(FusedBgmvArgs p)
         const int b = tid * per, e = min(n_ad, b + per);
         int local = 0;
         unsigned long long lcls = 0;
-        for (int a = b; a < e; ++a) {
-            const int gr = (ipre[a] + kFT - 1) / kFT;
-            local += gr;
-            if (gr)
-                lcls += (unsigned long long)gr << (16 * rank_class(p.pool, a));
+        for (int a0 = b; a0 < e; a0 += 8) {
+            int rk[8];
+            load_ranks8(p.pool, a0, e, rk);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int a = a0 + u;
+                if (a < e) {
+                    const int gr = (ipre[a] + kFT - 1) / kFT;
+                    local += gr;
+                    if (gr)
+                        lcls += (unsigned long long)gr << (16 * rank_class(p.pool, rk[u]));
+                }
+            }
         }
         int incl = local;
         unsigned long long icls = lcls;
@@ -478,20 +493,28 @@ __global__ void __launch_bounds__(kFThreads, 5) k_bgmv_fused(FusedBgmvArgs p)
         cbase[2] = (int)(tot >> 48);
         cbase[1] = cbase[2] + (int)((tot >> 32) & 0xFFFF);
         cbase[0] = cbase[1] + (int)((tot >> 16) & 0xFFFF);
-        for (int a = b; a < e; ++a) {
-            const int gr = (ipre[a] + kFT - 1) / kFT;
-            ipre[a] = run;
-            if (gr) {
-                const int c = rank_class(p.pool, a);
-                const int pos = cbase[c] + (int)((runc >> (16 * c)) & 0xFFFF);
-                for (int j = 0; j < gr && run + j < L.n_tab; ++j) {
-                    item_ad[run + j] = (int16_t)a;
-                    if (pos + j < L.n_tab)
-                        order[pos + j] = (int16_t)(run + j);
+        for (int a0 = b; a0 < e; a0 += 8) {
+            int rk[8];
+            load_ranks8(p.pool, a0, e, rk);       // L1 hits now
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int a = a0 + u;
+                if (a < e) {
+                    const int gr = (ipre[a] + kFT - 1) / kFT;
+                    ipre[a] = run;
+                    if (gr) {
+                        const int c = rank_class(p.pool, rk[u]);
+                        const int pos = cbase[c] + (int)((runc >> (16 * c)) & 0xFFFF);
+                        for (int j = 0; j < gr && run + j < L.n_tab; ++j) {
+                            item_ad[run + j] = (int16_t)a;
+                            if (pos + j < L.n_tab)
+                                order[pos + j] = (int16_t)(run + j);
+                        }
+                        runc += (unsigned long long)gr << (16 * c);
+                    }
+                    run += gr;
                 }
-                runc += (unsigned long long)gr << (16 * c);
             }
-            run += gr;
         }
         if (tid == 0)
             ipre[n_ad] = sm_scan[kFWarps];
