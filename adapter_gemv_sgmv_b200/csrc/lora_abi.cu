@@ -628,8 +628,10 @@ lora_status lora_sgmv_apply_proj(const void *X, int64_t ldx, void *const *Y, con
         tc = tc_encode_y(te[p], Y[p], N, pools[p].d_out, ldy[p]);
     }
     LORA_CUDA(run_proj_shrinks(tc, ta, X, ldx, V, ldv, pools, n_proj, vcol, seg_off, seg_ad, n_seg, N, L, ws, s));
-    for (int p = 0; p < n_proj; ++p) {
-        if (tc) {
+    if (tc) {
+        // every projection's expand in one launch, the GPU's CTAs split among them
+        int kk = 0;
+        for (int p = 0; p < n_proj; ++p) {
             TcArgs &e = te[p];
             e.mode = kModeSgmv;
             e.groups = groups;
@@ -644,8 +646,13 @@ lora_status lora_sgmv_apply_proj(const void *X, int64_t ldx, void *const *Y, con
             e.Y = static_cast<__nv_bfloat16 *>(Y[p]);
             e.ldy = ldy[p];
             e.err = &hdr->err;
-            LORA_CUDA(launch_tc_expand(e, pools[p].max_rank, s));
-        } else {
+            kk = pools[p].max_rank > kk ? pools[p].max_rank : kk;
+        }
+        LORA_CUDA(launch_tc_expand_multi(te, n_proj, kk, s));
+        return LORA_OK;
+    }
+    for (int p = 0; p < n_proj; ++p) {
+        {
             ExpandArgs ea = {};
             ea.Y = static_cast<__nv_bfloat16 *>(Y[p]);
             ea.ldy = ldy[p];

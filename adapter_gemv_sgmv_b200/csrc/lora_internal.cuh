@@ -282,6 +282,8 @@ bool tc_encode_b(TcArgs &a, const void *B, int64_t B_elems);
 cudaError_t launch_tc_shrink(const TcArgs &a, int max_tiles, int kk, cudaStream_t s);
 // kk: the largest stacked rank of any item (max_rank, or max_ads * max_rank)
 cudaError_t launch_tc_expand(const TcArgs &a, int kk, cudaStream_t s);
+// n expands over the same tiles in one launch (kk: the largest stacked rank of any)
+cudaError_t launch_tc_expand_multi(const TcArgs *a, int n, int kk, cudaStream_t s);
 bool tc_enabled();
 
 // ------------------------------------------- projection + LoRA delta (tcgen05)

@@ -451,7 +451,9 @@ constexpr int kY = kBM * kBN * 2;                  // y: 128 rows x 128 outputs 
 constexpr int kMaxYStages = 6;
 constexpr int kStaging = kEpiWarps * 1024;         // per epilogue warp: 32 rows x 16 outputs of bf16
 
-__global__ void __launch_bounds__(kExpandThreads, 1) k_tc_expand(const __grid_constant__ TcArgs p)
+// The expand of one CTA: block bid of G working on p's units.  p must refer to
+// kernel-parameter memory (its tensor maps are read by the copy engine).
+__device__ __forceinline__ void tc_expand_cta(const TcArgs &p, int bid, int G)
 {
     extern __shared__ __align__(1024) unsigned char sm_dyn[];
     unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(sm_dyn) + 1023) & ~(uintptr_t)1023);
@@ -471,7 +473,6 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_tc_expand(const __grid_co
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int d_out = p.pool.d_out;
     const int n_ns = (d_out + kBN - 1) / kBN;           // output slices
-    const int G = gridDim.x;
     const int n_ys = p.e_ystages;
     const int szB = p.e_natoms * kAtom;                 // one B stage (and each half of V)
     unsigned char *const smV = sm;                      // V high parts, then V low parts
@@ -507,7 +508,7 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_tc_expand(const __grid_co
     pdl_wait();                                  // tiles and V of the previous kernels are complete
     pdl_trigger();
     const int64_t n_units = (int64_t)p.hdr->n_groups * n_ns;
-    const int64_t u0 = (int64_t)blockIdx.x * n_units / G, u1 = (int64_t)(blockIdx.x + 1) * n_units / G;
+    const int64_t u0 = (int64_t)bid * n_units / G, u1 = (int64_t)(bid + 1) * n_units / G;
     int y_issued = 0, b_issued = 0;              // producer: y and B stage fills issued
 
     if (warp == 0) {
@@ -865,6 +866,29 @@ done:
     }
 }
 
+__global__ void __launch_bounds__(kExpandThreads, 1) k_tc_expand(const __grid_constant__ TcArgs p)
+{
+    tc_expand_cta(p, blockIdx.x, gridDim.x);
+}
+
+// The expands of projections that share V's tiles (q, k, v of one x) in one launch:
+// CTAs [cta0[i], cta0[i + 1]) take projection i's units, the split proportional to
+// each projection's output slices, so that the small projections no longer run
+// alone on the whole GPU with a few units per CTA.
+struct TcExpandMulti {
+    TcArgs a[kMaxProj];
+    int32_t n;
+    int32_t cta0[kMaxProj + 1];
+};
+
+__global__ void __launch_bounds__(kExpandThreads, 1) k_tc_expand_multi(const __grid_constant__ TcExpandMulti m)
+{
+    int i = 0;
+    while (i + 1 < m.n && (int)blockIdx.x >= m.cta0[i + 1])
+        ++i;
+    tc_expand_cta(m.a[i], (int)blockIdx.x - m.cta0[i], m.cta0[i + 1] - m.cta0[i]);
+}
+
 // attr_set: this kernel's per-device "shared-memory opt-in done" flags (one
 // array per kernel: the kernels share a type, so they cannot share the flags)
 cudaError_t launch_tc(void (*kernel)(TcArgs), bool *attr_set, const TcArgs &a, int threads, int smem, int grid,
@@ -1015,6 +1039,75 @@ cudaError_t launch_tc_expand(const TcArgs &args, int kk, cudaStream_t s)
     }
     bool done = true;
     return launch_tc(k_tc_expand, &done, a, kExpandThreads, smem, sm_count(), s);
+}
+
+cudaError_t launch_tc_expand_multi(const TcArgs *args, int n, int kk, cudaStream_t s)
+{
+    constexpr int kTileCost = 4;     // per-tile overhead of a CTA, in output slices (measured: 0 and 8 slower)
+    if (n < 1 || n > kMaxProj)
+        return cudaErrorInvalidValue;
+    static bool attr_set[64] = {};
+    int dev = 0, optin = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    if ((e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess)
+        return e;
+    cudaFuncAttributes fa;
+    if ((e = cudaFuncGetAttributes(&fa, k_tc_expand_multi)) != cudaSuccess)
+        return e;
+    TcExpandMulti m = {};
+    m.n = n;
+    // one shared-memory layout for all: the largest stacked rank of any projection
+    const int natoms = kk > 64 ? 2 : 1;
+    const int fixed = (2 + kExpandBStages) * natoms * kAtom + kStaging + 1024;
+    const int room = optin - (int)fa.sharedSizeBytes - fixed;
+    const int ys = room / kY < kMaxYStages ? room / kY : kMaxYStages;
+    if (ys < 2)
+        return cudaErrorInvalidConfiguration;
+    const int smem = fixed + ys * kY;
+    const int G = sm_count();
+    int64_t slices = 0;
+    for (int i = 0; i < n; ++i) {
+        m.a[i] = args[i];
+        m.a[i].wait_ns = wait_bound_ns();
+        m.a[i].test_stall = test_stall_mode();
+        m.a[i].e_natoms = natoms;
+        m.a[i].e_ystages = ys;
+        slices += (m.a[i].pool.d_out + kBN - 1) / kBN + kTileCost;
+    }
+    if (G < n)
+        return cudaErrorInvalidConfiguration;
+    // CTAs in proportion to output slices (plus a per-tile cost: V staged once per
+    // tile and the first unit's latency weigh most on projections with few slices),
+    // at least one each
+    int64_t acc = 0;
+    m.cta0[0] = 0;
+    for (int i = 0; i < n; ++i) {
+        acc += (m.a[i].pool.d_out + kBN - 1) / kBN + kTileCost;
+        int c = (int)((acc * G + slices / 2) / slices);
+        c = c < m.cta0[i] + 1 ? m.cta0[i] + 1 : c;
+        c = c > G - (n - 1 - i) ? G - (n - 1 - i) : c;
+        m.cta0[i + 1] = c;
+    }
+    m.cta0[n] = G;
+    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+        if ((e = cudaFuncSetAttribute(k_tc_expand_multi, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      optin - (int)fa.sharedSizeBytes)) != cudaSuccess)
+            return e;
+        attr_set[dev] = true;
+    }
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(G);
+    cfg.blockDim = dim3(kExpandThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl_enabled() ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, k_tc_expand_multi, m);
 }
 
 }  // namespace lora

@@ -251,8 +251,9 @@ def shrink_proj_passes(max_ranks, limit=256) -> int:
 def launches_per_step(wl) -> int:
     import adapter_gemv_sgmv_b200 as L
     if wl.desc.get("op") == "sgmv_proj":
-        # lora_sgmv_apply_proj on long segments: one plan, the stacked shrinks, one expand each
-        return 1 + shrink_proj_passes([c.pool.max_rank for c in wl.calls]) + len(wl.calls)
+        # lora_sgmv_apply_proj on long segments: one plan, the stacked shrinks, one expand
+        # launch for all the projections
+        return 1 + shrink_proj_passes([c.pool.max_rank for c in wl.calls]) + 1
     return sum(launches_per_call(c) for c in wl.calls)
 
 

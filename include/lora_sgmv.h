@@ -226,9 +226,10 @@ LORA_API lora_status lora_sgmv_shrink_proj(const void *X, int64_t ldx, float *V,
  * (the shrink of lora_sgmv_shrink_proj, then every projection's expand):
  *   Y_p[n] += scale[p] * B_p[a] (A_p[a] X[n]),  a = seg_ad[k], seg_off[k] <= n < seg_off[k+1],
  * for p < n_proj.  One plan serves the shrink and all the expands, and the
- * intermediate stays in the workspace: 1 + (tensor-core shrink launches) +
- * n_proj kernels on the tensor-core path (long segments), 1 + 2 n_proj on the
- * CUDA-core path.  Y, ldy, scale: HOST arrays of n_proj entries (Y[p] a device
+ * intermediate stays in the workspace: 1 + (tensor-core shrink launches) + 1
+ * kernels on the tensor-core path (long segments: every projection's expand runs
+ * in one launch, the GPU's CTAs split among the projections in proportion to
+ * their outputs), 1 + 2 n_proj on the CUDA-core path.  Y, ldy, scale: HOST arrays of n_proj entries (Y[p] a device
  * bf16 [N, ldy[p]] matrix, ldy[p] >= pools[p].d_out).  Pools and segments as
  * in lora_sgmv_shrink_proj.  Workspace: lora_workspace_size(LORA_OP_APPLY_PROJ,
  * N, n_adapters, d_in, 0, sum of the pools' max_rank, n_seg, 0).

@@ -92,7 +92,7 @@ def test_bench_counts_the_fused_calls():
     assert bench.shrink_proj_passes([16, 16, 16, 16]) == 1
     wl = make_workload("prefill_qkv", n_req=3, len_range=(200, 300), d_in=64, d_outs=(64, 16, 16), rank=8,
                        n_adapters=5)
-    assert bench.launches_per_step(wl) == 1 + 1 + 3              # one plan, one shrink, 3 expands
+    assert bench.launches_per_step(wl) == 1 + 1 + 1              # one plan, one shrink, one expand launch
     wl = make_workload("prefill_linear_up", n_req=3, len_range=(4, 9), d_in=64, d_out=48, rank=16,
                        n_adapters=5)
     assert bench._is_linear(wl.calls[0]) and bench.launches_per_step(wl) == 3
