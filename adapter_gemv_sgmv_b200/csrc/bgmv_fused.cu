@@ -200,31 +200,51 @@ __device__ __forceinline__ void shrink_tiles(const __nv_bfloat16 *Aa, int d_in, 
     }
 }
 
+// Position (in bf16 elements) of V[t][j] (token t < 16, rank j) in the fragment-
+// ordered V buffer, hi part (the lo part follows: +512 per 32-rank block, +256 for
+// ranks <= 16).  For an m16n8k16 A operand, lane (g, qd) holds rows g and g + 8 at
+// k-slot pairs {2qd, 2qd+1} and {2qd+8, 2qd+9}; inside a 32-rank block quad qd
+// owns ranks 8qd .. 8qd+7 (pairs 0, 1 for MMA 0 and pairs 2, 3 for MMA 1), and for
+// ranks <= 16 ranks 4qd .. 4qd+3 (pairs 0, 1 of the single MMA).  Each quad is
+// stored as the four registers the MMA takes: (row g, pair p), (row g+8, pair p),
+// (row g, pair p+1), (row g+8, pair p+1), so one 16-byte load yields an operand.
+__device__ __forceinline__ int vfrag_index(int t, int j, bool r16)
+{
+    const int g = t & 7, hi8 = t >> 3;
+    if (r16) {
+        const int qd = j >> 2, w = j & 3;
+        return (g * 4 + qd) * 8 + (((w >> 1) << 1) | hi8) * 2 + (w & 1);
+    }
+    const int kb = j >> 5, jj = j & 31, qd = jj >> 3, w = jj & 7, pair = w >> 1;
+    const int m = pair >> 1;
+    return ((kb * 4 + m) * 32 + g * 4 + qd) * 8 + (((pair & 1) << 1) | hi8) * 2 + (w & 1);
+}
+
 // Expand of one warp over its output tiles ot = warp, warp + nw, ... < n_ot
 // (8 outputs each, from output o0): Y += s (V_hi + V_lo) B^T with NKB
 // 32-rank blocks; a batch's B fragments and y values are all requested
 // before its MMAs, and the V fragments are read from shared memory once.
+// vq: V_hi and V_lo in fragment order (vfrag_index): quad vq[((kb * 2 + hl) * 2
+// + m) * 32 + lane] is the A operand of MMA m of block kb as it stands.
 // ST: B and y come from the staged copies in shared memory (bst: [Wo][r] from
 // output o0; yst: [kFT][Wo]), else from global memory.
 template <int NKB, bool ST>
 __device__ __forceinline__ void expand_tiles(const __nv_bfloat16 *Ba, int r, int o0, int n_ot, int warp, int nw,
-                                             const __nv_bfloat16 *vhi, const __nv_bfloat16 *vlo, int vs, int g,
-                                             int qd, __nv_bfloat16 *y0row, __nv_bfloat16 *y1row, bool row0,
-                                             bool row1, float sc, const __nv_bfloat16 *bst,
-                                             const __nv_bfloat16 *yst, int Wo)
+                                             const uint4 *vq, int lane, int g, int qd, __nv_bfloat16 *y0row,
+                                             __nv_bfloat16 *y1row, bool row0, bool row1, float sc,
+                                             const __nv_bfloat16 *bst, const __nv_bfloat16 *yst, int Wo)
 {
     constexpr int TPB = ST ? 16 : (NKB == 1 ? 8 : NKB == 2 ? 4 : 2);   // tiles per batch
     constexpr bool HOIST = NKB <= 2;                                  // keep V fragments in registers
-    uint4 h0[HOIST ? NKB : 1], h1[HOIST ? NKB : 1], l0[HOIST ? NKB : 1], l1[HOIST ? NKB : 1];
+    uint4 qv[HOIST ? NKB : 1][2][2];     // [kb][hi, lo][MMA]
     if (HOIST) {
 #pragma unroll
-        for (int kb = 0; kb < (HOIST ? NKB : 1); ++kb) {
-            const int kc = kb * 32 + qd * 8;
-            h0[kb] = *reinterpret_cast<const uint4 *>(vhi + g * vs + kc);
-            h1[kb] = *reinterpret_cast<const uint4 *>(vhi + (g + 8) * vs + kc);
-            l0[kb] = *reinterpret_cast<const uint4 *>(vlo + g * vs + kc);
-            l1[kb] = *reinterpret_cast<const uint4 *>(vlo + (g + 8) * vs + kc);
-        }
+        for (int kb = 0; kb < (HOIST ? NKB : 1); ++kb)
+#pragma unroll
+            for (int hl = 0; hl < 2; ++hl)
+#pragma unroll
+                for (int m = 0; m < 2; ++m)
+                    qv[kb][hl][m] = vq[((kb * 2 + hl) * 2 + m) * 32 + lane];
     }
     for (int ot0 = warp; ot0 < n_ot; ot0 += TPB * nw) {
         uint4 bw[ST ? 1 : TPB][NKB];
@@ -272,23 +292,22 @@ __device__ __forceinline__ void expand_tiles(const __nv_bfloat16 *Ba, int r, int
                 float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int kb = 0; kb < NKB; ++kb) {
-                    uint4 a0, a1, c0, c1;
+                    uint4 h0, h1, l0, l1;     // hi / lo quads of the two MMAs
                     if (HOIST) {
-                        a0 = h0[HOIST ? kb : 0];
-                        a1 = h1[HOIST ? kb : 0];
-                        c0 = l0[HOIST ? kb : 0];
-                        c1 = l1[HOIST ? kb : 0];
+                        h0 = qv[HOIST ? kb : 0][0][0];
+                        h1 = qv[HOIST ? kb : 0][0][1];
+                        l0 = qv[HOIST ? kb : 0][1][0];
+                        l1 = qv[HOIST ? kb : 0][1][1];
                     } else {
-                        const int kc = kb * 32 + qd * 8;
-                        a0 = *reinterpret_cast<const uint4 *>(vhi + g * vs + kc);
-                        a1 = *reinterpret_cast<const uint4 *>(vhi + (g + 8) * vs + kc);
-                        c0 = *reinterpret_cast<const uint4 *>(vlo + g * vs + kc);
-                        c1 = *reinterpret_cast<const uint4 *>(vlo + (g + 8) * vs + kc);
+                        h0 = vq[(kb * 4 + 0) * 32 + lane];
+                        h1 = vq[(kb * 4 + 1) * 32 + lane];
+                        l0 = vq[(kb * 4 + 2) * 32 + lane];
+                        l1 = vq[(kb * 4 + 3) * 32 + lane];
                     }
-                    mma16816(d, a0.x, a1.x, a0.y, a1.y, bfr[kb].x, bfr[kb].y);
-                    mma16816(d, c0.x, c1.x, c0.y, c1.y, bfr[kb].x, bfr[kb].y);
-                    mma16816(d, a0.z, a1.z, a0.w, a1.w, bfr[kb].z, bfr[kb].w);
-                    mma16816(d, c0.z, c1.z, c0.w, c1.w, bfr[kb].z, bfr[kb].w);
+                    mma16816(d, h0.x, h0.y, h0.z, h0.w, bfr[kb].x, bfr[kb].y);
+                    mma16816(d, l0.x, l0.y, l0.z, l0.w, bfr[kb].x, bfr[kb].y);
+                    mma16816(d, h1.x, h1.y, h1.z, h1.w, bfr[kb].z, bfr[kb].w);
+                    mma16816(d, l1.x, l1.y, l1.z, l1.w, bfr[kb].z, bfr[kb].w);
                 }
                 // D fragment: tokens g, g+8; outputs ob + 2qd, ob + 2qd + 1
                 const int o = o0 + ol + 2 * qd;
@@ -315,20 +334,16 @@ __device__ __forceinline__ void expand_tiles(const __nv_bfloat16 *Ba, int r, int
 // V_hi and V_lo halves.
 template <bool ST>
 __device__ __forceinline__ void expand_tiles16(const __nv_bfloat16 *Ba, int r, int o0, int n_ot, int warp, int nw,
-                                               const __nv_bfloat16 *vhi, const __nv_bfloat16 *vlo, int vs, int g,
-                                               int qd, __nv_bfloat16 *y0row, __nv_bfloat16 *y1row, bool row0,
-                                               bool row1, float sc, const __nv_bfloat16 *bst,
-                                               const __nv_bfloat16 *yst, int Wo)
+                                               const uint4 *vq, int lane, int g, int qd, __nv_bfloat16 *y0row,
+                                               __nv_bfloat16 *y1row, bool row0, bool row1, float sc,
+                                               const __nv_bfloat16 *bst, const __nv_bfloat16 *yst, int Wo)
 {
     // global operands: a batch's B fragments and y values are requested before its MMAs;
     // staged operands (shared memory) are read tile by tile
     constexpr int TPB = ST ? 1 : 8;
     const int kc = qd * 4;
     const bool kin = kc < r;
-    const uint2 h0 = *reinterpret_cast<const uint2 *>(vhi + g * vs + kc);
-    const uint2 h1 = *reinterpret_cast<const uint2 *>(vhi + (g + 8) * vs + kc);
-    const uint2 l0 = *reinterpret_cast<const uint2 *>(vlo + g * vs + kc);
-    const uint2 l1 = *reinterpret_cast<const uint2 *>(vlo + (g + 8) * vs + kc);
+    const uint4 qh = vq[lane], ql = vq[32 + lane];     // hi / lo quads (ranks <= 16 order)
     const __nv_bfloat162 z = __floats2bfloat162_rn(0.f, 0.f);
     for (int ot0 = warp; ot0 < n_ot; ot0 += TPB * nw) {
         uint2 bw[TPB];
@@ -354,8 +369,8 @@ __device__ __forceinline__ void expand_tiles16(const __nv_bfloat16 *Ba, int r, i
             const int ot = ot0 + t * nw;
             if (ot < n_ot) {
                 float d[4] = {0.f, 0.f, 0.f, 0.f};
-                mma16816(d, h0.x, h1.x, h0.y, h1.y, bw[t].x, bw[t].y);
-                mma16816(d, l0.x, l1.x, l0.y, l1.y, bw[t].x, bw[t].y);
+                mma16816(d, qh.x, qh.y, qh.z, qh.w, bw[t].x, bw[t].y);
+                mma16816(d, ql.x, ql.y, ql.z, ql.w, bw[t].x, bw[t].y);
                 const int o = o0 + ot * 8 + 2 * qd;
                 if (row0) {
                     const float2 y = __bfloat1622float2(ya[t]);
@@ -376,16 +391,15 @@ __global__ void __launch_bounds__(kFThreads, 5) k_bgmv_fused(FusedBgmvArgs p)
 {
     extern __shared__ __align__(16) unsigned char sm_raw[];
     const FusedSmem L = fused_smem_layout(p.N, p.pool.n_adapters, p.pool.max_rank, p.Wo);
-    const int vs = L.vs;
     int16_t *item_ad = reinterpret_cast<int16_t *>(sm_raw + L.items);   // adapter of items < L.n_tab
     int16_t *order = reinterpret_cast<int16_t *>(sm_raw + L.order);    // item at each schedule position
     const int mr = p.pool.max_rank < kMaxRank ? p.pool.max_rank : kMaxRank;
     int32_t *ids_s = reinterpret_cast<int32_t *>(sm_raw + L.ids);
     int32_t *ipre = reinterpret_cast<int32_t *>(sm_raw + L.cnt);    // [n_ad + 1]
     float *vpart = reinterpret_cast<float *>(sm_raw + L.vpart);     // [max_rank][kFT], read by the cluster
-    // V split into bf16 hi and lo parts, token-major: [kFT][vs] each
-    __nv_bfloat16 *vhi = reinterpret_cast<__nv_bfloat16 *>(sm_raw + L.vsum);
-    __nv_bfloat16 *vlo = vhi + kFT * vs;
+    // V split into bf16 hi and lo parts, in MMA fragment order (vfrag_index)
+    __nv_bfloat16 *vfr = reinterpret_cast<__nv_bfloat16 *>(sm_raw + L.vsum);
+    const uint4 *vq = reinterpret_cast<const uint4 *>(sm_raw + L.vsum);
     // staged (when L.staged): this CTA's B chunk [Wo][r] and the item's y rows [kFT][Wo]
     __nv_bfloat16 *bst = reinterpret_cast<__nv_bfloat16 *>(sm_raw + L.bst);
     __nv_bfloat16 *yst = reinterpret_cast<__nv_bfloat16 *>(sm_raw + L.yst);
@@ -747,8 +761,11 @@ __global__ void __launch_bounds__(kFThreads, 5) k_bgmv_fused(FusedBgmvArgs p)
                     if (idx < kFT * rp) {
                         const int t = idx & (kFT - 1), j = idx >> 4;
                         const __nv_bfloat16 h = __float2bfloat16_rn(s[u]);
-                        vhi[t * vs + j] = h;
-                        vlo[t * vs + j] = __float2bfloat16_rn(s[u] - __bfloat162float(h));
+                        if (r > 16 || j < 16) {
+                            const int e = vfrag_index(t, j, r <= 16);
+                            vfr[e] = h;
+                            vfr[e + (r <= 16 ? 256 : 512)] = __float2bfloat16_rn(s[u] - __bfloat162float(h));
+                        }
                     }
                 }
             }
@@ -766,14 +783,14 @@ __global__ void __launch_bounds__(kFThreads, 5) k_bgmv_fused(FusedBgmvArgs p)
             __nv_bfloat16 *y0row = p.Y + (int64_t)(row0 ? tok[g] : 0) * p.ldy;
             __nv_bfloat16 *y1row = p.Y + (int64_t)(row1 ? tok[g + 8] : 0) * p.ldy;
 #define LORA_EXPAND(NKB, ST)                                                                             \
-    expand_tiles<NKB, ST>(Ba, r, o0, n_ot, warp, kFWarps, vhi, vlo, vs, g, qd, y0row, y1row, row0, row1, p.scale, \
+    expand_tiles<NKB, ST>(Ba, r, o0, n_ot, warp, kFWarps, vq, lane, g, qd, y0row, y1row, row0, row1, p.scale, \
                           bst, yst, p.Wo)
             if (r <= 16) {
                 if (L.staged)
-                    expand_tiles16<true>(Ba, r, o0, n_ot, warp, kFWarps, vhi, vlo, vs, g, qd, y0row, y1row, row0,
+                    expand_tiles16<true>(Ba, r, o0, n_ot, warp, kFWarps, vq, lane, g, qd, y0row, y1row, row0,
                                          row1, p.scale, bst, yst, p.Wo);
                 else
-                    expand_tiles16<false>(Ba, r, o0, n_ot, warp, kFWarps, vhi, vlo, vs, g, qd, y0row, y1row, row0,
+                    expand_tiles16<false>(Ba, r, o0, n_ot, warp, kFWarps, vq, lane, g, qd, y0row, y1row, row0,
                                           row1, p.scale, bst, yst, p.Wo);
             } else if (L.staged) {
                 switch ((r + 31) >> 5) {
