@@ -53,13 +53,16 @@ namespace lora {
 namespace {
 
 // Read-only 16-byte load that does not allocate in L1 (weights are used once
-// per CTA).  Not volatile: the compiler may batch independent loads.
-__device__ __forceinline__ uint4 ld_stream(const void *p)
+// per CTA), or zeros when ok is false.  The predicate is inside the asm so that
+// the compiler needs no branch around it.  Not volatile: the compiler may batch
+// independent loads.
+__device__ __forceinline__ uint4 ld_stream(const void *p, bool ok)
 {
-    uint4 r;
-    asm("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-        : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-        : "l"(p));
+    uint4 r = make_uint4(0, 0, 0, 0);
+    asm("{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %5, 0;\n\t"
+        "@q ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];\n\t}"
+        : "+r"(r.x), "+r"(r.y), "+r"(r.z), "+r"(r.w)
+        : "l"(p), "r"((int)ok));
     return r;
 }
 
@@ -184,7 +187,7 @@ __device__ __forceinline__ void shrink_tiles(const __nv_bfloat16 *Aa, int d_in, 
             const bool ok = bb + k < b1 && col < k1;
 #pragma unroll
             for (int i = 0; i < NT; ++i)
-                aw[k][i] = ok ? ld_stream(Aa + (int64_t)((nt0 + i) * 8 + g) * d_in + col) : make_uint4(0, 0, 0, 0);
+                aw[k][i] = ld_stream(Aa + (int64_t)((nt0 + i) * 8 + g) * d_in + col, ok);
             xa[k] = (ok && row0) ? __ldg(reinterpret_cast<const uint4 *>(x0 + col)) : make_uint4(0, 0, 0, 0);
             xb[k] = (ok && row1) ? __ldg(reinterpret_cast<const uint4 *>(x1 + col)) : make_uint4(0, 0, 0, 0);
         }
@@ -259,7 +262,7 @@ __device__ __forceinline__ void expand_tiles(const __nv_bfloat16 *Ba, int r, int
 #pragma unroll
                 for (int kb = 0; kb < NKB; ++kb) {
                     const int kc = kb * 32 + qd * 8;   // r and kc are multiples of 8
-                    bw[ST ? 0 : t][kb] = (ok && kc < r) ? ld_stream(brow + kc) : make_uint4(0, 0, 0, 0);
+                    bw[ST ? 0 : t][kb] = ld_stream(brow + kc, ok && kc < r);
                 }
                 const __nv_bfloat162 z = __floats2bfloat162_rn(0.f, 0.f);
                 ya[ST ? 0 : t] = (ok && row0) ? *reinterpret_cast<const __nv_bfloat162 *>(y0row + ob + 2 * qd) : z;
