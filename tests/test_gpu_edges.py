@@ -105,6 +105,28 @@ def test_ragged_bgmv_with_no_adapter_rows():
     assert np.array_equal(got[ids == -1], widen(Y0)[ids == -1])
 
 
+@pytest.mark.parametrize("d_out", [136, 4096])
+def test_bgmv_every_rank(d_out):
+    """Every rank the pool allows (8 .. 128 in steps of 8: one to four 32-rank blocks,
+    the k16 path at ranks <= 16), with adapters used by 1 to 40 tokens (several
+    16-token items per adapter), on the staged path (small d_out) and the unstaged one
+    (d_out = 4096: the B chunk per CTA exceeds the shared-memory stage)."""
+    rng = np.random.default_rng(7 + d_out)
+    ranks = list(range(8, 129, 8))
+    hp = rand_host_pool(rng, ranks, 520, d_out)
+    n_ad = len(ranks)
+    counts = np.concatenate([[40, 17, 16], rng.integers(1, 6, n_ad - 3)])
+    ids = np.concatenate([np.full(c, a, np.int32) for a, c in enumerate(counts)] + [np.full(5, -1, np.int32)])
+    ids = ids[rng.permutation(ids.size)]
+    N = ids.size
+    X = rand_x(rng, N, 520)
+    Y0 = rand_x(rng, N, d_out)
+    Y = dev_bf16(Y0)
+    ws = L.lora_bgmv(dev_bf16(X), Y, DevPool(hp), _i32(ids), 0.75)
+    assert L.lora_get_error(ws) == 0
+    check_parity(_f64(Y), widen(Y0) + oracle.bgmv_delta(X, hp, ids, 0.75), f"bgmv every rank, d_out {d_out}")
+
+
 def test_ragged_sgmv_empty_segments_and_uncovered_rows():
     rng, hp, X, Y0 = _ragged_case(1)
     seg_off = np.array([3, 3, 10, 11, 30, 30], np.int32)   # rows 0-2 and 30-36 outside
