@@ -35,13 +35,18 @@
 //   tiles and/or the chunk, reduced into shared memory;
 // * the cluster sums the kFC partials through distributed shared memory
 //   (fixed order: deterministic) and splits V into bf16 hi + lo parts, so the
-//   expand MMAs see V to ~16 significant bits instead of bf16's 8;
+//   expand MMAs see V to ~16 significant bits instead of bf16's 8; V is kept
+//   in MMA fragment order, so a lane's 16-byte read is one A operand as the
+//   MMA takes it;
 // * expand: CTA c owns a d_out chunk; its warps walk 8-output tiles,
 //   Y_tile += s * (V_hi + V_lo) B[tile]^T, and update y in place;
-// * the item's y rows are bulk-prefetched into L2 early; the grouping and
-//   the first A fragments are loaded before griddepcontrol.wait
-//   (programmatic dependent launch), i.e. while the previous kernel on the
-//   stream is still finishing -- they only read immutable inputs.
+// * when a CTA's B chunk and the item's y rows fit 16 KB each (decode shapes)
+//   both are copied to shared memory as soon as the item is known; otherwise
+//   the CTA's A rows are requested into L2 line by line before the shrink; the
+//   grouping, the item metadata and those requests come before
+//   griddepcontrol.wait (programmatic dependent launch), i.e. while the
+//   previous kernel on the stream is still finishing -- they only read
+//   immutable inputs.
 
 #include <cooperative_groups.h>
 
